@@ -1,0 +1,213 @@
+/*
+ * maglev.h -- C ABI of the B200 (sm_100a) implementation of Maglev's injected
+ * sliding-window attention ("Maglev: Sliding Recurrent Memory", arXiv 2608.02870).
+ *
+ * Page citations: [rainbus] = paper.rainbus.top, sections 前置知识 (SWA, KV cache,
+ * RoPE), 研究动机 (the interface p(x_{t+1}, m_t | x_{t-W+1:t}, M_{t-1})) and
+ * 方法步骤详情 (every formula); [gist] = gist.science, section Inferentiemechanisme.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Ownership: every tensor argument is a caller-owned DEVICE pointer (any
+ *    allocator). The library never allocates device memory and never frees
+ *    the caller's. Scratch memory is passed in by the caller; its size comes
+ *    from the matching *_bytes() query.
+ *  - Layout: dense, row-major, innermost index last, 16-byte aligned base.
+ *    Token-major activations: [B, T, H, hd] (equivalently [B, T, D], D = H*hd).
+ *  - dtype: MAGLEV_BF16 (bf16 storage, fp32 accumulation; tensor-core path) or
+ *    MAGLEV_F32 (fp32 storage and arithmetic on CUDA cores). Gate logits, LSE,
+ *    gate gradients and the loss are always fp32.
+ *  - Streams: `stream` is a cudaStream_t (NULL = legacy default stream). Every
+ *    call only enqueues work; none synchronises the device.
+ *  - Errors: arguments are validated on the host before any launch. A call
+ *    returns MAGLEV_OK, or an error code with nothing enqueued (INVALID_ARG,
+ *    UNSUPPORTED) or after a CUDA launch error (CUDA). maglev_last_error()
+ *    returns the message of the calling thread's last failure. Kernels that
+ *    wait on asynchronous copies bound every wait by desc->spin_limit polls;
+ *    on expiry they record MAGLEV_ERR_TIMEOUT in a device status word, abandon
+ *    the tile and return; read it with maglev_device_status().
+ *  - Empty problems (B == 0 or T == 0, rows == 0) are valid and enqueue nothing.
+ */
+#ifndef MAGLEV_H
+#define MAGLEV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MAGLEV_OK = 0,
+  MAGLEV_ERR_INVALID_ARG = 1,
+  MAGLEV_ERR_UNSUPPORTED = 2,
+  MAGLEV_ERR_CUDA = 3,
+  MAGLEV_ERR_TIMEOUT = 4
+} maglev_status;
+
+typedef enum { MAGLEV_F32 = 0, MAGLEV_BF16 = 1 } maglev_dtype;
+
+/* Shapes and options of one injected sliding-window attention layer.
+ * B batch, T sequence length, H heads, hd head dim (64 or 128), d_mem memory
+ * width, window W >= 1 (keys j in [i-W+1, i]; W >= T is full causal attention),
+ * rope_base (10000 in the d20 model), rms_eps (1e-6), inject (0: plain SWA --
+ * memory arguments may be NULL), pos0 (absolute position of row 0), dtype,
+ * spin_limit (bound on each in-kernel wait, 0 = library default). */
+typedef struct {
+  int B, T, H, hd, d_mem, window;
+  float rope_base, rms_eps;
+  int inject;
+  int pos0;
+  int dtype;
+  int64_t spin_limit;
+} maglev_swa_desc;
+
+/* Shapes of one recurrent decode layer: B sequences, H heads, hd, d_mem,
+ * window W = ring length. */
+typedef struct {
+  int B, H, hd, d_mem, window;
+  float rope_base, rms_eps;
+  int inject;
+  int dtype;
+  int64_t spin_limit;
+} maglev_decode_desc;
+
+/* Library version string (static storage). */
+const char* maglev_version(void);
+
+/* Tracing. maglev_launch_count() returns the number of kernels this library
+ * has launched in the process so far (all threads, all devices).
+ * maglev_profile_enable(1) brackets every later launch with CUDA events
+ * recorded on the launch's own stream; maglev_profile_report() waits for the
+ * recorded events, writes one line "name kernels milliseconds" per traced
+ * launch into buf (NUL-terminated, truncated to n bytes), clears the record
+ * and returns the full text length. Tracing is off by default. */
+long long maglev_launch_count(void);
+void maglev_profile_enable(int on);
+size_t maglev_profile_report(char* buf, size_t n);
+
+/* Copies the calling thread's last error message into buf (NUL-terminated,
+ * truncated to n bytes). Returns the full message length. */
+size_t maglev_last_error(char* buf, size_t n);
+
+/* Reads and clears the device status word of the current device after the
+ * work queued on `stream` completes (this call synchronises that stream).
+ * *code receives MAGLEV_OK or the first MAGLEV_ERR_TIMEOUT recorded. */
+maglev_status maglev_device_status(void* stream, int* code);
+
+/* Bytes of the activations the forward saves for the backward ("saved"):
+ * the rotated queries and the mixed keys/values, 3 x [B,T,H,hd] of dtype. */
+size_t maglev_swa_saved_bytes(const maglev_swa_desc* desc);
+
+/* Bytes of scratch memory maglev_inject_swa_bwd needs ("workspace"). */
+size_t maglev_swa_bwd_workspace_bytes(const maglev_swa_desc* desc);
+
+/* a1 -- memory projection ([rainbus] 方法步骤详情: k_rec, v_rec come from the
+ * shared projections W_k^rec, W_v^rec applied to m'_{t-1}).
+ *   m_shift [B,T,d_mem]: row t holds m'_{t-1}, row 0 holds m'_0 = 0.
+ *   w_mk, w_mv [D, d_mem]: the shared projections (no layer index).
+ *   R_k, R_v [B,T,D] (out): R_k = m_shift W_mk^T, R_v = m_shift W_mv^T (raw:
+ *   no norm, no rotation). One call serves every layer of a step. */
+maglev_status maglev_mem_project(const maglev_swa_desc* desc, const void* m_shift,
+                                 const void* w_mk, const void* w_mv, void* R_k, void* R_v,
+                                 void* stream);
+
+/* a1-a5 -- forward of one injected sliding-window attention layer
+ * ([rainbus] 方法步骤详情; 前置知识 for SWA and for rotating both keys before the
+ * mix; [gist] Inferentiemechanisme: the memory rides in the existing K/V entry).
+ *   q, k, v [B,T,H,hd]: local projections before RoPE.
+ *   m_shift, w_mk, w_mv: if m_shift != NULL (and inject) the call first runs
+ *     maglev_mem_project into R_k, R_v; if m_shift == NULL, R_k and R_v are
+ *     inputs computed earlier (shared across layers). Unused when inject == 0.
+ *   R_k, R_v [B,T,D]: raw projected memory (see a1), written or read as above.
+ *   gate_logits [4,H] fp32: (k_loc, k_rec, v_loc, v_rec); g = 2*sigmoid(a),
+ *     a = -inf allowed (g = 0).
+ *   out [B,T,H,hd] (out): o_i = sum_j softmax_j(q~_i . k_bar_j / sqrt(hd)) v_bar_j
+ *     over j in [i-W+1, i], with q~ = RoPE(q), k_bar = g_kl RoPE(k) +
+ *     g_kr RoPE(RMSNorm_head(R_k)), v_bar = g_vl v + g_vr R_v.
+ *   lse [B,H,T] fp32 (out): log-sum-exp of each row's scaled scores.
+ *   saved (out): maglev_swa_saved_bytes(desc) bytes, read by the backward. */
+maglev_status maglev_inject_swa_fwd(const maglev_swa_desc* desc, const void* q, const void* k,
+                                    const void* v, const void* m_shift, const void* w_mk,
+                                    const void* w_mv, void* R_k, void* R_v,
+                                    const float* gate_logits, void* out, float* lse, void* saved,
+                                    void* stream);
+
+/* a6 -- backward of maglev_inject_swa_fwd (chain rule of the forward above).
+ *   Inputs: the forward's k, v, R_k, R_v, gate_logits, out, lse, saved, and
+ *   dout [B,T,H,hd] = dL/dout.
+ *   dq, dk, dv [B,T,H,hd] (out, overwritten).
+ *   dR_k, dR_v [B,T,D] (out): dL/dR; overwritten, or added to when
+ *     accumulate_dR != 0 (summing the shared projection's gradient over layers).
+ *     May be NULL when inject == 0.
+ *   dgate_logits [4,H] fp32 (out, overwritten); NULL when inject == 0.
+ *   m_shift, w_mk, w_mv, dm_shift, dw_mk, dw_mv: if m_shift != NULL the call
+ *     finishes with maglev_mem_project_bwd on the (accumulated) dR_k, dR_v.
+ *   workspace: maglev_swa_bwd_workspace_bytes(desc) bytes of scratch. */
+maglev_status maglev_inject_swa_bwd(const maglev_swa_desc* desc, const void* k, const void* v,
+                                    const void* R_k, const void* R_v, const float* gate_logits,
+                                    const void* out, const float* lse, const void* saved,
+                                    const void* dout, void* dq, void* dk, void* dv, void* dR_k,
+                                    void* dR_v, int accumulate_dR, float* dgate_logits,
+                                    const void* m_shift, const void* w_mk, const void* w_mv,
+                                    void* dm_shift, void* dw_mk, void* dw_mv, void* workspace,
+                                    void* stream);
+
+/* a6 -- backward of the shared memory projection.
+ *   dm_shift [B,T,d_mem] = dR_k W_mk + dR_v W_mv (overwritten);
+ *   dw_mk, dw_mv [D,d_mem] = dR^T m_shift summed over all B*T rows (overwritten). */
+maglev_status maglev_mem_project_bwd(const maglev_swa_desc* desc, const void* m_shift,
+                                     const void* w_mk, const void* w_mv, const void* dR_k,
+                                     const void* dR_v, void* dm_shift, void* dw_mk, void* dw_mv,
+                                     void* stream);
+
+/* Bytes of scratch memory maglev_consistency_loss needs for `rows` x `d`. */
+size_t maglev_consistency_workspace_bytes(int64_t rows, int d);
+
+/* a7 -- consistency loss ([rainbus] 方法步骤详情):
+ *   loss = lambda * inv_count * sum_t ||m_t - m'_t||^2 / sqrt(d)
+ *   m, m_target [rows, d] of dtype; inv_count = 1/|I| (0 means 1/rows).
+ *   loss: device fp32 scalar (out). The sum is reduced in a fixed order, so the
+ *   result is bitwise reproducible.
+ *   dm (nullable): dL/dm = 2 lambda inv_count (m - m') / sqrt(d); written, or
+ *     added to when accumulate_dm != 0. dm_target (nullable): -dL/dm, written.
+ *   workspace: maglev_consistency_workspace_bytes(rows, d) bytes. */
+maglev_status maglev_consistency_loss(const void* m, const void* m_target, int64_t rows, int d,
+                                      int dtype, float lambda, float inv_count, float* loss,
+                                      void* dm, void* dm_target, int accumulate_dm,
+                                      void* workspace, void* stream);
+
+/* a8 -- decode-side memory projection, once per token step (W^rec is shared by
+ * all layers and m_{p-1} is the same for all of them):
+ *   pos [B] int64 (device): absolute position p of each sequence's new token.
+ *   m_prev [B,d_mem]: m_{p-1}, the previous step's memory.
+ *   krec_rot [B,D] (out) = RoPE_p(RMSNorm_head(W_mk m_{p-1})); vrec [B,D] (out)
+ *   = W_mv m_{p-1}. */
+maglev_status maglev_decode_mem_project(const maglev_decode_desc* desc, const int64_t* pos,
+                                        const void* m_prev, const void* w_mk, const void* w_mv,
+                                        void* krec_rot, void* vrec, void* stream);
+
+/* a8 -- one recurrent decode step of one layer over its rolling W-entry K/V
+ * ring ([rainbus] 研究动机: m_t = P(x_{t-W+1:t}, M_{t-1}); 前置知识: the cache is
+ * that of plain SWA; [gist] Inferentiemechanisme).
+ *   pos [B] int64 (device): absolute position p of the new token. A negative
+ *     entry leaves that sequence's ring untouched and writes zeros to its out.
+ *   q, k, v [B,H,hd]: local projections of the new token, before RoPE.
+ *   krec_rot, vrec [B,H,hd]: from maglev_decode_mem_project (unused if inject == 0).
+ *   gate_logits [4,H] fp32: this layer's gates.
+ *   k_ring, v_ring [B,H,W,hd] (in/out): post-RoPE, post-mix entries; the entry
+ *     of position j lives in slot j mod W. The call writes the new entry to slot
+ *     p mod W (no other slot changes), then attends over the live slots
+ *     (positions max(0, p-W+1)..p).
+ *   out [B,H,hd] (out). */
+maglev_status maglev_decode_step(const maglev_decode_desc* desc, const int64_t* pos,
+                                 const void* q, const void* k, const void* v,
+                                 const void* krec_rot, const void* vrec, const float* gate_logits,
+                                 void* k_ring, void* v_ring, void* out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MAGLEV_H */

@@ -1,0 +1,56 @@
+// Device helpers shared by the kernels of libmaglev (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace maglev {
+
+typedef __nv_bfloat16 bf16;
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(bf16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ bf16 from_f<bf16>(float x) { return __float2bfloat16_rn(x); }
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+// g = 2*sigmoid(a); finite for a = +-inf.
+__device__ __forceinline__ float gate_value(float a) { return 2.0f / (1.0f + expf(-a)); }
+// dg/da = 2 s (1 - s).
+__device__ __forceinline__ float gate_slope(float a) {
+  float s = 1.0f / (1.0f + expf(-a));
+  return 2.0f * s * (1.0f - s);
+}
+
+// RoPE angle of pair c at absolute position p: p * base^(-2c/hd). The product
+// is formed in double and reduced to [-pi, pi] before the float sincos, so
+// positions in the thousands keep full float accuracy.
+__device__ __forceinline__ void rope_cos_sin(int64_t p, int c, int hd, double log2_base,
+                                             float* cs, float* sn) {
+  const double two_pi = 6.283185307179586476925286766559;
+  double inv_freq = exp2(-(2.0 * (double)c / (double)hd) * log2_base);
+  double ang = (double)p * inv_freq;
+  ang -= two_pi * rint(ang / two_pi);
+  sincosf((float)ang, sn, cs);
+}
+
+// Device status word (per device, defined in api.cu); kernels receive its address.
+enum { DEV_OK = 0, DEV_TIMEOUT = 4 };
+
+__device__ __forceinline__ void record_error(int* err, int code) {
+  if (err) atomicCAS(err, 0, code);
+}
+
+}  // namespace maglev

@@ -1,0 +1,73 @@
+// Host-side launchers of libmaglev's kernels (internal C++ interface between
+// the extern "C" boundary in api.cu and the kernel translation units).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace maglev {
+
+// C[M,N] (+)= A1[M,K1] B1[K1,N] + A2[M,K2] B2[K2,N], fp32 accumulation, any
+// element strides. A2/B2 may be null (K2 = 0). dtype: 0 = fp32, 1 = bf16 for
+// all of A, B and C.
+struct GemmArgs {
+  int64_t M, N, K1, K2;
+  const void *A1, *B1, *A2, *B2;
+  int64_t sa1m, sa1k, sb1k, sb1n, sa2m, sa2k, sb2k, sb2n;
+  void* C;
+  int64_t scm, scn;
+  int accumulate;
+  int dtype;
+};
+cudaError_t launch_gemm_simt(const GemmArgs& g, cudaStream_t s);
+
+struct SwaShape {
+  int B, T, H, hd, W, pos0, inject, dtype;
+  double log2_base;
+  float eps;
+};
+
+// q_rot = RoPE(q); k_bar, v_bar = gated mix (or RoPE(k), v when inject == 0).
+cudaError_t launch_prep(const SwaShape& s, const void* q, const void* k, const void* v,
+                        const void* Rk, const void* Rv, const float* gates, void* q_rot,
+                        void* k_bar, void* v_bar, cudaStream_t st);
+cudaError_t launch_attn_fwd_simt(const SwaShape& s, const void* q_rot, const void* k_bar,
+                                 const void* v_bar, void* out, float* lse, cudaStream_t st);
+// delta[b,h,i] = dout_i . out_i
+cudaError_t launch_attn_delta(const SwaShape& s, const void* out, const void* dout, float* delta,
+                              cudaStream_t st);
+// dq = RoPE^T(dq_rot) written in dtype.
+cudaError_t launch_attn_bwd_dq_simt(const SwaShape& s, const void* q_rot, const void* k_bar,
+                                    const void* v_bar, const void* dout, const float* lse,
+                                    const float* delta, void* dq, cudaStream_t st);
+// dk_bar, dv_bar in fp32.
+cudaError_t launch_attn_bwd_dkdv_simt(const SwaShape& s, const void* q_rot, const void* k_bar,
+                                      const void* v_bar, const void* dout, const float* lse,
+                                      const float* delta, float* dk_bar, float* dv_bar,
+                                      cudaStream_t st);
+// dk, dv, dR_k, dR_v and per-row gate partials gpart[B*T][4][H] from dk_bar, dv_bar.
+cudaError_t launch_unmix(const SwaShape& s, const float* dk_bar, const float* dv_bar,
+                         const void* k, const void* v, const void* Rk, const void* Rv,
+                         const float* gates, void* dk, void* dv, void* dRk, void* dRv,
+                         int accumulate, float* gpart, cudaStream_t st);
+cudaError_t launch_gate_reduce(int rows, int H, const float* gpart, const float* gates,
+                               float* dgate, cudaStream_t st);
+
+int loss_partial_blocks(int64_t n);
+cudaError_t launch_consistency_loss(const void* m, const void* mt, int64_t rows, int d, int dtype,
+                                    float scale_loss, float scale_grad, float* loss, void* dm,
+                                    void* dmt, int accumulate, float* partials, cudaStream_t st);
+
+struct DecShape {
+  int B, H, hd, W, inject, dtype;
+  double log2_base;
+  float eps;
+};
+cudaError_t launch_rmsnorm_rope_rows(const DecShape& s, const int64_t* pos, void* x,
+                                     cudaStream_t st);
+cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void* q, const void* k,
+                               const void* v, const void* krec, const void* vrec,
+                               const float* gates, void* k_ring, void* v_ring, void* out,
+                               cudaStream_t st);
+
+}  // namespace maglev

@@ -1,0 +1,112 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+include/maglev.h declares, and validates its arguments before any launch
+(no GPU needed: no call here reaches a kernel)."""
+import ctypes
+
+import pytest
+
+from sliding_window_recurrent_b200 import build as _build
+
+_build.build(quiet=True)
+
+import sliding_window_recurrent_b200 as mg  # noqa: E402
+
+
+def desc(**kw):
+    base = dict(B=1, T=16, H=2, hd=64, d_mem=32, window=8, rope_base=10000.0, rms_eps=1e-6,
+                inject=1, pos0=0, dtype=mg.MAGLEV_F32, spin_limit=0)
+    base.update(kw)
+    return mg.SwaDesc(**base)
+
+
+def test_every_declared_symbol_is_exported():
+    names = mg.header_symbols()
+    assert len(names) >= 13
+    lib = ctypes.CDLL(mg.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version():
+    assert "sm_100a" in mg.maglev_version()
+
+
+def test_sizes():
+    d = desc(B=2, T=100, H=3, hd=128, dtype=mg.MAGLEV_BF16)
+    n = 2 * 100 * 3 * 128 * 2
+    assert mg.maglev_swa_saved_bytes(d) >= 3 * n
+    assert mg.maglev_swa_bwd_workspace_bytes(d) >= 2 * (n * 2)
+    assert mg.maglev_swa_saved_bytes(desc(hd=96)) == 0          # invalid desc -> 0
+    assert mg.maglev_consistency_workspace_bytes(1000, 1280) >= 4
+
+
+FAKE = 1 << 20   # aligned, never dereferenced: validation fails first
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(hd=96), mg.MAGLEV_ERR_UNSUPPORTED),
+    (dict(window=0), mg.MAGLEV_ERR_INVALID_ARG),
+    (dict(H=0), mg.MAGLEV_ERR_INVALID_ARG),
+    (dict(T=-1), mg.MAGLEV_ERR_INVALID_ARG),
+    (dict(dtype=7), mg.MAGLEV_ERR_INVALID_ARG),
+    (dict(pos0=-3), mg.MAGLEV_ERR_INVALID_ARG),
+    (dict(rope_base=0.5), mg.MAGLEV_ERR_INVALID_ARG),
+    (dict(d_mem=0), mg.MAGLEV_ERR_INVALID_ARG),
+])
+def test_fwd_rejects_bad_desc(bad, status):
+    with pytest.raises(mg.MaglevError) as e:
+        mg.maglev_inject_swa_fwd(desc(**bad), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                 FAKE, FAKE, FAKE, stream=0)
+    assert e.value.status == status
+
+
+def test_fwd_rejects_null_and_misaligned_pointers():
+    with pytest.raises(mg.MaglevError) as e:
+        mg.maglev_inject_swa_fwd(desc(), None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                 FAKE, FAKE, FAKE, stream=0)
+    assert e.value.status == mg.MAGLEV_ERR_INVALID_ARG and "q" in str(e.value)
+    with pytest.raises(mg.MaglevError) as e:
+        mg.maglev_inject_swa_fwd(desc(), FAKE, FAKE + 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                 FAKE, FAKE, FAKE, stream=0)
+    assert "aligned" in str(e.value)
+    # injection needs gate logits
+    with pytest.raises(mg.MaglevError):
+        mg.maglev_inject_swa_fwd(desc(), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                                 FAKE, FAKE, FAKE, stream=0)
+
+
+def test_empty_problems_enqueue_nothing():
+    # B = 0 or T = 0 is valid and returns before any launch.
+    for d in (desc(B=0), desc(T=0)):
+        mg.maglev_inject_swa_fwd(d, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                 FAKE, FAKE, stream=0)
+        mg.maglev_inject_swa_bwd(d, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                 FAKE, FAKE, FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                 FAKE, FAKE, stream=0)
+    mg.maglev_consistency_loss(FAKE, FAKE, 0, 16, mg.MAGLEV_F32, 1.0, 0.0, FAKE, None, None, 0,
+                               FAKE, stream=0)
+
+
+def test_bwd_and_loss_and_decode_validation():
+    with pytest.raises(mg.MaglevError):
+        mg.maglev_inject_swa_bwd(desc(), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                 FAKE, FAKE, FAKE, None, FAKE, 0, FAKE, None, None, None, None,
+                                 None, None, FAKE, stream=0)
+    with pytest.raises(mg.MaglevError):
+        mg.maglev_consistency_loss(FAKE, FAKE, 10, 0, mg.MAGLEV_F32, 1.0, 0.0, FAKE, None, None,
+                                   0, FAKE, stream=0)
+    with pytest.raises(mg.MaglevError):
+        mg.maglev_consistency_loss(FAKE, FAKE, 10, 8, mg.MAGLEV_F32, float("nan"), 0.0, FAKE,
+                                   None, None, 0, FAKE, stream=0)
+    dd = mg.DecodeDesc(B=2, H=2, hd=64, d_mem=16, window=0, rope_base=1e4, rms_eps=1e-6,
+                       inject=1, dtype=mg.MAGLEV_F32, spin_limit=0)
+    with pytest.raises(mg.MaglevError):
+        mg.maglev_decode_step(dd, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, stream=0)
+    dd.window = 64
+    dd.hd = 80
+    with pytest.raises(mg.MaglevError) as e:
+        mg.maglev_decode_step(dd, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, stream=0)
+    assert e.value.status == mg.MAGLEV_ERR_UNSUPPORTED
+    dd.hd = 64
+    dd.B = 0
+    mg.maglev_decode_step(dd, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, stream=0)
