@@ -325,7 +325,7 @@ def run_decode_bench(torch, dev, steps, warmup, peaks):
 
     def one_step():
         S.mem_project(pos, m_prev, wk, wv)
-        h = h_bank[it % 16].float()
+        h = torch.index_select(h_bank, 0, torch.remainder(it, 16).view(1))[0].float()
         for l in range(L):
             xn = torch.nn.functional.rms_norm(h, (d,), eps=1e-6).to(bf)
             q, k, v = ((xn @ w.t()).view(B, H, hd) for w in wqkv[l])

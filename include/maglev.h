@@ -80,9 +80,10 @@ const char* maglev_version(void);
  * has launched in the process so far (all threads, all devices).
  * maglev_profile_enable(1) brackets every later launch with CUDA events
  * recorded on the launch's own stream; maglev_profile_report() waits for the
- * recorded events, writes one line "name kernels milliseconds" per traced
- * launch into buf (NUL-terminated, truncated to n bytes), clears the record
- * and returns the full text length. Tracing is off by default. */
+ * recorded events and returns the length of the report text, one line
+ * "name kernels milliseconds" per traced launch. With buf != NULL it also
+ * copies the text into buf (NUL-terminated, truncated to n bytes) and clears
+ * it; with buf == NULL it only returns the length. Tracing is off by default. */
 long long maglev_launch_count(void);
 void maglev_profile_enable(int on);
 size_t maglev_profile_report(char* buf, size_t n);

@@ -43,6 +43,7 @@ struct ProfRec {
 };
 std::mutex g_prof_mu;
 std::vector<ProfRec> g_prof;
+std::string g_prof_text;  // resolved records not yet handed out
 
 struct ProfScope {
   const char* name;
@@ -275,26 +276,25 @@ void maglev_profile_enable(int on) { g_prof_on.store(on ? 1 : 0); }
 
 size_t maglev_profile_report(char* buf, size_t n) {
   std::vector<ProfRec> recs;
-  {
-    std::lock_guard<std::mutex> lock(g_prof_mu);
-    recs.swap(g_prof);
-  }
-  std::string text;
-  for (const ProfRec& r : recs) {
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  recs.swap(g_prof);
+  for (const ProfRec& r : recs) {  // resolve finished records into the pending text
     float ms = -1.0f;
     if (cudaEventSynchronize(r.b) == cudaSuccess) cudaEventElapsedTime(&ms, r.a, r.b);
     char line[160];
     snprintf(line, sizeof(line), "%s %d %.6f\n", r.name, r.kernels, ms);
-    text += line;
+    g_prof_text += line;
     cudaEventDestroy(r.a);
     cudaEventDestroy(r.b);
   }
-  if (buf && n) {
-    size_t k = text.size() < n - 1 ? text.size() : n - 1;
-    memcpy(buf, text.data(), k);
+  const size_t len = g_prof_text.size();
+  if (buf && n) {  // hand the text over and clear it
+    size_t k = len < n - 1 ? len : n - 1;
+    memcpy(buf, g_prof_text.data(), k);
     buf[k] = '\0';
+    g_prof_text.clear();
   }
-  return text.size();
+  return len;
 }
 
 size_t maglev_last_error(char* buf, size_t n) {
