@@ -179,6 +179,27 @@ maglev_status maglev_consistency_loss(const void* m, const void* m_target, int64
                                       void* dm, void* dm_target, int accumulate_dm,
                                       void* workspace, void* stream);
 
+/* Scratch-free variant of maglev_consistency_loss, for callers that cannot
+ * allocate device memory: e.g. a plugin or custom-op interface that hands over
+ * its input and output tensors but no workspace, or a latency-critical loop in
+ * which cudaMalloc (which may synchronise the device) is not allowed. The
+ * paper has no counterpart: this is an interface convenience of this library,
+ * not a step of the method.
+ * Same arguments and results as maglev_consistency_loss, minus `workspace`:
+ * the per-block partial sums live in a file-scope device array of 32768 floats
+ * (128 KiB) that every device which loads the library keeps until exit.
+ * Limit: rows * d <= 67,108,864 elements; larger inputs return
+ * MAGLEV_ERR_UNSUPPORTED with a message. The first call on each device looks
+ * up the array's device address (cudaGetSymbolAddress) with that device
+ * current: make that first call before any stream capture. All calls share
+ * the array and each call overwrites the partials it reads, so nothing needs
+ * clearing, but calls that overlap on the GPU race and must be serialised.
+ * The call allocates no memory. */
+maglev_status maglev_consistency_loss_noalloc(const void* m, const void* m_target, int64_t rows,
+                                              int d, int dtype, float lambda, float inv_count,
+                                              float* loss, void* dm, void* dm_target,
+                                              int accumulate_dm, void* stream);
+
 /* a8 -- decode-side memory projection, once per token step (W^rec is shared by
  * all layers and m_{p-1} is the same for all of them):
  *   pos [B] int64 (device): absolute position p of each sequence's new token.

@@ -67,6 +67,7 @@ _SIGS = {
     "maglev_inject_swa_bwd": ([ctypes.POINTER(SwaDesc)] + [_P] * 14 + [_I] + [_P] * 9, _I),
     "maglev_mem_project_bwd": ([ctypes.POINTER(SwaDesc)] + [_P] * 9, _I),
     "maglev_consistency_loss": ([_P, _P, _I64, _I, _I, _F, _F, _P, _P, _P, _I, _P, _P], _I),
+    "maglev_consistency_loss_noalloc": ([_P, _P, _I64, _I, _I, _F, _F, _P, _P, _P, _I, _P], _I),
     "maglev_decode_mem_project": ([ctypes.POINTER(DecodeDesc)] + [_P] * 7, _I),
     "maglev_decode_step": ([ctypes.POINTER(DecodeDesc)] + [_P] * 11, _I),
 }
@@ -202,6 +203,15 @@ def maglev_consistency_loss(m, m_target, rows, d, dtype, lam, inv_count, loss, d
                                         float(lam), float(inv_count), _ptr(loss), _ptr(dm),
                                         _ptr(dm_target), int(accumulate_dm), _ptr(workspace),
                                         _stream(stream)))
+
+
+def maglev_consistency_loss_noalloc(m, m_target, rows, d, dtype, lam, inv_count, loss, dm, dm_target,
+                                    accumulate_dm, stream=None):
+    """Scratch-free consistency loss: same results as maglev_consistency_loss,
+    no workspace argument (for callers that cannot allocate device memory)."""
+    _check(_lib.maglev_consistency_loss_noalloc(_ptr(m), _ptr(m_target), int(rows), int(d), int(dtype),
+                                                float(lam), float(inv_count), _ptr(loss), _ptr(dm),
+                                                _ptr(dm_target), int(accumulate_dm), _stream(stream)))
 
 
 def maglev_decode_mem_project(desc, pos, m_prev, w_mk, w_mv, krec_rot, vrec, stream=None):

@@ -266,6 +266,10 @@ maglev_status status_word(int** out) {
 
 }  // namespace
 
+namespace maglev {
+void set_last_error(const char* msg) { g_last_error = msg; }
+}  // namespace maglev
+
 extern "C" {
 
 const char* maglev_version(void) { return "maglev-b200 0.1.0 (sm_100a)"; }

@@ -70,4 +70,7 @@ cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void
                                const float* gates, void* k_ring, void* v_ring, void* out,
                                cudaStream_t st);
 
+// Sets the calling thread's message returned by maglev_last_error().
+void set_last_error(const char* msg);
+
 }  // namespace maglev
