@@ -168,9 +168,22 @@ const P* at(const void* base, size_t off) {
   return reinterpret_cast<const P*>(static_cast<const char*>(base) + off);
 }
 
+maglev_status status_word(int** out);
+
+int64_t spin_limit_of(int64_t v) { return v > 0 ? v : DEFAULT_SPIN_LIMIT; }
+
 maglev_status run_mem_project(const maglev_swa_desc* d, const void* m, const void* wk,
                               const void* wv, void* Rk, void* Rv, cudaStream_t st) {
   const int64_t M = (int64_t)d->B * d->T, D = (int64_t)d->H * d->hd, K = d->d_mem;
+  if (d->dtype == MAGLEV_BF16 && K % 8 == 0 && D % 256 == 0) {
+    int* err = nullptr;
+    maglev_status s = status_word(&err);
+    if (s != MAGLEV_OK) return s;
+    MAGLEV_LAUNCH(1, st, launch_proj_fwd_tc(M, (int)D, (int)K, m, wk, wv, Rk, Rv,
+                                            spin_limit_of(d->spin_limit), err, st),
+                  "mem_project_tc");
+    return MAGLEV_OK;
+  }
   for (int which = 0; which < 2; ++which) {
     GemmArgs g{};
     g.M = M;
@@ -197,6 +210,22 @@ maglev_status run_mem_project_bwd(const maglev_swa_desc* d, const void* m, const
                                   const void* wv, const void* dRk, const void* dRv, void* dm,
                                   void* dwk, void* dwv, cudaStream_t st) {
   const int64_t M = (int64_t)d->B * d->T, D = (int64_t)d->H * d->hd, K = d->d_mem;
+  int* err = nullptr;
+  maglev_status stw = status_word(&err);
+  if (stw != MAGLEV_OK) return stw;
+  const bool tc = d->dtype == MAGLEV_BF16 && K % 8 == 0;
+  if (dm && tc && D % 64 == 0) {
+    MAGLEV_LAUNCH(1, st, launch_proj_bwd_dm_tc(M, (int)D, (int)K, dRk, dRv, wk, wv, dm,
+                                               spin_limit_of(d->spin_limit), err, st),
+                  "mem_project_bwd_dm_tc");
+    dm = nullptr;
+  }
+  if (dwk && dwv && tc && D % 128 == 0) {
+    MAGLEV_LAUNCH(1, st, launch_proj_bwd_dw_tc(M, (int)D, (int)K, dRk, dRv, m, dwk, dwv,
+                                               spin_limit_of(d->spin_limit), err, st),
+                  "mem_project_bwd_dw_tc");
+    dwk = dwv = nullptr;
+  }
   if (dm) {  // dm[M, K] = dRk[M, D] W_mk[D, K] + dRv W_mv
     GemmArgs g{};
     g.M = M;

@@ -70,6 +70,24 @@ cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void
                                const float* gates, void* k_ring, void* v_ring, void* out,
                                cudaStream_t st);
 
+// tcgen05 projection GEMMs (bf16 in/out, fp32 accumulation in TMEM).
+// R_k | R_v [M, D] = m_shift [M, d] x [W_mk; W_mv]^T. Needs d % 8 == 0, D % 256 == 0.
+cudaError_t launch_proj_fwd_tc(int64_t M, int D, int d, const void* m_shift, const void* w_mk,
+                               const void* w_mv, void* Rk, void* Rv, int64_t spin_limit, int* err,
+                               cudaStream_t s);
+// dm [M, d] = dR_k W_mk + dR_v W_mv. Needs d % 8 == 0, D % 64 == 0.
+cudaError_t launch_proj_bwd_dm_tc(int64_t M, int D, int d, const void* dRk, const void* dRv,
+                                  const void* w_mk, const void* w_mv, void* dm, int64_t spin_limit,
+                                  int* err, cudaStream_t s);
+// dW_mk | dW_mv [D, d] = dR^T m_shift. Needs d % 8 == 0, D % 128 == 0.
+cudaError_t launch_proj_bwd_dw_tc(int64_t M, int D, int d, const void* dRk, const void* dRv,
+                                  const void* m_shift, void* dwk, void* dwv, int64_t spin_limit,
+                                  int* err, cudaStream_t s);
+int num_sms();
+
+// Default bound on the polls of one in-kernel wait (about a second).
+constexpr int64_t DEFAULT_SPIN_LIMIT = (int64_t)1 << 22;
+
 // Sets the calling thread's message returned by maglev_last_error().
 void set_last_error(const char* msg);
 

@@ -1,0 +1,397 @@
+// Persistent tcgen05 GEMM for the shared memory projection of Maglev's
+// recurrent K/V injection ("Maglev: Sliding Recurrent Memory",
+// paper.rainbus.top, 方法步骤详情: k_rec and v_rec come from the projections
+// W_k^rec, W_v^rec shared by all layers) and its backward:
+//   forward  R = m_shift [B*T, d] x [W_mk; W_mv]^T           -> R_k | R_v
+//   backward dm = [dR_k | dR_v] x [W_mk; W_mv]                (K = 2D)
+//            dW = [dR_k | dR_v]^T x m_shift                   (M = 2D)
+//
+// One CTA per SM, 6 warps: warp 0 issues TMA loads of 64-wide K blocks into a
+// ring of 128B-swizzled shared-memory stages, warp 1 issues tcgen05.mma
+// (128 x BN x 16, bf16 -> fp32) into one of two TMEM accumulators, warps 2-5
+// drain the other accumulator (tcgen05.ld) and store bf16. Operands may be
+// K-major or MN-major; a second tensor map per operand lets one launch span
+// the two halves (k/v) without a concatenated copy. Every wait is bounded.
+#include <cuda.h>
+
+#include <mutex>
+
+#include "launchers.h"
+#include "tc_common.cuh"
+
+namespace maglev {
+namespace {
+
+using namespace tc;
+
+constexpr int BM = 128, BK = 64;
+constexpr int NUM_THREADS = 192;
+
+struct TcGemmParams {
+  int M, N, K;
+  int tiles_m, tiles_n;
+  int a_switch_m, a_switch_k;  // rows / K index where operand A moves to map 1
+  int b_switch_n, b_switch_k;
+  int out_switch_m, out_switch_n;
+  void* out0;
+  void* out1;
+  int64_t ldo;
+  int64_t spin_limit;
+  int* err;
+};
+
+template <int BN, bool A_MN, bool B_MN>
+struct Cfg {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+};
+
+template <int BN, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                   const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+                   TcGemmParams p) {
+  using C = Cfg<BN, A_MN, B_MN>;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const Abort ab{abort_flag, p.err, p.spin_limit};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA0);
+    tma_prefetch_desc(&tmA1);
+    tma_prefetch_desc(&tmB0);
+    tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_tiles = p.tiles_m * p.tiles_n;
+  const int kblocks = (p.K + BK - 1) / BK;
+  constexpr uint32_t IDESC = idesc_bf16(BM, BN, A_MN, B_MN);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0;           // bit s: stage s was armed at least once
+      uint32_t armed_parity = 0;    // bit s: parity of the last arming of stage s
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int tm = t % p.tiles_m, tn = t / p.tiles_m;
+        const int m0 = tm * BM, n0 = tn * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, ab)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          armed |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          const int k0 = kb * BK;
+          // operand A
+          {
+            const bool second = (p.a_switch_m > 0 && m0 >= p.a_switch_m) || (p.a_switch_k > 0 && k0 >= p.a_switch_k);
+            const CUtensorMap* m = second ? &tmA1 : &tmA0;
+            const int mm = (p.a_switch_m > 0 && m0 >= p.a_switch_m) ? m0 - p.a_switch_m : m0;
+            const int kk = (p.a_switch_k > 0 && k0 >= p.a_switch_k) ? k0 - p.a_switch_k : k0;
+            uint8_t* dst = sA + stage * C::A_BYTES;
+            if (A_MN) {
+              tma_load_2d(dst, m, &full[stage], mm, kk);
+              tma_load_2d(dst + 8192, m, &full[stage], mm + 64, kk);
+            } else {
+              tma_load_2d(dst, m, &full[stage], kk, mm);
+            }
+          }
+          // operand B
+          {
+            const bool second = (p.b_switch_n > 0 && n0 >= p.b_switch_n) || (p.b_switch_k > 0 && k0 >= p.b_switch_k);
+            const CUtensorMap* m = second ? &tmB1 : &tmB0;
+            const int nn = (p.b_switch_n > 0 && n0 >= p.b_switch_n) ? n0 - p.b_switch_n : n0;
+            const int kk = (p.b_switch_k > 0 && k0 >= p.b_switch_k) ? k0 - p.b_switch_k : k0;
+            uint8_t* dst = sB + stage * C::B_BYTES;
+            if (B_MN) {
+#pragma unroll
+              for (int j = 0; j < BN / 64; ++j) tma_load_2d(dst + j * 8192, m, &full[stage], nn + 64 * j, kk);
+            } else {
+              tma_load_2d(dst, m, &full[stage], kk, nn);
+            }
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // every armed stage's last load must land before the CTA may exit
+      for (int s = 0; s < STAGES; ++s)
+        if (armed & (1u << s)) mbar_drain(&full[s], (armed_parity >> s) & 1u, p.spin_limit);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, ab)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, ab)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int k16 = 0; k16 < BK / 16; ++k16) {
+            const uint64_t ad = A_MN ? mnmajor_desc(a_addr, k16) : kmajor_desc(a_addr, k16);
+            const uint64_t bd = B_MN ? mnmajor_desc(b_addr, k16) : kmajor_desc(b_addr, k16);
+            mma_ss(d_tmem, ad, bd, IDESC, (kb > 0 || k16 > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&tfull[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      // all issued MMAs must finish before TMEM is released
+      mma_commit(drain);
+      mbar_drain(drain, 0, p.spin_limit);
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      const int tm = t % p.tiles_m, tn = t / p.tiles_m;
+      int m0 = tm * BM, n0 = tn * BN;
+      if (!mbar_wait(&tfull[acc], acc_phase, ab)) break;
+      tc_fence_after();
+      const int gm = m0 + row;
+      bf16* out = static_cast<bf16*>(p.out0);
+      int om = gm, on0 = n0;
+      if (p.out_switch_m > 0 && m0 >= p.out_switch_m) {
+        out = static_cast<bf16*>(p.out1);
+        om -= p.out_switch_m;
+      }
+      if (p.out_switch_n > 0 && n0 >= p.out_switch_n) {
+        out = static_cast<bf16*>(p.out1);
+        on0 -= p.out_switch_n;
+      }
+      const int n_lim = (p.out_switch_n > 0 && n0 < p.out_switch_n) ? p.out_switch_n : p.N;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c0), r);
+        tmem_wait_ld();
+        if (gm < p.M && n0 + c0 < n_lim) {
+          bf16* dst = out + (int64_t)om * p.ldo + on0 + c0;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            if (n0 + c0 + 8 * g < n_lim) {
+              uint4 v;
+              v.x = pack_bf16(__uint_as_float(r[8 * g + 0]), __uint_as_float(r[8 * g + 1]));
+              v.y = pack_bf16(__uint_as_float(r[8 * g + 2]), __uint_as_float(r[8 * g + 3]));
+              v.z = pack_bf16(__uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5]));
+              v.w = pack_bf16(__uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7]));
+              *reinterpret_cast<uint4*>(dst + 8 * g) = v;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::once_flag g_encode_once;
+EncodeTiledFn g_encode = nullptr;
+
+}  // namespace
+
+cudaError_t make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                              uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+  std::call_once(g_encode_once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  if (!g_encode) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+namespace {
+
+template <int BN, bool A_MN, bool B_MN>
+cudaError_t run_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0, const CUtensorMap& b1,
+                     TcGemmParams p, cudaStream_t s) {
+  using C = Cfg<BN, A_MN, B_MN>;
+  auto kern = tc_gemm_kernel<BN, A_MN, B_MN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int tiles = p.tiles_m * p.tiles_n;
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  kern<<<grid, NUM_THREADS, C::SMEM, s>>>(a0, a1, b0, b1, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// R_k | R_v [M, D] = m_shift [M, d] x W^T, W_mk / W_mv [D, d].
+cudaError_t launch_proj_fwd_tc(int64_t M, int D, int d, const void* m_shift, const void* w_mk,
+                               const void* w_mv, void* Rk, void* Rv, int64_t spin_limit, int* err,
+                               cudaStream_t s) {
+  constexpr int BN = 256;
+  CUtensorMap a, b0, b1;
+  cudaError_t e;
+  if ((e = make_tmap_bf16_2d(&a, m_shift, d, M, (uint64_t)d * 2, 64, BM)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&b0, w_mk, d, D, (uint64_t)d * 2, 64, BN)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&b1, w_mv, d, D, (uint64_t)d * 2, 64, BN)) != cudaSuccess) return e;
+  TcGemmParams p{};
+  p.M = (int)M;
+  p.N = 2 * D;
+  p.K = d;
+  p.tiles_m = (int)((M + BM - 1) / BM);
+  p.tiles_n = (2 * D + BN - 1) / BN;
+  p.b_switch_n = D;
+  p.out_switch_n = D;
+  p.out0 = Rk;
+  p.out1 = Rv;
+  p.ldo = D;
+  p.spin_limit = spin_limit;
+  p.err = err;
+  return run_gemm<BN, false, false>(a, a, b0, b1, p, s);
+}
+
+// dm [M, d] = dR_k [M, D] W_mk [D, d] + dR_v W_mv (K = 2D, B operand N-contiguous).
+cudaError_t launch_proj_bwd_dm_tc(int64_t M, int D, int d, const void* dRk, const void* dRv,
+                                  const void* w_mk, const void* w_mv, void* dm, int64_t spin_limit,
+                                  int* err, cudaStream_t s) {
+  constexpr int BN = 256;
+  CUtensorMap a0, a1, b0, b1;
+  cudaError_t e;
+  if ((e = make_tmap_bf16_2d(&a0, dRk, D, M, (uint64_t)D * 2, 64, BM)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&a1, dRv, D, M, (uint64_t)D * 2, 64, BM)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&b0, w_mk, d, D, (uint64_t)d * 2, 64, 64)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&b1, w_mv, d, D, (uint64_t)d * 2, 64, 64)) != cudaSuccess) return e;
+  TcGemmParams p{};
+  p.M = (int)M;
+  p.N = d;
+  p.K = 2 * D;
+  p.tiles_m = (int)((M + BM - 1) / BM);
+  p.tiles_n = (d + BN - 1) / BN;
+  p.a_switch_k = D;
+  p.b_switch_k = D;
+  p.out0 = dm;
+  p.out1 = dm;
+  p.ldo = d;
+  p.spin_limit = spin_limit;
+  p.err = err;
+  return run_gemm<BN, false, true>(a0, a1, b0, b1, p, s);
+}
+
+// dW_mk | dW_mv [D, d] = dR^T [D, M] m_shift [M, d] (A and B both M-contiguous in memory).
+cudaError_t launch_proj_bwd_dw_tc(int64_t M, int D, int d, const void* dRk, const void* dRv,
+                                  const void* m_shift, void* dwk, void* dwv, int64_t spin_limit,
+                                  int* err, cudaStream_t s) {
+  constexpr int BN = 256;
+  CUtensorMap a0, a1, b;
+  cudaError_t e;
+  if ((e = make_tmap_bf16_2d(&a0, dRk, D, M, (uint64_t)D * 2, 64, 64)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&a1, dRv, D, M, (uint64_t)D * 2, 64, 64)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&b, m_shift, d, M, (uint64_t)d * 2, 64, 64)) != cudaSuccess) return e;
+  TcGemmParams p{};
+  p.M = 2 * D;
+  p.N = d;
+  p.K = (int)M;
+  p.tiles_m = (2 * D + BM - 1) / BM;
+  p.tiles_n = (d + BN - 1) / BN;
+  p.a_switch_m = D;
+  p.out_switch_m = D;
+  p.out0 = dwk;
+  p.out1 = dwv;
+  p.ldo = d;
+  p.spin_limit = spin_limit;
+  p.err = err;
+  return run_gemm<BN, true, true>(a0, a1, b, b, p, s);
+}
+
+}  // namespace maglev
