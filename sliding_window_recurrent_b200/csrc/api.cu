@@ -416,9 +416,19 @@ maglev_status maglev_inject_swa_fwd(const maglev_swa_desc* d, const void* q, con
   MAGLEV_LAUNCH(1, s, launch_prep(sh, q, k, v, R_k, R_v, gate_logits, at<char>(saved, L.q),
                                    at<char>(saved, L.k), at<char>(saved, L.v), s),
                 "inject_prep");
-  MAGLEV_LAUNCH(1, s, launch_attn_fwd_simt(sh, at<char>(saved, L.q), at<char>(saved, L.k),
-                                            at<char>(saved, L.v), out, lse, s),
-                "attn_fwd");
+  if (d->dtype == MAGLEV_BF16) {
+    int* err = nullptr;
+    st = status_word(&err);
+    if (st != MAGLEV_OK) return st;
+    MAGLEV_LAUNCH(1, s, launch_attn_fwd_tc(sh, at<char>(saved, L.q), at<char>(saved, L.k),
+                                            at<char>(saved, L.v), out, lse, spin_limit_of(d->spin_limit),
+                                            err, s),
+                  "attn_fwd_tc");
+  } else {
+    MAGLEV_LAUNCH(1, s, launch_attn_fwd_simt(sh, at<char>(saved, L.q), at<char>(saved, L.k),
+                                              at<char>(saved, L.v), out, lse, s),
+                  "attn_fwd");
+  }
   return MAGLEV_OK;
 }
 

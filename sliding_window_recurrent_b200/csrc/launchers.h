@@ -85,6 +85,10 @@ cudaError_t launch_proj_bwd_dw_tc(int64_t M, int D, int d, const void* dRk, cons
                                   int* err, cudaStream_t s);
 int num_sms();
 
+// tcgen05 banded attention forward on the saved bf16 q_rot / k_bar / v_bar.
+cudaError_t launch_attn_fwd_tc(const SwaShape& s, const void* q_rot, const void* k_bar, const void* v_bar,
+                               void* out, float* lse, int64_t spin_limit, int* err, cudaStream_t st);
+
 // Default bound on the polls of one in-kernel wait (about a second).
 constexpr int64_t DEFAULT_SPIN_LIMIT = (int64_t)1 << 22;
 
