@@ -23,9 +23,11 @@
  *    returns MAGLEV_OK, or an error code with nothing enqueued (INVALID_ARG,
  *    UNSUPPORTED) or after a CUDA launch error (CUDA). maglev_last_error()
  *    returns the message of the calling thread's last failure. Kernels that
- *    wait on asynchronous copies bound every wait by desc->spin_limit polls;
- *    on expiry they record MAGLEV_ERR_TIMEOUT in a device status word, abandon
- *    the tile and return; read it with maglev_device_status().
+ *    wait on asynchronous copies or tensor-core work bound every wait by
+ *    desc->spin_limit microseconds of GPU time (0 = 1 s); on expiry they
+ *    record MAGLEV_ERR_TIMEOUT in a device status word, stop issuing work,
+ *    drain what is in flight (bounded by 2 s), free their tensor memory and
+ *    return; read the word with maglev_device_status().
  *  - Empty problems (B == 0 or T == 0, rows == 0) are valid and enqueue nothing.
  */
 #ifndef MAGLEV_H
@@ -53,7 +55,7 @@ typedef enum { MAGLEV_F32 = 0, MAGLEV_BF16 = 1 } maglev_dtype;
  * width, window W >= 1 (keys j in [i-W+1, i]; W >= T is full causal attention),
  * rope_base (10000 in the d20 model), rms_eps (1e-6), inject (0: plain SWA --
  * memory arguments may be NULL), pos0 (absolute position of row 0), dtype,
- * spin_limit (bound on each in-kernel wait, 0 = library default). */
+ * spin_limit (bound on each in-kernel wait in microseconds, 0 = 1 s). */
 typedef struct {
   int B, T, H, hd, d_mem, window;
   float rope_base, rms_eps;

@@ -146,7 +146,7 @@ SavedLayout saved_layout(const maglev_swa_desc* d) {
 
 // Offsets inside the backward's workspace.
 struct BwdLayout {
-  size_t dkb, dvb, delta, gpart, total;
+  size_t dkb, dvb, delta, gpart, dq_acc, total;
 };
 BwdLayout bwd_layout(const maglev_swa_desc* d) {
   BwdLayout L;
@@ -155,7 +155,8 @@ BwdLayout bwd_layout(const maglev_swa_desc* d) {
   L.dvb = L.dkb + align256(n * 4);
   L.delta = L.dvb + align256(n * 4);
   L.gpart = L.delta + align256((size_t)d->B * d->H * d->T * 4);
-  L.total = L.gpart + align256((size_t)d->B * d->T * 4 * d->H * 4);
+  L.dq_acc = L.gpart + align256((size_t)d->B * d->T * 4 * d->H * 4);
+  L.total = L.dq_acc + (d->dtype == MAGLEV_BF16 ? align256(n * 4) : 0);
   return L;
 }
 
@@ -481,11 +482,22 @@ maglev_status maglev_inject_swa_bwd(const maglev_swa_desc* d, const void* k, con
   float* dvb = at<float>(workspace, Wk.dvb);
   float* gpart = at<float>(workspace, Wk.gpart);
   MAGLEV_LAUNCH(1, s, launch_attn_delta(sh, out, dout, delta, s), "attn_delta");
-  MAGLEV_LAUNCH(1, s, launch_attn_bwd_dq_simt(sh, qr, kb, vb, dout, lse, delta, dq, s), "attn_bwd_dq");
-  MAGLEV_LAUNCH(1, s, launch_attn_bwd_dkdv_simt(sh, qr, kb, vb, dout, lse, delta, dkb, dvb, s),
-                "attn_bwd_dkdv");
+  float* dq_acc = nullptr;
+  if (d->dtype == MAGLEV_BF16) {
+    int* err = nullptr;
+    st = status_word(&err);
+    if (st != MAGLEV_OK) return st;
+    dq_acc = at<float>(workspace, Wk.dq_acc);
+    MAGLEV_LAUNCH(1, s, launch_attn_bwd_tc(sh, qr, kb, vb, dout, lse, delta, dq_acc, dkb, dvb,
+                                           spin_limit_of(d->spin_limit), err, s),
+                  "attn_bwd_tc");
+  } else {
+    MAGLEV_LAUNCH(1, s, launch_attn_bwd_dq_simt(sh, qr, kb, vb, dout, lse, delta, dq, s), "attn_bwd_dq");
+    MAGLEV_LAUNCH(1, s, launch_attn_bwd_dkdv_simt(sh, qr, kb, vb, dout, lse, delta, dkb, dvb, s),
+                  "attn_bwd_dkdv");
+  }
   MAGLEV_LAUNCH(1, s, launch_unmix(sh, dkb, dvb, k, v, R_k, R_v, gate_logits, dk, dv, dR_k, dR_v,
-                                   accumulate_dR ? 1 : 0, gpart, s),
+                                   accumulate_dR ? 1 : 0, gpart, dq_acc, dq, s),
                 "unmix");
   if (d->inject) {
     MAGLEV_LAUNCH(1, s, launch_gate_reduce(d->B * d->T, d->H, gpart, gate_logits, dgate_logits, s),

@@ -49,7 +49,8 @@ cudaError_t launch_attn_bwd_dkdv_simt(const SwaShape& s, const void* q_rot, cons
 cudaError_t launch_unmix(const SwaShape& s, const float* dk_bar, const float* dv_bar,
                          const void* k, const void* v, const void* Rk, const void* Rv,
                          const float* gates, void* dk, void* dv, void* dRk, void* dRv,
-                         int accumulate, float* gpart, cudaStream_t st);
+                         int accumulate, float* gpart, const float* dq_acc, void* dq,
+                         cudaStream_t st);
 cudaError_t launch_gate_reduce(int rows, int H, const float* gpart, const float* gates,
                                float* dgate, cudaStream_t st);
 
@@ -85,12 +86,18 @@ cudaError_t launch_proj_bwd_dw_tc(int64_t M, int D, int d, const void* dRk, cons
                                   int* err, cudaStream_t s);
 int num_sms();
 
+// tcgen05 banded attention backward: dk_bar, dv_bar (fp32) and the rotated-frame
+// dq accumulated with fp32 atomics into dq_acc (zeroed by the launcher).
+cudaError_t launch_attn_bwd_tc(const SwaShape& s, const void* q_rot, const void* k_bar, const void* v_bar,
+                               const void* dout, const float* lse, const float* delta, float* dq_acc,
+                               float* dk_bar, float* dv_bar, int64_t spin_limit, int* err, cudaStream_t st);
+
 // tcgen05 banded attention forward on the saved bf16 q_rot / k_bar / v_bar.
 cudaError_t launch_attn_fwd_tc(const SwaShape& s, const void* q_rot, const void* k_bar, const void* v_bar,
                                void* out, float* lse, int64_t spin_limit, int* err, cudaStream_t st);
 
-// Default bound on the polls of one in-kernel wait (about a second).
-constexpr int64_t DEFAULT_SPIN_LIMIT = (int64_t)1 << 22;
+// Default bound of one in-kernel wait, in microseconds of GPU time (1 s).
+constexpr int64_t DEFAULT_SPIN_LIMIT = 1000000;
 
 // Sets the calling thread's message returned by maglev_last_error().
 void set_last_error(const char* msg);

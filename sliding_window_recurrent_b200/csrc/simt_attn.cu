@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(256) unmix_kernel(
     const T* __restrict__ k, const T* __restrict__ v, const T* __restrict__ Rk,
     const T* __restrict__ Rv, const float* __restrict__ gates, T* __restrict__ dk,
     T* __restrict__ dv, T* __restrict__ dRk, T* __restrict__ dRv, int accumulate,
-    float* __restrict__ gpart) {
+    float* __restrict__ gpart, const float* __restrict__ dq_acc, T* __restrict__ dq) {
   constexpr int NP = HD / 64, HALF = HD / 2;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t row = (int64_t)blockIdx.x * 8 + warp;
@@ -375,6 +375,15 @@ __global__ void __launch_bounds__(256) unmix_kernel(
   float cs[NP], sn[NP];
 #pragma unroll
   for (int r = 0; r < NP; ++r) rope_cos_sin(p, lane + 32 * r, HD, s.log2_base, &cs[r], &sn[r]);
+  if (dq_acc) {  // dq = RoPE^T(dq_rot), dq_rot accumulated in fp32 by the attention backward
+#pragma unroll
+    for (int r = 0; r < NP; ++r) {
+      const int c = lane + 32 * r;
+      const float x1 = dq_acc[base + c], x2 = dq_acc[base + c + HALF];
+      dq[base + c] = from_f<T>(x1 * cs[r] + x2 * sn[r]);
+      dq[base + c + HALF] = from_f<T>(-x1 * sn[r] + x2 * cs[r]);
+    }
+  }
   float d1[NP], d2[NP];  // dk_bar pairs
 #pragma unroll
   for (int r = 0; r < NP; ++r) {
@@ -545,11 +554,12 @@ cudaError_t launch_attn_bwd_dkdv_simt(const SwaShape& s, const void* q_rot, cons
 cudaError_t launch_unmix(const SwaShape& s, const float* dk_bar, const float* dv_bar,
                          const void* k, const void* v, const void* Rk, const void* Rv,
                          const float* gates, void* dk, void* dv, void* dRk, void* dRv,
-                         int accumulate, float* gpart, cudaStream_t st) {
+                         int accumulate, float* gpart, const float* dq_acc, void* dq,
+                         cudaStream_t st) {
   MAGLEV_DISPATCH(s.dtype, s.hd,
                   unmix_kernel<T, HD><<<rows_blocks(s), 256, 0, st>>>(
                       s, dk_bar, dv_bar, (const T*)k, (const T*)v, (const T*)Rk, (const T*)Rv,
-                      gates, (T*)dk, (T*)dv, (T*)dRk, (T*)dRv, accumulate, gpart));
+                      gates, (T*)dk, (T*)dv, (T*)dRk, (T*)dRv, accumulate, gpart, dq_acc, (T*)dq));
   return cudaGetLastError();
 }
 

@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const Abort ab{abort_flag, p.err, p.spin_limit};
+  const Abort ab{abort_flag, p.err, p.spin_limit * 1000};
   const int i0 = blockIdx.x * 128, h = blockIdx.y, b = blockIdx.z;
   const int first_key = max(0, i0 - p.W + 1);
   const int last_key = min(p.T - 1, i0 + 127);
@@ -127,9 +127,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tma_load_4d(smem + C::OFF_V + buf * C::TILE + c * C::CHUNK, &tmV, &kv_full[buf], 64 * c, h, kt, b);
         }
       }
-      if (armed_q) mbar_drain(q_full, 0, p.spin_limit);
+      if (armed_q) mbar_drain(q_full, 0, DRAIN_LIMIT_NS);
       for (int s = 0; s < 2; ++s)
-        if (armed_kv & (1u << s)) mbar_drain(&kv_full[s], (par_kv >> s) & 1u, p.spin_limit);
+        if (armed_kv & (1u << s)) mbar_drain(&kv_full[s], (par_kv >> s) & 1u, DRAIN_LIMIT_NS);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mma_commit(&pv_done[j & 1]);
       }
       mma_commit(drain);
-      mbar_drain(drain, 0, p.spin_limit);
+      mbar_drain(drain, 0, DRAIN_LIMIT_NS);
     }
   } else {
     // -------------------------------------------------------------- softmax / epilogue
@@ -193,7 +193,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       const int buf = j & 1;
-      if (!mbar_wait(&s_full[buf], (uint32_t)(j >> 1) & 1u, ab)) {
+      if (!warp_wait(&s_full[buf], (uint32_t)(j >> 1) & 1u, ab)) {
         ok = false;
         break;
       }
@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         m_ref = mt;
       }
       if (j >= 2) {  // P buffer `buf` was read by PV_{j-2}
-        if (!mbar_wait(&pv_done[buf], (uint32_t)((j - 2) >> 1) & 1u, ab)) {
+        if (!warp_wait(&pv_done[buf], (uint32_t)((j - 2) >> 1) & 1u, ab)) {
           ok = false;
           break;
         }
@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       l = l * alpha + rs;
       if (__any_sync(0xffffffffu, rescale)) {  // O must hold PV_{j-1} before it is scaled
-        if (!mbar_wait(&pv_done[buf ^ 1], (uint32_t)((j - 1) >> 1) & 1u, ab)) {
+        if (!warp_wait(&pv_done[buf ^ 1], (uint32_t)((j - 1) >> 1) & 1u, ab)) {
           ok = false;
           break;
         }
@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_arrive(p_full);
     }
     const int last = n_tiles - 1;
-    if (ok && n_tiles > 0 && mbar_wait(&pv_done[last & 1], (uint32_t)(last >> 1) & 1u, ab)) {
+    if (__all_sync(0xffffffffu, ok) && n_tiles > 0 && warp_wait(&pv_done[last & 1], (uint32_t)(last >> 1) & 1u, ab)) {
       tc_fence_after();
       const float inv = 1.f / l;
       bf16* dst = static_cast<bf16*>(p.out) + (((int64_t)b * p.T + i) * p.H + h) * HD;

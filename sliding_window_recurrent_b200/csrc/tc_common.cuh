@@ -41,35 +41,59 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
   return done != 0;
 }
 
-// Shared abort state of one CTA: a timed-out wait sets `flag` and records
-// MAGLEV_ERR_TIMEOUT in the device status word; every role then stops.
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Shared abort state of one CTA: a wait that outlives `limit_ns` sets `flag`
+// and records MAGLEV_ERR_TIMEOUT in the device status word; every role then
+// stops issuing work.
 struct Abort {
   volatile int* flag;
   int* err;
-  int64_t limit;
+  int64_t limit_ns;
 };
 
-// Waits for the phase of parity `parity` of `bar` to complete, polling at most
-// ab.limit times. Returns false (and raises the abort flag) on expiry, or at
-// once when another role has aborted.
+// Bound of the waits that drain in-flight copies / MMAs before a CTA exits.
+constexpr int64_t DRAIN_LIMIT_NS = 2000000000LL;
+
+// Waits for the phase of parity `parity` of `bar` to complete. Returns false
+// (and raises the abort flag) once ab.limit_ns of GPU time have passed, or
+// soon after another role has aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Abort& ab) {
   const uint32_t addr = smem_u32(bar);
-  for (int64_t i = 0;; ++i) {
+  if (mbar_try_wait(addr, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(addr, parity)) return true;
-    if ((i & 255) == 255 && *ab.flag) return false;
-    if (i >= ab.limit) {
-      *ab.flag = 1;
-      record_error(ab.err, DEV_TIMEOUT);
-      return false;
+    if ((i & 63) == 0) {
+      if (*ab.flag) return false;
+      if ((int64_t)(global_ns() - t0) > ab.limit_ns) {
+        *ab.flag = 1;
+        record_error(ab.err, DEV_TIMEOUT);
+        return false;
+      }
     }
   }
 }
 
+// mbar_wait for a whole warp whose next step is a warp-collective tcgen05.ld /
+// st: the result is the same on every lane (false if any lane gave up).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const Abort& ab) {
+  const bool ok = mbar_wait(bar, parity, ab);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // Bounded wait used while draining on exit; never raises the abort flag.
-__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, int64_t limit) {
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, int64_t limit_ns) {
   const uint32_t addr = smem_u32(bar);
-  for (int64_t i = 0; i < limit; ++i)
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 0;; ++i) {
     if (mbar_try_wait(addr, parity)) return;
+    if ((i & 63) == 0 && (int64_t)(global_ns() - t0) > limit_ns) return;
+  }
 }
 
 // ---------------------------------------------------------------- TMA

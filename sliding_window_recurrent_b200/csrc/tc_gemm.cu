@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const Abort ab{abort_flag, p.err, p.spin_limit};
+  const Abort ab{abort_flag, p.err, p.spin_limit * 1000};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       // every armed stage's last load must land before the CTA may exit
       for (int s = 0; s < STAGES; ++s)
-        if (armed & (1u << s)) mbar_drain(&full[s], (armed_parity >> s) & 1u, p.spin_limit);
+        if (armed & (1u << s)) mbar_drain(&full[s], (armed_parity >> s) & 1u, DRAIN_LIMIT_NS);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       // all issued MMAs must finish before TMEM is released
       mma_commit(drain);
-      mbar_drain(drain, 0, p.spin_limit);
+      mbar_drain(drain, 0, DRAIN_LIMIT_NS);
     }
   } else {
     // -------------------------------------------------------------- epilogue
@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
       const int tm = t % p.tiles_m, tn = t / p.tiles_m;
       int m0 = tm * BM, n0 = tn * BN;
-      if (!mbar_wait(&tfull[acc], acc_phase, ab)) break;
+      if (!warp_wait(&tfull[acc], acc_phase, ab)) break;
       tc_fence_after();
       const int gm = m0 + row;
       bf16* out = static_cast<bf16*>(p.out0);
