@@ -313,7 +313,8 @@ def run_decode_bench(torch, dev, steps, warmup, peaks):
     bf = torch.bfloat16
     kr = [torch.randn(B, H, W, hd, generator=gen, device=dev, dtype=torch.float32).to(bf) for _ in range(L)]
     vr = [torch.randn(B, H, W, hd, generator=gen, device=dev, dtype=torch.float32).to(bf) for _ in range(L)]
-    wqkv = [[(torch.randn(D, d, generator=gen, device=dev) / d ** 0.5).to(bf) for _ in range(3)] for _ in range(L)]
+    # per-layer stand-in projection weights, [3, d, D]: q | k | v = RMSNorm(h) W[i]
+    wqkv = [(torch.randn(3, d, D, generator=gen, device=dev) / d ** 0.5).to(bf) for _ in range(L)]
     gates = [(torch.rand(4, H, generator=gen, device=dev) * 4 - 2) for _ in range(L)]
     wk = (torch.randn(D, d, generator=gen, device=dev) / d ** 0.5).to(bf)
     wv = (torch.randn(D, d, generator=gen, device=dev) / d ** 0.5).to(bf)
@@ -328,8 +329,9 @@ def run_decode_bench(torch, dev, steps, warmup, peaks):
         h = torch.index_select(h_bank, 0, torch.remainder(it, 16).view(1))[0].float()
         for l in range(L):
             xn = torch.nn.functional.rms_norm(h, (d,), eps=1e-6).to(bf)
-            q, k, v = ((xn @ w.t()).view(B, H, hd) for w in wqkv[l])
-            o = S.step(pos, q, k, v, gates[l], kr[l], vr[l])
+            qkv = torch.matmul(xn, wqkv[l])          # [3, B, D], one batched GEMM
+            o = S.step(pos, qkv[0].view(B, H, hd), qkv[1].view(B, H, hd), qkv[2].view(B, H, hd),
+                       gates[l], kr[l], vr[l])
             h = h + o.view(B, D).float()
         m_prev.copy_(torch.nn.functional.rms_norm(h, (d,), eps=1e-6).to(bf))
         pos.add_(1)

@@ -481,13 +481,12 @@ maglev_status maglev_inject_swa_bwd(const maglev_swa_desc* d, const void* k, con
   float* dkb = at<float>(workspace, Wk.dkb);
   float* dvb = at<float>(workspace, Wk.dvb);
   float* gpart = at<float>(workspace, Wk.gpart);
-  MAGLEV_LAUNCH(1, s, launch_attn_delta(sh, out, dout, delta, s), "attn_delta");
-  float* dq_acc = nullptr;
+  float* dq_acc = d->dtype == MAGLEV_BF16 ? at<float>(workspace, Wk.dq_acc) : nullptr;
+  MAGLEV_LAUNCH(1, s, launch_attn_delta(sh, out, dout, delta, dq_acc, s), "attn_delta");
   if (d->dtype == MAGLEV_BF16) {
     int* err = nullptr;
     st = status_word(&err);
     if (st != MAGLEV_OK) return st;
-    dq_acc = at<float>(workspace, Wk.dq_acc);
     MAGLEV_LAUNCH(1, s, launch_attn_bwd_tc(sh, qr, kb, vb, dout, lse, delta, dq_acc, dkb, dvb,
                                            spin_limit_of(d->spin_limit), err, s),
                   "attn_bwd_tc");
@@ -500,7 +499,7 @@ maglev_status maglev_inject_swa_bwd(const maglev_swa_desc* d, const void* k, con
                                    accumulate_dR ? 1 : 0, gpart, dq_acc, dq, s),
                 "unmix");
   if (d->inject) {
-    MAGLEV_LAUNCH(1, s, launch_gate_reduce(d->B * d->T, d->H, gpart, gate_logits, dgate_logits, s),
+    MAGLEV_LAUNCH(1, s, launch_gate_reduce((int64_t)d->B * d->T, d->H, gpart, gate_logits, dgate_logits, s),
                   "gate_reduce");
     if (m_shift) {
       st = run_mem_project_bwd(d, m_shift, w_mk, w_mv, dR_k, dR_v, dm_shift, dw_mk, dw_mv, s);
@@ -602,6 +601,16 @@ maglev_status maglev_decode_mem_project(const maglev_decode_desc* d, const int64
   if (d->B == 0) return MAGLEV_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t D = (int64_t)d->H * d->hd, K = d->d_mem;
+  if (d->dtype == MAGLEV_BF16 && K % 8 == 0 && D % 256 == 0) {
+    int* err = nullptr;
+    st = status_word(&err);
+    if (st != MAGLEV_OK) return st;
+    MAGLEV_LAUNCH(1, s, launch_proj_fwd_tc(d->B, (int)D, (int)K, m_prev, w_mk, w_mv, krec_rot, vrec,
+                                           spin_limit_of(d->spin_limit), err, s),
+                  "decode_mem_project_tc");
+    MAGLEV_LAUNCH(1, s, launch_rmsnorm_rope_rows(dec_shape(d), pos, krec_rot, s), "decode_krec_norm_rope");
+    return MAGLEV_OK;
+  }
   for (int which = 0; which < 2; ++which) {
     GemmArgs g{};
     g.M = d->B;
@@ -643,8 +652,11 @@ maglev_status maglev_decode_step(const maglev_decode_desc* d, const int64_t* pos
   }
   if (d->B == 0) return MAGLEV_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* err = nullptr;
+  st = status_word(&err);
+  if (st != MAGLEV_OK) return st;
   MAGLEV_LAUNCH(1, s, launch_decode_step(dec_shape(d), pos, q, k, v, krec_rot, vrec, gate_logits, k_ring,
-                                          v_ring, out, s),
+                                          v_ring, out, spin_limit_of(d->spin_limit), err, s),
                 "decode_step");
   return MAGLEV_OK;
 }

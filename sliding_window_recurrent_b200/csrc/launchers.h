@@ -33,9 +33,9 @@ cudaError_t launch_prep(const SwaShape& s, const void* q, const void* k, const v
                         void* k_bar, void* v_bar, cudaStream_t st);
 cudaError_t launch_attn_fwd_simt(const SwaShape& s, const void* q_rot, const void* k_bar,
                                  const void* v_bar, void* out, float* lse, cudaStream_t st);
-// delta[b,h,i] = dout_i . out_i
+// delta[b,h,i] = dout_i . out_i; zeroes dq_acc ([B,T,H,hd] fp32) when non-null.
 cudaError_t launch_attn_delta(const SwaShape& s, const void* out, const void* dout, float* delta,
-                              cudaStream_t st);
+                              float* dq_acc, cudaStream_t st);
 // dq = RoPE^T(dq_rot) written in dtype.
 cudaError_t launch_attn_bwd_dq_simt(const SwaShape& s, const void* q_rot, const void* k_bar,
                                     const void* v_bar, const void* dout, const float* lse,
@@ -45,13 +45,14 @@ cudaError_t launch_attn_bwd_dkdv_simt(const SwaShape& s, const void* q_rot, cons
                                       const void* v_bar, const void* dout, const float* lse,
                                       const float* delta, float* dk_bar, float* dv_bar,
                                       cudaStream_t st);
-// dk, dv, dR_k, dR_v and per-row gate partials gpart[B*T][4][H] from dk_bar, dv_bar.
+// dk, dv, dR_k, dR_v (and dq from dq_acc when non-null) and per-row gate
+// partials gpart[(g*H + h) * B*T + row] from dk_bar, dv_bar.
 cudaError_t launch_unmix(const SwaShape& s, const float* dk_bar, const float* dv_bar,
                          const void* k, const void* v, const void* Rk, const void* Rv,
                          const float* gates, void* dk, void* dv, void* dRk, void* dRv,
                          int accumulate, float* gpart, const float* dq_acc, void* dq,
                          cudaStream_t st);
-cudaError_t launch_gate_reduce(int rows, int H, const float* gpart, const float* gates,
+cudaError_t launch_gate_reduce(int64_t rows, int H, const float* gpart, const float* gates,
                                float* dgate, cudaStream_t st);
 
 int loss_partial_blocks(int64_t n);
@@ -69,7 +70,7 @@ cudaError_t launch_rmsnorm_rope_rows(const DecShape& s, const int64_t* pos, void
 cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void* q, const void* k,
                                const void* v, const void* krec, const void* vrec,
                                const float* gates, void* k_ring, void* v_ring, void* out,
-                               cudaStream_t st);
+                               int64_t limit_us, int* err, cudaStream_t st);
 
 // tcgen05 projection GEMMs (bf16 in/out, fp32 accumulation in TMEM).
 // R_k | R_v [M, D] = m_shift [M, d] x [W_mk; W_mv]^T. Needs d % 8 == 0, D % 256 == 0.

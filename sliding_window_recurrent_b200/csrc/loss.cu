@@ -11,6 +11,32 @@ namespace {
 constexpr int LOSS_THREADS = 256;
 constexpr int LOSS_MAX_BLOCKS = 1184;  // 8 x 148 SMs
 
+__device__ __forceinline__ void load8f(const bf16* p, float* x) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void load8f(const float* p, float* x) {
+  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+__device__ __forceinline__ void store8f(bf16* p, const float* x) {
+  uint4 u;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+__device__ __forceinline__ void store8f(float* p, const float* x) {
+  *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+  *reinterpret_cast<float4*>(p + 4) = make_float4(x[4], x[5], x[6], x[7]);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(LOSS_THREADS) loss_partial_kernel(
     const T* __restrict__ m, const T* __restrict__ mt, int64_t n, int64_t chunk, float scale_grad,
@@ -19,12 +45,32 @@ __global__ void __launch_bounds__(LOSS_THREADS) loss_partial_kernel(
   const int64_t lo = (int64_t)blockIdx.x * chunk;
   const int64_t hi = min(n, lo + chunk);
   float acc = 0.f;
-  for (int64_t i = lo + threadIdx.x; i < hi; i += LOSS_THREADS) {
-    const float diff = to_f(m[i]) - to_f(mt[i]);
-    acc = fmaf(diff, diff, acc);
-    const float g = scale_grad * diff;
-    if (dm) dm[i] = from_f<T>(accumulate ? to_f(dm[i]) + g : g);
-    if (dmt) dmt[i] = from_f<T>(-g);
+  if ((chunk & 7) == 0 && (n & 7) == 0) {
+    // 8 elements (16 or 32 bytes) per step; chunk boundaries stay 8-aligned
+    for (int64_t i = lo + 8 * threadIdx.x; i < hi; i += 8 * LOSS_THREADS) {
+      float a[8], b[8], d[8];
+      load8f(m + i, a);
+      load8f(mt + i, b);
+      if (dm && accumulate) load8f(dm + i, d);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float diff = a[e] - b[e];
+        acc = fmaf(diff, diff, acc);
+        const float g = scale_grad * diff;
+        a[e] = (dm && accumulate) ? d[e] + g : g;
+        b[e] = -g;
+      }
+      if (dm) store8f(dm + i, a);
+      if (dmt) store8f(dmt + i, b);
+    }
+  } else {
+    for (int64_t i = lo + threadIdx.x; i < hi; i += LOSS_THREADS) {
+      const float diff = to_f(m[i]) - to_f(mt[i]);
+      acc = fmaf(diff, diff, acc);
+      const float g = scale_grad * diff;
+      if (dm) dm[i] = from_f<T>(accumulate ? to_f(dm[i]) + g : g);
+      if (dmt) dmt[i] = from_f<T>(-g);
+    }
   }
   acc = warp_sum(acc);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x / 32] = acc;
@@ -66,7 +112,7 @@ cudaError_t launch_consistency_loss(const void* m, const void* mt, int64_t rows,
                                     void* dmt, int accumulate, float* partials, cudaStream_t st) {
   const int64_t n = rows * (int64_t)d;
   const int nblk = loss_partial_blocks(n);
-  const int64_t chunk = (n + nblk - 1) / nblk;
+  const int64_t chunk = (((n + nblk - 1) / nblk) + 7) & ~(int64_t)7;
   if (dtype == 1)
     loss_partial_kernel<bf16><<<nblk, LOSS_THREADS, 0, st>>>(
         (const bf16*)m, (const bf16*)mt, n, chunk, scale_grad, (bf16*)dm, (bf16*)dmt, accumulate,

@@ -1,6 +1,7 @@
-// CUDA-core kernels of the injected sliding-window attention layer: the
-// element-wise injection (RoPE of both keys, RMSNorm of the memory key, gated
-// mix), the fp32 attention forward/backward, and the un-mix of the gradients.
+// CUDA-core kernels of the injected sliding-window attention layer for the
+// fp32 path: banded attention forward and backward (dq, dk_bar / dv_bar) on
+// the saved rotated / mixed entries. The element-wise injection and un-mix
+// live in ew.cu.
 //
 // Source: "Maglev: Sliding Recurrent Memory", paper.rainbus.top, sections
 // 前置知识 (SWA over the most recent W tokens; RoPE rotation of q and k) and
@@ -17,80 +18,6 @@ namespace maglev {
 namespace {
 
 constexpr unsigned FULL = 0xffffffffu;
-
-// ---------------------------------------------------------------------------
-// a2-a4: q_rot = RoPE(q); k_bar = g_kl RoPE(k) + g_kr RoPE(RMSNorm(R_k));
-// v_bar = g_vl v + g_vr R_v. One warp per (b,t,h); lane owns pairs
-// (c, c + hd/2) for c = lane + 32 r.
-// ---------------------------------------------------------------------------
-template <typename T, int HD>
-__global__ void __launch_bounds__(256) prep_kernel(SwaShape s, const T* __restrict__ q,
-                                                   const T* __restrict__ k,
-                                                   const T* __restrict__ v,
-                                                   const T* __restrict__ Rk,
-                                                   const T* __restrict__ Rv,
-                                                   const float* __restrict__ gates,
-                                                   T* __restrict__ qr, T* __restrict__ kb,
-                                                   T* __restrict__ vb) {
-  constexpr int NP = HD / 64, HALF = HD / 2;
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int64_t row = (int64_t)blockIdx.x * 8 + warp;
-  if (row >= (int64_t)s.B * s.T * s.H) return;
-  const int h = (int)(row % s.H);
-  const int t = (int)((row / s.H) % s.T);
-  const int64_t p = (int64_t)s.pos0 + t;
-  const int64_t base = row * HD;
-  float cs[NP], sn[NP];
-#pragma unroll
-  for (int r = 0; r < NP; ++r) rope_cos_sin(p, lane + 32 * r, HD, s.log2_base, &cs[r], &sn[r]);
-#pragma unroll
-  for (int r = 0; r < NP; ++r) {
-    const int c = lane + 32 * r;
-    float x1 = to_f(q[base + c]), x2 = to_f(q[base + c + HALF]);
-    qr[base + c] = from_f<T>(x1 * cs[r] - x2 * sn[r]);
-    qr[base + c + HALF] = from_f<T>(x1 * sn[r] + x2 * cs[r]);
-  }
-  float kl1[NP], kl2[NP];
-#pragma unroll
-  for (int r = 0; r < NP; ++r) {
-    const int c = lane + 32 * r;
-    float x1 = to_f(k[base + c]), x2 = to_f(k[base + c + HALF]);
-    kl1[r] = x1 * cs[r] - x2 * sn[r];
-    kl2[r] = x1 * sn[r] + x2 * cs[r];
-  }
-  if (!s.inject) {
-#pragma unroll
-    for (int r = 0; r < NP; ++r) {
-      const int c = lane + 32 * r;
-      kb[base + c] = from_f<T>(kl1[r]);
-      kb[base + c + HALF] = from_f<T>(kl2[r]);
-      vb[base + c] = v[base + c];
-      vb[base + c + HALF] = v[base + c + HALF];
-    }
-    return;
-  }
-  const float gkl = gate_value(gates[0 * s.H + h]), gkr = gate_value(gates[1 * s.H + h]);
-  const float gvl = gate_value(gates[2 * s.H + h]), gvr = gate_value(gates[3 * s.H + h]);
-  float r1[NP], r2[NP], ss = 0.f;
-#pragma unroll
-  for (int r = 0; r < NP; ++r) {
-    const int c = lane + 32 * r;
-    r1[r] = to_f(Rk[base + c]);
-    r2[r] = to_f(Rk[base + c + HALF]);
-    ss += r1[r] * r1[r] + r2[r] * r2[r];
-  }
-  const float rinv = rsqrtf(warp_sum(ss) / HD + s.eps);
-#pragma unroll
-  for (int r = 0; r < NP; ++r) {
-    const int c = lane + 32 * r;
-    const float n1 = r1[r] * rinv, n2 = r2[r] * rinv;
-    const float kr1 = n1 * cs[r] - n2 * sn[r], kr2 = n1 * sn[r] + n2 * cs[r];
-    kb[base + c] = from_f<T>(gkl * kl1[r] + gkr * kr1);
-    kb[base + c + HALF] = from_f<T>(gkl * kl2[r] + gkr * kr2);
-    vb[base + c] = from_f<T>(gvl * to_f(v[base + c]) + gvr * to_f(Rv[base + c]));
-    vb[base + c + HALF] = from_f<T>(gvl * to_f(v[base + c + HALF]) + gvr * to_f(Rv[base + c + HALF]));
-  }
-}
 
 // ---------------------------------------------------------------------------
 // a5 forward: one warp per query row i, 8 rows per block sharing 32-key tiles
@@ -163,23 +90,6 @@ __global__ void __launch_bounds__(256) attn_fwd_kernel(SwaShape s, const T* __re
     for (int r = 0; r < NC; ++r) out[rowp(i) + lane + 32 * r] = from_f<T>(acc[r] * inv);
     if (lane == 0) lse[((int64_t)b * H + h) * T_ + i] = m + logf(l);
   }
-}
-
-// delta[b,h,i] = sum_c dout[b,i,h,c] * out[b,i,h,c]
-template <typename T>
-__global__ void __launch_bounds__(256) delta_kernel(SwaShape s, const T* __restrict__ out,
-                                                    const T* __restrict__ dout,
-                                                    float* __restrict__ delta) {
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int64_t row = (int64_t)blockIdx.x * 8 + warp;
-  if (row >= (int64_t)s.B * s.T * s.H) return;
-  const int h = (int)(row % s.H);
-  const int64_t bt = row / s.H;
-  const int t = (int)(bt % s.T), b = (int)(bt / s.T);
-  float acc = 0.f;
-  for (int c = lane; c < s.hd; c += 32) acc += to_f(out[row * s.hd + c]) * to_f(dout[row * s.hd + c]);
-  acc = warp_sum(acc);
-  if (lane == 0) delta[((int64_t)b * s.H + h) * s.T + t] = acc;
 }
 
 // ---------------------------------------------------------------------------
@@ -346,141 +256,6 @@ __global__ void __launch_bounds__(256) attn_bwd_dkdv_kernel(
   }
 }
 
-// ---------------------------------------------------------------------------
-// a6 un-mix: from dk_bar, dv_bar to dk, dv, dR_k (through RoPE^T and the
-// RMSNorm backward), dR_v, and per-row partial sums of the gate gradients.
-// ---------------------------------------------------------------------------
-template <typename T>
-__device__ __forceinline__ void store_acc(T* p, int64_t i, float x, int accumulate) {
-  if (accumulate) x += to_f(p[i]);
-  p[i] = from_f<T>(x);
-}
-
-template <typename T, int HD>
-__global__ void __launch_bounds__(256) unmix_kernel(
-    SwaShape s, const float* __restrict__ dkb, const float* __restrict__ dvb,
-    const T* __restrict__ k, const T* __restrict__ v, const T* __restrict__ Rk,
-    const T* __restrict__ Rv, const float* __restrict__ gates, T* __restrict__ dk,
-    T* __restrict__ dv, T* __restrict__ dRk, T* __restrict__ dRv, int accumulate,
-    float* __restrict__ gpart, const float* __restrict__ dq_acc, T* __restrict__ dq) {
-  constexpr int NP = HD / 64, HALF = HD / 2;
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int64_t row = (int64_t)blockIdx.x * 8 + warp;
-  if (row >= (int64_t)s.B * s.T * s.H) return;
-  const int h = (int)(row % s.H);
-  const int64_t bt = row / s.H;
-  const int t = (int)(bt % s.T);
-  const int64_t p = (int64_t)s.pos0 + t;
-  const int64_t base = row * HD;
-  float cs[NP], sn[NP];
-#pragma unroll
-  for (int r = 0; r < NP; ++r) rope_cos_sin(p, lane + 32 * r, HD, s.log2_base, &cs[r], &sn[r]);
-  if (dq_acc) {  // dq = RoPE^T(dq_rot), dq_rot accumulated in fp32 by the attention backward
-#pragma unroll
-    for (int r = 0; r < NP; ++r) {
-      const int c = lane + 32 * r;
-      const float x1 = dq_acc[base + c], x2 = dq_acc[base + c + HALF];
-      dq[base + c] = from_f<T>(x1 * cs[r] + x2 * sn[r]);
-      dq[base + c + HALF] = from_f<T>(-x1 * sn[r] + x2 * cs[r]);
-    }
-  }
-  float d1[NP], d2[NP];  // dk_bar pairs
-#pragma unroll
-  for (int r = 0; r < NP; ++r) {
-    d1[r] = dkb[base + lane + 32 * r];
-    d2[r] = dkb[base + lane + 32 * r + HALF];
-  }
-  if (!s.inject) {
-#pragma unroll
-    for (int r = 0; r < NP; ++r) {
-      const int c = lane + 32 * r;
-      dk[base + c] = from_f<T>(d1[r] * cs[r] + d2[r] * sn[r]);
-      dk[base + c + HALF] = from_f<T>(-d1[r] * sn[r] + d2[r] * cs[r]);
-      dv[base + c] = from_f<T>(dvb[base + c]);
-      dv[base + c + HALF] = from_f<T>(dvb[base + c + HALF]);
-    }
-    return;
-  }
-  const float gkl = gate_value(gates[0 * s.H + h]), gkr = gate_value(gates[1 * s.H + h]);
-  const float gvl = gate_value(gates[2 * s.H + h]), gvr = gate_value(gates[3 * s.H + h]);
-  float r1[NP], r2[NP], ss = 0.f;
-#pragma unroll
-  for (int r = 0; r < NP; ++r) {
-    r1[r] = to_f(Rk[base + lane + 32 * r]);
-    r2[r] = to_f(Rk[base + lane + 32 * r + HALF]);
-    ss += r1[r] * r1[r] + r2[r] * r2[r];
-  }
-  const float rinv = rsqrtf(warp_sum(ss) / HD + s.eps);
-  float s_kl = 0.f, s_kr = 0.f, s_vl = 0.f, s_vr = 0.f, s_ndn = 0.f;
-  float n1[NP], n2[NP], dn1[NP], dn2[NP];
-#pragma unroll
-  for (int r = 0; r < NP; ++r) {
-    const int c = lane + 32 * r;
-    // local key and its gradient
-    const float k1 = to_f(k[base + c]), k2 = to_f(k[base + c + HALF]);
-    const float kl1 = k1 * cs[r] - k2 * sn[r], kl2 = k1 * sn[r] + k2 * cs[r];
-    s_kl += d1[r] * kl1 + d2[r] * kl2;
-    const float bk1 = d1[r] * cs[r] + d2[r] * sn[r];   // RoPE^T dk_bar
-    const float bk2 = -d1[r] * sn[r] + d2[r] * cs[r];
-    dk[base + c] = from_f<T>(gkl * bk1);
-    dk[base + c + HALF] = from_f<T>(gkl * bk2);
-    // memory key
-    n1[r] = r1[r] * rinv;
-    n2[r] = r2[r] * rinv;
-    const float kr1 = n1[r] * cs[r] - n2[r] * sn[r], kr2 = n1[r] * sn[r] + n2[r] * cs[r];
-    s_kr += d1[r] * kr1 + d2[r] * kr2;
-    dn1[r] = gkr * bk1;
-    dn2[r] = gkr * bk2;
-    s_ndn += n1[r] * dn1[r] + n2[r] * dn2[r];
-    // values
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int cc = c + u * HALF;
-      const float dvv = dvb[base + cc];
-      s_vl += dvv * to_f(v[base + cc]);
-      s_vr += dvv * to_f(Rv[base + cc]);
-      store_acc(dv, base + cc, gvl * dvv, 0);
-      store_acc(dRv, base + cc, gvr * dvv, accumulate);
-    }
-  }
-  const float mean_ndn = warp_sum(s_ndn) / HD;
-#pragma unroll
-  for (int r = 0; r < NP; ++r) {
-    const int c = lane + 32 * r;
-    store_acc(dRk, base + c, (dn1[r] - n1[r] * mean_ndn) * rinv, accumulate);
-    store_acc(dRk, base + c + HALF, (dn2[r] - n2[r] * mean_ndn) * rinv, accumulate);
-  }
-  s_kl = warp_sum(s_kl);
-  s_kr = warp_sum(s_kr);
-  s_vl = warp_sum(s_vl);
-  s_vr = warp_sum(s_vr);
-  if (lane == 0) {
-    float* g = gpart + bt * 4 * s.H;
-    g[0 * s.H + h] = s_kl;
-    g[1 * s.H + h] = s_kr;
-    g[2 * s.H + h] = s_vl;
-    g[3 * s.H + h] = s_vr;
-  }
-}
-
-// dgate[g,h] = (sum over rows of gpart[row][g][h]) * dg/da, in a fixed order.
-__global__ void __launch_bounds__(256) gate_reduce_kernel(int rows, int H,
-                                                          const float* __restrict__ gpart,
-                                                          const float* __restrict__ gates,
-                                                          float* __restrict__ dgate) {
-  __shared__ float red[256];
-  const int col = blockIdx.x;  // g * H + h
-  float acc = 0.f;
-  for (int r = threadIdx.x; r < rows; r += 256) acc += gpart[(int64_t)r * 4 * H + col];
-  red[threadIdx.x] = acc;
-  __syncthreads();
-  for (int w = 128; w > 0; w >>= 1) {
-    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) dgate[col] = red[0] * gate_slope(gates[col]);
-}
-
 }  // namespace
 
 #define MAGLEV_DISPATCH(DT, HDV, ...)                                 \
@@ -492,19 +267,6 @@ __global__ void __launch_bounds__(256) gate_reduce_kernel(int rows, int H,
     else return cudaErrorInvalidValue;                                \
   } while (0)
 
-static inline unsigned rows_blocks(const SwaShape& s) {
-  return (unsigned)(((int64_t)s.B * s.T * s.H + 7) / 8);
-}
-
-cudaError_t launch_prep(const SwaShape& s, const void* q, const void* k, const void* v,
-                        const void* Rk, const void* Rv, const float* gates, void* q_rot,
-                        void* k_bar, void* v_bar, cudaStream_t st) {
-  MAGLEV_DISPATCH(s.dtype, s.hd,
-                  prep_kernel<T, HD><<<rows_blocks(s), 256, 0, st>>>(
-                      s, (const T*)q, (const T*)k, (const T*)v, (const T*)Rk, (const T*)Rv, gates,
-                      (T*)q_rot, (T*)k_bar, (T*)v_bar));
-  return cudaGetLastError();
-}
 
 cudaError_t launch_attn_fwd_simt(const SwaShape& s, const void* q_rot, const void* k_bar,
                                  const void* v_bar, void* out, float* lse, cudaStream_t st) {
@@ -514,15 +276,6 @@ cudaError_t launch_attn_fwd_simt(const SwaShape& s, const void* q_rot, const voi
                   attn_fwd_kernel<T, HD><<<grid, 256, 0, st>>>(s, (const T*)q_rot, (const T*)k_bar,
                                                                (const T*)v_bar, (T*)out, lse,
                                                                scale));
-  return cudaGetLastError();
-}
-
-cudaError_t launch_attn_delta(const SwaShape& s, const void* out, const void* dout, float* delta,
-                              cudaStream_t st) {
-  if (s.dtype == 1)
-    delta_kernel<bf16><<<rows_blocks(s), 256, 0, st>>>(s, (const bf16*)out, (const bf16*)dout, delta);
-  else
-    delta_kernel<float><<<rows_blocks(s), 256, 0, st>>>(s, (const float*)out, (const float*)dout, delta);
   return cudaGetLastError();
 }
 
@@ -548,24 +301,6 @@ cudaError_t launch_attn_bwd_dkdv_simt(const SwaShape& s, const void* q_rot, cons
                   attn_bwd_dkdv_kernel<T, HD><<<grid, 256, 0, st>>>(
                       s, (const T*)q_rot, (const T*)k_bar, (const T*)v_bar, (const T*)dout, lse,
                       delta, dk_bar, dv_bar, scale));
-  return cudaGetLastError();
-}
-
-cudaError_t launch_unmix(const SwaShape& s, const float* dk_bar, const float* dv_bar,
-                         const void* k, const void* v, const void* Rk, const void* Rv,
-                         const float* gates, void* dk, void* dv, void* dRk, void* dRv,
-                         int accumulate, float* gpart, const float* dq_acc, void* dq,
-                         cudaStream_t st) {
-  MAGLEV_DISPATCH(s.dtype, s.hd,
-                  unmix_kernel<T, HD><<<rows_blocks(s), 256, 0, st>>>(
-                      s, dk_bar, dv_bar, (const T*)k, (const T*)v, (const T*)Rk, (const T*)Rv,
-                      gates, (T*)dk, (T*)dv, (T*)dRk, (T*)dRv, accumulate, gpart, dq_acc, (T*)dq));
-  return cudaGetLastError();
-}
-
-cudaError_t launch_gate_reduce(int rows, int H, const float* gpart, const float* gates,
-                               float* dgate, cudaStream_t st) {
-  gate_reduce_kernel<<<4 * H, 256, 0, st>>>(rows, H, gpart, gates, dgate);
   return cudaGetLastError();
 }
 

@@ -344,8 +344,6 @@ cudaError_t launch_attn_bwd_tc(const SwaShape& s, const void* q_rot, const void*
   if ((e = make_tmap_tokens(&tk, k_bar, s.B, s.T, s.H, s.hd, 128)) != cudaSuccess) return e;
   if ((e = make_tmap_tokens(&tv, v_bar, s.B, s.T, s.H, s.hd, 128)) != cudaSuccess) return e;
   if ((e = make_tmap_tokens(&tdo, dout, s.B, s.T, s.H, s.hd, 128)) != cudaSuccess) return e;
-  const size_t acc_bytes = (size_t)s.B * s.T * s.H * s.hd * sizeof(float);
-  if ((e = cudaMemsetAsync(dq_acc, 0, acc_bytes, st)) != cudaSuccess) return e;
   BwdParams p;
   p.B = s.B;
   p.T = s.T;
