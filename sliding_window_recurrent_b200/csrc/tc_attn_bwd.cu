@@ -10,10 +10,12 @@
 //   dQ_i = dS K -> fp32 vector atomics into a zeroed dQ accumulator
 //   warp 0     TMA: K, V once; Q_i, dO_i per query tile
 //   warp 1     tcgen05.mma issue
-//   warps 2-5  one key row per thread: masked P^T and dS^T in registers,
+//   warps 2-9  two warps per TMEM lane quarter, each taking half of the 128
+//              query columns of a key row: masked P^T and dS^T in registers,
 //              written bf16 128B-swizzled into shared memory (K-major for the
 //              dV / dK MMAs, read back MN-major as dS for the dQ MMA); then
-//              the dQ drain; finally dK, dV rows stored in fp32.
+//              half of the dQ drain; finally dK, dV rows stored in fp32.
+//              LSE and Delta of each query tile are staged in shared memory.
 // Delta = rowsum(dO * O) comes from the delta kernel. Every wait is bounded.
 #include <cuda.h>
 
@@ -28,7 +30,8 @@ namespace {
 
 using namespace tc;
 
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;  // producer, MMA, 8 softmax warps
+constexpr int SOFT_THREADS = 256;
 constexpr float LOG2E = 1.4426950408889634f;
 
 template <int HD>
@@ -43,7 +46,8 @@ struct BwdCfg {
   static constexpr int OFF_DO = 3 * TILE;
   static constexpr int OFF_P = 4 * TILE;
   static constexpr int OFF_DS = 4 * TILE + PT;
-  static constexpr int OFF_BAR = 4 * TILE + 2 * PT;
+  static constexpr int OFF_LD = 4 * TILE + 2 * PT;  // [2][2][128] floats: LSE*log2e, Delta
+  static constexpr int OFF_BAR = OFF_LD + 2 * 2 * 128 * 4;
   static constexpr size_t SMEM = 1024 + OFF_BAR + 256;
   // TMEM columns
   static constexpr uint32_t R_S = 0;     // S^T, later dQ_i
@@ -111,9 +115,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(qdo_full, 1);
     mbar_init(qdo_empty, 1);
     mbar_init(s_full, 1);
-    mbar_init(ds_full, 128);
+    mbar_init(ds_full, SOFT_THREADS);
     mbar_init(dq_full, 1);
-    mbar_init(dq_empty, 128);
+    mbar_init(dq_empty, SOFT_THREADS);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -214,26 +218,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // -------------------------------------------------------------- softmax-backward / drains
     const int q4 = warp & 3;
-    const int r = q4 * 32 + lane;   // TMEM lane: key row (S^T, dV, dK) / query row (dQ)
+    const int half = (warp - 2) >> 2;  // which 64 of the 128 columns this warp takes
+    const int r = q4 * 32 + lane;      // TMEM lane: key row (S^T, dV, dK) / query row (dQ)
+    const int st = threadIdx.x - 64;   // 0..255 among the softmax threads
     const int kj = kt + r;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const int64_t lrow = ((int64_t)b * p.H + h) * p.T;
-    const bool vec_ok = (p.T & 3) == 0;  // 16-byte aligned LSE / Delta rows
+    float* sLD = reinterpret_cast<float*>(smem + C::OFF_LD);
     uint8_t* sPT = smem + C::OFF_P;
     uint8_t* sDS = smem + C::OFF_DS;
     bool ok = true;
+    float pre_l = 0.f, pre_d = 0.f;  // this thread's LSE / Delta entry of the next tile
+    auto fetch = [&](int i) {
+      const int qi = kt + 128 * i + (st & 127);
+      const bool in = qi < p.T;
+      pre_l = in ? p.lse[lrow + qi] * LOG2E : 0.f;
+      pre_d = in ? p.delta[lrow + qi] : 0.f;
+    };
+    fetch(0);
     for (int i = 0; i < n_q; ++i) {
       const uint32_t par = (uint32_t)i & 1u;
       const int qt = kt + 128 * i;
-      if (!warp_wait(s_full, par, ab)) {
-        ok = false;
-        break;
-      }
+      float* lds = sLD + (i & 1) * 256;  // [0,128): LSE*log2e, [128,256): Delta
+      if (st < 128) lds[st] = pre_l;
+      else lds[st] = pre_d;
+      // every softmax thread reaches this barrier on every tile, aborted or not
+      asm volatile("bar.sync 1, %0;" ::"n"(SOFT_THREADS) : "memory");
+      if (i + 1 < n_q) fetch(i + 1);
+      ok = ok && warp_wait(s_full, par, ab);
+      if (!ok) continue;
       tc_fence_after();
-      const int lo = kj - qt;               // first valid column (query >= key)
+      const int lo = kj - qt;  // first valid column (query >= key)
       const int hi = min(kj + p.W - 1, p.T - 1) - qt;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * half + cc;  // 32-column chunk index
         uint32_t sv[32], dv[32];
         tmem_ld32(tmem + lane_off + C::R_S + 32u * (uint32_t)c, sv);
         tmem_ld32(tmem + lane_off + C::R_DP + 32u * (uint32_t)c, dv);
@@ -241,26 +260,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         float pt[32], ds[32];
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
-          const int col0 = 32 * c + 4 * e4;
-          const int qi = qt + col0;
-          float4 L = make_float4(0.f, 0.f, 0.f, 0.f), D = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (vec_ok && qi + 3 < p.T) {
-            L = __ldg(reinterpret_cast<const float4*>(p.lse + lrow + qi));
-            D = __ldg(reinterpret_cast<const float4*>(p.delta + lrow + qi));
-          } else {
-            if (qi + 0 < p.T) { L.x = p.lse[lrow + qi + 0]; D.x = p.delta[lrow + qi + 0]; }
-            if (qi + 1 < p.T) { L.y = p.lse[lrow + qi + 1]; D.y = p.delta[lrow + qi + 1]; }
-            if (qi + 2 < p.T) { L.z = p.lse[lrow + qi + 2]; D.z = p.delta[lrow + qi + 2]; }
-            if (qi + 3 < p.T) { L.w = p.lse[lrow + qi + 3]; D.w = p.delta[lrow + qi + 3]; }
-          }
+          const float4 L = *reinterpret_cast<const float4*>(lds + 32 * c + 4 * e4);
+          const float4 D = *reinterpret_cast<const float4*>(lds + 128 + 32 * c + 4 * e4);
           const float Ls[4] = {L.x, L.y, L.z, L.w};
           const float Ds[4] = {D.x, D.y, D.z, D.w};
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int e = 4 * e4 + u;
-            const int col = col0 + u;
+            const int col = 32 * c + e;
             const bool valid = col >= lo && col <= hi && kj < p.T;
-            const float pe = valid ? exp2f(__uint_as_float(sv[e]) * p.scale_log2 - Ls[u] * LOG2E) : 0.f;
+            const float pe = valid ? exp2f(__uint_as_float(sv[e]) * p.scale_log2 - Ls[u]) : 0.f;
             pt[e] = pe;
             ds[e] = pe * (__uint_as_float(dv[e]) - Ds[u]) * p.scale;
           }
@@ -271,16 +280,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(ds_full);
-      // dQ_i = dS K: lane r is query qt + r
-      if (!warp_wait(dq_full, par, ab)) {
-        ok = false;
-        break;
-      }
+      // dQ_i = dS K: lane r is query qt + r; this warp drains hd columns [64*half, 64*half+64)
+      ok = warp_wait(dq_full, par, ab);
+      if (!ok) continue;
       tc_fence_after();
       const int qi = qt + r;
       float* dst = p.dq_acc + (((int64_t)b * p.T + qi) * p.H + h) * HD;
 #pragma unroll 1
-      for (int c = 0; c < HD / 32; ++c) {
+      for (int c = half * (HD / 64); c < (half + 1) * (HD / 64); ++c) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_off + C::R_S + 32u * (uint32_t)c, v);
         tmem_wait_ld();
@@ -302,7 +309,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool row_ok = kj < p.T;
       const int64_t row = (((int64_t)b * p.T + (row_ok ? kj : 0)) * p.H + h) * HD;
 #pragma unroll 1
-      for (int c = 0; c < HD / 32; ++c) {
+      for (int c = half * (HD / 64); c < (half + 1) * (HD / 64); ++c) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_off + C::R_DK + 32u * (uint32_t)c, v);
         tmem_wait_ld();
