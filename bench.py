@@ -74,6 +74,11 @@ def kernel_work(name: str, cfg: dict) -> tuple[float, str]:
         "attn_bwd_dq": (f["attn_bwd"] * 3 / 5, "flop"),
         "attn_bwd_dkdv": (f["attn_bwd"] * 4 / 5, "flop"),
         "attn_bwd": (f["attn_bwd"], "flop"),
+        "attn_fwd_tc": (f["attn_fwd"], "flop"),
+        "attn_bwd_tc": (f["attn_bwd"], "flop"),
+        "mem_project_tc": (f["proj_fwd"], "flop"),
+        "mem_project_bwd_dm_tc": (f["proj_fwd"], "flop"),
+        "mem_project_bwd_dw_tc": (f["proj_fwd"], "flop"),
         "inject_prep": (B * T * D * 2.0 * (5 + 3), "byte"),
         "unmix": (B * T * D * (4 * 2 + 2 * 4 + 4 * 2.0), "byte"),
         "consistency_loss": (B * T * D * 2.0 * 3, "byte"),
@@ -96,6 +101,23 @@ def src_sha(fname: str) -> str:
     if not os.path.exists(p):
         return ""
     return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+# --------------------------------------------------------------------------- ranks
+def max_over_ranks(dist, x: float, device) -> float:
+    """The largest of every rank's x (identity without a process group)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest
+    rank's time (weak scaling: each replica does the same work)."""
+    return units_per_rank * world / (ms_max * 1e-3)
 
 
 # --------------------------------------------------------------------------- clocks
@@ -232,11 +254,8 @@ def run_layer_bench(torch, dist, rank, world, dev, steps, warmup, peaks, peaks_s
     prof = aggregate_profile(mg.maglev_profile_report())
     clocks = sampler.stop()
     ms = e0.elapsed_time(e1) / steps
-    ms_max = ms
+    ms_max = max_over_ranks(dist, ms, dev)
     if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
         dist.barrier()
     # dominant kernel and its roofline
     dom = max(prof.items(), key=lambda kv: kv[1][1]) if prof else None
@@ -495,26 +514,19 @@ def main():
         gpu_uuid = None
 
     r = run_layer_bench(torch, dist, rank, world, dev, args.steps, args.warmup, peaks, peaks_src, gpu_uuid)
-    total_flops = r["flops"]["total"] * world
-    value = total_flops / (r["ms"] * 1e-3) / 1e12
+    value = job_rate(r["flops"]["total"], world, r["ms"]) / 1e12
 
     e2e = None
     if not args.no_e2e:
         ms_e2e, h2d, d2h = run_layer_e2e(torch, dev, args.steps, args.warmup, r["step"])
-        if dist is not None:
-            t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        e2e = {"value": round(total_flops / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+        ms_e2e = max_over_ranks(dist, ms_e2e, dev)
+        e2e = {"value": round(job_rate(r["flops"]["total"], world, ms_e2e) / 1e12, 3), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 4)}
 
     dec = None
     if not args.no_decode:
         dec = run_decode_bench(torch, dev, args.decode_steps, args.warmup, peaks)
-        if dist is not None:
-            t = torch.tensor([dec["ms_per_step"]], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            dec["tokens_per_s"] = DECODE["B"] * world * 1000.0 / float(t.item())
+        dec["tokens_per_s"] = job_rate(DECODE["B"], world, max_over_ranks(dist, dec["ms_per_step"], dev))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

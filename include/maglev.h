@@ -165,6 +165,29 @@ maglev_status maglev_mem_project_bwd(const maglev_swa_desc* desc, const void* m_
                                      const void* dR_v, void* dm_shift, void* dw_mk, void* dw_mv,
                                      void* stream);
 
+/* Memory state of a decoder stack ([rainbus] 方法步骤详情: m_t is the stack's
+ * final state after RMSNorm; the injection reads the shifted memory m_{t-1},
+ * with m_0 = 0). Reading: RMSNorm over the d channels of each row, no weight.
+ *   o [B,T,d]: the last layer's output (dtype).
+ *   m [B,T,d] (out): m[b,t] = o[b,t] / sqrt(mean_c o[b,t,c]^2 + eps).
+ *   m_shift [B,T,d] (out, nullable): m_shift[b,0] = 0, m_shift[b,t] = m[b,t-1],
+ *     the layout maglev_inject_swa_fwd reads.
+ *   rstd [B*T] fp32 (out): 1/sqrt(mean(o^2) + eps), read by the backward.
+ * Errors: MAGLEV_ERR_INVALID_ARG for negative sizes, d < 1, eps < 0, bad dtype or
+ * a NULL pointer that is not marked nullable. */
+maglev_status maglev_memory_state(int B, int T, int d, float eps, int dtype, const void* o,
+                                  void* m, void* m_shift, float* rstd, void* stream);
+
+/* Backward of maglev_memory_state. The incoming gradient of row (b,t) is
+ * g = dm[b,t] + dm_shift[b,t+1] (a term is absent when its pointer is NULL or
+ * t+1 = T); its image through RMSNorm is rstd * (g - m * mean_c(m * g)), with m
+ * recomputed from o in fp32.
+ *   d_o [B,T,d] (out) = dout_in + that image; dout_in (nullable) is the
+ *   gradient o already receives from elsewhere and may alias d_o. */
+maglev_status maglev_memory_state_bwd(int B, int T, int d, int dtype, const void* o,
+                                      const float* rstd, const void* dm, const void* dm_shift,
+                                      const void* dout_in, void* d_o, void* stream);
+
 /* Bytes of scratch memory maglev_consistency_loss needs for `rows` x `d`. */
 size_t maglev_consistency_workspace_bytes(int64_t rows, int d);
 

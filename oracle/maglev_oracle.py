@@ -246,6 +246,88 @@ def consistency_loss(m, m_target, lam: float, inv_count: float | None = None):
 
 
 # --------------------------------------------------------------------------
+# stack: prefiller Q and decoder P around one shared memory
+# --------------------------------------------------------------------------
+def memory_state(o, eps: float = 1e-6):
+    """m_t = RMSNorm(o_t) over the d channels of each row (rainbus, 方法步骤详情:
+    the memory is the stack's final state after RMSNorm; no weight). o [B,T,d]."""
+    return rmsnorm(o, eps)
+
+
+def shift_memory(m):
+    """The memory read at position t is m_{t-1}; row 0 reads m_0 = 0
+    (rainbus, 方法步骤详情). m [B,T,d] -> [B,T,d]."""
+    out = np.zeros_like(m)
+    out[:, 1:] = m[:, :-1]
+    return out
+
+
+def stack_forward_backward(q_layers, p_layers, w_mk, w_mv, lam: float, rope_base: float = 10000.0,
+                           eps: float = 1e-6, store=None):
+    """One training step of a prefiller Q and a decoder P that share a memory.
+
+    Q's layers (no injection; dicts with q, k, v, dout, window) run first;
+    m' = RMSNorm(O of Q's last layer) is its memory, and P reads the shifted
+    memory m_shift = shift(m') through one projection shared by every layer
+    (rainbus, 方法步骤详情: 共享投影, rows t read m'_{t-1}). P's layers (dicts with
+    q, k, v, gates, dout, window) run injected; m = RMSNorm(O of P's last
+    layer) meets m' in the consistency loss. The objective is
+        J = sum over all layers <O_l, dout_l> + L_cons(m, m').
+    Every layer has d = H * hd channels. Returns the forward values and the
+    gradients of J (chain rule through the functions above).
+    `store` (optional) maps the combined upstream gradient of each last layer
+    (its dout plus the memory's gradient) to the values kept in storage, for
+    comparison with an implementation that keeps it in a narrower type.
+    """
+    store = store if store is not None else (lambda x: x)
+    B, T, H, hd = q_layers[-1]["q"].shape
+    D = H * hd
+    qf = [inject_swa_forward(L["q"], L["k"], L["v"], None, None, None, L["window"], 0, rope_base, eps,
+                             inject=False) for L in q_layers]
+    oq = qf[-1]["out"].reshape(B, T, D)
+    m_prime = memory_state(oq, eps)
+    m_shift = shift_memory(m_prime)
+    R_k, R_v = mem_project(m_shift, w_mk, w_mv)
+    pf = [inject_swa_forward(L["q"], L["k"], L["v"], R_k, R_v, L["gates"], L["window"], 0, rope_base, eps)
+          for L in p_layers]
+    op = pf[-1]["out"].reshape(B, T, D)
+    m = memory_state(op, eps)
+    loss, dm, dm_prime = consistency_loss(m.reshape(B * T, D), m_prime.reshape(B * T, D), lam)
+    dm = dm.reshape(B, T, D)
+    dm_prime = dm_prime.reshape(B, T, D)
+
+    # P: the last layer also receives the loss through RMSNorm
+    p_grads = []
+    dR_k = np.zeros_like(R_k)
+    dR_v = np.zeros_like(R_v)
+    for i, L in enumerate(p_layers):
+        dout = L["dout"]
+        if i == len(p_layers) - 1:
+            dout = store(dout + rmsnorm_backward(op, dm, eps).reshape(B, T, H, hd))
+        g = inject_swa_backward(L["q"], L["k"], L["v"], R_k, R_v, L["gates"], dout, L["window"], 0,
+                                rope_base, eps)
+        dR_k += g["dR_k"]
+        dR_v += g["dR_v"]
+        p_grads.append({"dq": g["dq"], "dk": g["dk"], "dv": g["dv"], "dgate": g["dgate"], "dout": dout})
+    dm_shift, dw_mk, dw_mv = mem_project_backward(m_shift, w_mk, w_mv, dR_k, dR_v)
+    # m_shift[t] = m'[t-1]: its gradient lands one row earlier
+    dm_prime = dm_prime.copy()
+    dm_prime[:, :-1] += dm_shift[:, 1:]
+    q_grads = []
+    for i, L in enumerate(q_layers):
+        dout = L["dout"]
+        if i == len(q_layers) - 1:
+            dout = store(dout + rmsnorm_backward(oq, dm_prime, eps).reshape(B, T, H, hd))
+        g = inject_swa_backward(L["q"], L["k"], L["v"], None, None, None, dout, L["window"], 0, rope_base, eps,
+                                inject=False)
+        q_grads.append({"dq": g["dq"], "dk": g["dk"], "dv": g["dv"], "dout": dout})
+    return {"loss": loss, "q_out": [f["out"] for f in qf], "p_out": [f["out"] for f in pf],
+            "m": m, "m_prime": m_prime, "m_shift": m_shift, "R_k": R_k, "R_v": R_v,
+            "q_grads": q_grads, "p_grads": p_grads, "dR_k": dR_k, "dR_v": dR_v,
+            "dm_shift": dm_shift, "dw_mk": dw_mk, "dw_mv": dw_mv}
+
+
+# --------------------------------------------------------------------------
 # a8: recurrent decode step over a rolling W-entry ring
 # --------------------------------------------------------------------------
 def decode_mem_project(pos, m_prev, w_mk, w_mv, H: int, rope_base: float = 10000.0, eps: float = 1e-6):

@@ -68,6 +68,8 @@ _SIGS = {
     "maglev_mem_project_bwd": ([ctypes.POINTER(SwaDesc)] + [_P] * 9, _I),
     "maglev_consistency_loss": ([_P, _P, _I64, _I, _I, _F, _F, _P, _P, _P, _I, _P, _P], _I),
     "maglev_consistency_loss_noalloc": ([_P, _P, _I64, _I, _I, _F, _F, _P, _P, _P, _I, _P], _I),
+    "maglev_memory_state": ([_I, _I, _I, _F, _I] + [_P] * 5, _I),
+    "maglev_memory_state_bwd": ([_I, _I, _I, _I] + [_P] * 7, _I),
     "maglev_decode_mem_project": ([ctypes.POINTER(DecodeDesc)] + [_P] * 7, _I),
     "maglev_decode_step": ([ctypes.POINTER(DecodeDesc)] + [_P] * 11, _I),
 }
@@ -212,6 +214,16 @@ def maglev_consistency_loss_noalloc(m, m_target, rows, d, dtype, lam, inv_count,
     _check(_lib.maglev_consistency_loss_noalloc(_ptr(m), _ptr(m_target), int(rows), int(d), int(dtype),
                                                 float(lam), float(inv_count), _ptr(loss), _ptr(dm),
                                                 _ptr(dm_target), int(accumulate_dm), _stream(stream)))
+
+
+def maglev_memory_state(B, T, d, eps, dtype, o, m, m_shift, rstd, stream=None):
+    _check(_lib.maglev_memory_state(int(B), int(T), int(d), float(eps), int(dtype), _ptr(o), _ptr(m),
+                                    _ptr(m_shift), _ptr(rstd), _stream(stream)))
+
+
+def maglev_memory_state_bwd(B, T, d, dtype, o, rstd, dm, dm_shift, dout_in, d_o, stream=None):
+    _check(_lib.maglev_memory_state_bwd(int(B), int(T), int(d), int(dtype), _ptr(o), _ptr(rstd), _ptr(dm),
+                                        _ptr(dm_shift), _ptr(dout_in), _ptr(d_o), _stream(stream)))
 
 
 def maglev_decode_mem_project(desc, pos, m_prev, w_mk, w_mv, krec_rot, vrec, stream=None):

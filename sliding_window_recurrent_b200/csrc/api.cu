@@ -556,6 +556,43 @@ maglev_status maglev_consistency_loss(const void* m, const void* m_target, int64
   return MAGLEV_OK;
 }
 
+maglev_status maglev_memory_state(int B, int T, int d, float eps, int dtype, const void* o, void* m,
+                                  void* m_shift, float* rstd, void* stream) {
+  if (B < 0 || T < 0) return fail(MAGLEV_ERR_INVALID_ARG, "B and T must be >= 0");
+  if (d < 1) return fail(MAGLEV_ERR_INVALID_ARG, "d must be >= 1");
+  if (!(eps >= 0.0f) || !std::isfinite(eps)) return fail(MAGLEV_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  if (dtype != MAGLEV_F32 && dtype != MAGLEV_BF16)
+    return fail(MAGLEV_ERR_INVALID_ARG, "dtype must be MAGLEV_F32 or MAGLEV_BF16");
+  OPT_PTR(m_shift);
+  if ((int64_t)B * T == 0) return MAGLEV_OK;
+  NEED_PTR(o);
+  NEED_PTR(m);
+  NEED_PTR(rstd);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MAGLEV_LAUNCH(1, s, launch_memstate_fwd(o, m, m_shift, rstd, B, T, d, eps, dtype, s), "memory_state");
+  return MAGLEV_OK;
+}
+
+maglev_status maglev_memory_state_bwd(int B, int T, int d, int dtype, const void* o, const float* rstd,
+                                      const void* dm, const void* dm_shift, const void* dout_in, void* d_o,
+                                      void* stream) {
+  if (B < 0 || T < 0) return fail(MAGLEV_ERR_INVALID_ARG, "B and T must be >= 0");
+  if (d < 1) return fail(MAGLEV_ERR_INVALID_ARG, "d must be >= 1");
+  if (dtype != MAGLEV_F32 && dtype != MAGLEV_BF16)
+    return fail(MAGLEV_ERR_INVALID_ARG, "dtype must be MAGLEV_F32 or MAGLEV_BF16");
+  OPT_PTR(dm);
+  OPT_PTR(dm_shift);
+  OPT_PTR(dout_in);
+  if ((int64_t)B * T == 0) return MAGLEV_OK;
+  NEED_PTR(o);
+  NEED_PTR(rstd);
+  NEED_PTR(d_o);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MAGLEV_LAUNCH(1, s, launch_memstate_bwd(o, rstd, dm, dm_shift, dout_in, d_o, B, T, d, dtype, s),
+                "memory_state_bwd");
+  return MAGLEV_OK;
+}
+
 static maglev_status check_dec(const maglev_decode_desc* d) {
   if (!d) return fail(MAGLEV_ERR_INVALID_ARG, "desc must not be NULL");
   if (d->B < 0) return fail(MAGLEV_ERR_INVALID_ARG, "B must be >= 0");

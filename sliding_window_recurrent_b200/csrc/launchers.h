@@ -56,6 +56,15 @@ cudaError_t launch_gate_reduce(int64_t rows, int H, const float* gpart, const fl
                                float* dgate, cudaStream_t st);
 
 int loss_partial_blocks(int64_t n);
+// dtype codes as in maglev_dtype
+constexpr int DT_F32 = 0, DT_BF16 = 1;
+
+// memory state m = RMSNorm(o) per row of d, with the shifted copy, and its backward
+cudaError_t launch_memstate_fwd(const void* o, void* m, void* m_shift, float* rstd, int B, int T, int d,
+                                float eps, int dtype, cudaStream_t st);
+cudaError_t launch_memstate_bwd(const void* o, const float* rstd, const void* dm, const void* dm_shift,
+                                const void* dout_in, void* dout, int B, int T, int d, int dtype, cudaStream_t st);
+
 cudaError_t launch_consistency_loss(const void* m, const void* mt, int64_t rows, int d, int dtype,
                                     float scale_loss, float scale_grad, float* loss, void* dm,
                                     void* dmt, int accumulate, float* partials, cudaStream_t st);

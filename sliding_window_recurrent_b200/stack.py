@@ -1,0 +1,125 @@
+"""A prefiller Q and a decoder P that share one memory, as C-ABI calls.
+
+"Maglev: Sliding Recurrent Memory", paper.rainbus.top, 方法步骤详情: the
+prefiller reads the segment without memory and produces m' (its final state
+after RMSNorm); the decoder reads the shifted memory m'_{t-1} through one
+projection shared by all its layers, and the consistency loss ties its own
+final state m to m'. gptget.net, Abstract: Q interleaves full and
+sliding-window layers (SLSL), P uses sliding-window layers throughout.
+
+One training step:
+  forward   Q layers (no injection) -> memory_state(O_Q last) = m', m_shift
+            mem_project(m_shift) = R_k, R_v (once, shared)
+            P layers (injected, reading R_k, R_v) -> memory_state(O_P last) = m
+            consistency_loss(m, m') -> loss, dm, dm'
+  backward  memory_state_bwd(dm) + dout -> P's last layer; P layers in reverse,
+            summing dR_k, dR_v; mem_project_bwd -> dm_shift, dW_mk, dW_mv;
+            memory_state_bwd(dm' + shifted dm_shift) + dout -> Q's last layer;
+            Q layers in reverse.
+Every layer's own upstream gradient `dout` comes from the caller. This module
+owns buffers and issues library calls only; all arithmetic runs in libmaglev.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (SwaDesc, maglev_consistency_loss, maglev_consistency_workspace_bytes, maglev_inject_swa_bwd,
+               maglev_inject_swa_fwd, maglev_mem_project, maglev_mem_project_bwd, maglev_memory_state,
+               maglev_memory_state_bwd, maglev_swa_bwd_workspace_bytes, maglev_swa_saved_bytes)
+from .layer import CODE, TORCH_DTYPE, _bytes
+
+
+class _LayerBufs:
+    def __init__(self, desc, B, T, H, hd, td, device, inject):
+        self.desc = desc
+        self.out = torch.empty(B, T, H, hd, dtype=td, device=device)
+        self.lse = torch.empty(B, H, T, dtype=torch.float32, device=device)
+        self.saved = _bytes(maglev_swa_saved_bytes(desc), device)
+        self.dq = torch.empty(B, T, H, hd, dtype=td, device=device)
+        self.dk = torch.empty_like(self.dq)
+        self.dv = torch.empty_like(self.dq)
+        self.dgate = torch.empty(4, H, dtype=torch.float32, device=device) if inject else None
+
+
+class PrefillerDecoderStack:
+    """Buffers and call sequence of one Q + P training step.
+
+    q_windows / p_windows: the window of each layer (W >= T is full causal).
+    All layers have H heads of hd channels and d = H * hd memory channels.
+    """
+
+    def __init__(self, B, T, H, hd, q_windows, p_windows, lam=0.1, dtype="bf16", device="cuda",
+                 rope_base=10000.0, eps=1e-6, spin_limit=0):
+        self.B, self.T, self.H, self.hd = B, T, H, hd
+        self.d = H * hd
+        self.lam, self.eps, self.dtype, self.device = lam, eps, dtype, device
+        td = TORCH_DTYPE[dtype]
+        code = CODE[dtype]
+
+        def desc(w, inject):
+            return SwaDesc(B=B, T=T, H=H, hd=hd, d_mem=self.d, window=w, rope_base=rope_base, rms_eps=eps,
+                           inject=int(inject), pos0=0, dtype=code, spin_limit=spin_limit)
+
+        self.q = [_LayerBufs(desc(w, False), B, T, H, hd, td, device, False) for w in q_windows]
+        self.p = [_LayerBufs(desc(w, True), B, T, H, hd, td, device, True) for w in p_windows]
+        ws = max(maglev_swa_bwd_workspace_bytes(L.desc) for L in self.q + self.p)
+        self.workspace = _bytes(ws, device)  # layers run one after another on one stream
+        d = self.d
+        e = lambda *s, t=td: torch.empty(*s, dtype=t, device=device)
+        self.m_prime, self.m_shift, self.m = e(B, T, d), e(B, T, d), e(B, T, d)
+        self.rstd_q, self.rstd_p = e(B * T, t=torch.float32), e(B * T, t=torch.float32)
+        self.R_k, self.R_v = e(B, T, d), e(B, T, d)
+        self.dR_k, self.dR_v = e(B, T, d), e(B, T, d)
+        self.dm, self.dm_prime, self.dm_shift = e(B, T, d), e(B, T, d), e(B, T, d)
+        self.dw_mk, self.dw_mv = e(d, d), e(d, d)
+        self.dout_p_last, self.dout_q_last = e(B, T, H, hd), e(B, T, H, hd)
+        self.loss = torch.zeros((), dtype=torch.float32, device=device)
+        self.loss_ws = _bytes(maglev_consistency_workspace_bytes(B * T, d), device)
+
+    def forward(self, q_inputs, p_inputs, w_mk, w_mv, stream=None):
+        """q_inputs: per Q layer (q, k, v); p_inputs: per P layer (q, k, v, gate_logits)."""
+        B, T, d, code = self.B, self.T, self.d, CODE[self.dtype]
+        for L, (q, k, v) in zip(self.q, q_inputs):
+            maglev_inject_swa_fwd(L.desc, q, k, v, None, None, None, None, None, None, L.out, L.lse, L.saved,
+                                  stream)
+        maglev_memory_state(B, T, d, self.eps, code, self.q[-1].out, self.m_prime, self.m_shift, self.rstd_q,
+                            stream)
+        maglev_mem_project(self.p[0].desc, self.m_shift, w_mk, w_mv, self.R_k, self.R_v, stream)
+        for L, (q, k, v, g) in zip(self.p, p_inputs):
+            maglev_inject_swa_fwd(L.desc, q, k, v, None, w_mk, w_mv, self.R_k, self.R_v, g, L.out, L.lse,
+                                  L.saved, stream)
+        maglev_memory_state(B, T, d, self.eps, code, self.p[-1].out, self.m, None, self.rstd_p, stream)
+        maglev_consistency_loss(self.m, self.m_prime, B * T, d, code, self.lam, 0.0, self.loss, self.dm,
+                                self.dm_prime, False, self.loss_ws, stream)
+        return self.loss
+
+    def backward(self, q_inputs, p_inputs, q_douts, p_douts, w_mk, w_mv, stream=None):
+        """q_douts / p_douts: each layer's upstream gradient of its output."""
+        B, T, d, code = self.B, self.T, self.d, CODE[self.dtype]
+        maglev_memory_state_bwd(B, T, d, code, self.p[-1].out, self.rstd_p, self.dm, None, p_douts[-1],
+                                self.dout_p_last, stream)
+        n = len(self.p)
+        for i in reversed(range(n)):
+            L = self.p[i]
+            _, k, v, g = p_inputs[i]
+            dout = self.dout_p_last if i == n - 1 else p_douts[i]
+            maglev_inject_swa_bwd(L.desc, k, v, self.R_k, self.R_v, g, L.out, L.lse, L.saved, dout, L.dq, L.dk,
+                                  L.dv, self.dR_k, self.dR_v, i != n - 1, L.dgate, None, None, None, None, None,
+                                  None, self.workspace, stream)
+        maglev_mem_project_bwd(self.p[0].desc, self.m_shift, w_mk, w_mv, self.dR_k, self.dR_v, self.dm_shift,
+                               self.dw_mk, self.dw_mv, stream)
+        maglev_memory_state_bwd(B, T, d, code, self.q[-1].out, self.rstd_q, self.dm_prime, self.dm_shift,
+                                q_douts[-1], self.dout_q_last, stream)
+        n = len(self.q)
+        for i in reversed(range(n)):
+            L = self.q[i]
+            _, k, v = q_inputs[i]
+            dout = self.dout_q_last if i == n - 1 else q_douts[i]
+            maglev_inject_swa_bwd(L.desc, k, v, None, None, None, L.out, L.lse, L.saved, dout, L.dq, L.dk, L.dv,
+                                  None, None, False, None, None, None, None, None, None, None, self.workspace,
+                                  stream)
+
+    def step(self, q_inputs, p_inputs, q_douts, p_douts, w_mk, w_mv, stream=None):
+        self.forward(q_inputs, p_inputs, w_mk, w_mv, stream)
+        self.backward(q_inputs, p_inputs, q_douts, p_douts, w_mk, w_mv, stream)
+        return self.loss

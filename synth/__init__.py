@@ -138,6 +138,28 @@ def layer_inputs(wl: dict, seed: int, layer: int = 0, inject: bool = True) -> di
     return out
 
 
+def stack_inputs(wl: dict, seed: int, q_windows, p_windows) -> dict:
+    """Seeded inputs of a prefiller Q (no injection) and a decoder P sharing a
+    memory: per layer q, k, v, dout ~ N(0,1) [B,T,H,hd]; P's gate logits
+    ~ U[-2,2]; W_mk, W_mv [D,D] ~ N(0,1/D). P's layer l draws with layer index
+    l, Q's layer l with index 32 + l."""
+    B, T, H, hd, dt = wl["B"], wl["T"], wl["H"], wl["hd"], wl["dtype"]
+    D = H * hd
+
+    def one(layer, gates):
+        off = 64 * layer
+        x = {k: normal(seed, TID[k] + off, (B, T, H, hd), dtype=dt) for k in ("q", "k", "v", "dout")}
+        if gates:
+            x["gates"] = uniform(seed, TID["gates"] + off, (4, H), -2.0, 2.0)
+        return x
+
+    q_layers = [dict(one(32 + l, False), window=w) for l, w in enumerate(q_windows)]
+    p_layers = [dict(one(l, True), window=w) for l, w in enumerate(p_windows)]
+    return {"q_layers": q_layers, "p_layers": p_layers,
+            "w_mk": normal(seed, TID["w_mk"], (D, D), std=1.0 / np.sqrt(D), dtype=dt),
+            "w_mv": normal(seed, TID["w_mv"], (D, D), std=1.0 / np.sqrt(D), dtype=dt)}
+
+
 def ring_slice(seed: int, layer: int, b: int, H: int, W: int, hd: int, which: str, dtype: str = "bf16") -> Tensor:
     """Pre-filled ring entries of one (layer, batch row): [H, W, hd] ~ N(0,1)."""
     return normal(seed, TID[which], (H, W, hd), dtype=dtype, sub=(layer << 16) | b)

@@ -1,0 +1,80 @@
+"""Parity of the prefiller + decoder stack (Q -> memory -> P -> loss) with the oracle.
+
+The stack runs every layer through the C ABI (sliding_window_recurrent_b200.stack)
+and is compared, tensor by tensor, with oracle.stack_forward_backward on the
+same seeded inputs. The combined upstream gradient of each last layer is held
+in the activation type on the GPU; the oracle is told to round it the same way.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests.helpers import TOL, assert_close, dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+def _bf16(x):
+    return synth.bf16_bits_to_f64(synth.round_to_bf16_bits(np.asarray(x, dtype=np.float32)))
+
+
+def _run(wl, seed, q_windows, p_windows):
+    import torch
+    from sliding_window_recurrent_b200.stack import PrefillerDecoderStack
+
+    x = synth.stack_inputs(wl, seed, q_windows, p_windows)
+    B, T, H, hd = wl["B"], wl["T"], wl["H"], wl["hd"]
+    S = PrefillerDecoderStack(B, T, H, hd, q_windows, p_windows, lam=wl["lam"], dtype=wl["dtype"])
+    qi = [(dev(L["q"]), dev(L["k"]), dev(L["v"])) for L in x["q_layers"]]
+    pi = [(dev(L["q"]), dev(L["k"]), dev(L["v"]), dev(L["gates"])) for L in x["p_layers"]]
+    qd = [dev(L["dout"]) for L in x["q_layers"]]
+    pd = [dev(L["dout"]) for L in x["p_layers"]]
+    wk, wv = dev(x["w_mk"]), dev(x["w_mv"])
+    S.step(qi, pi, qd, pd, wk, wv)
+    torch.cuda.synchronize()
+
+    f64 = lambda L, keys: {k: (L[k].f64 if isinstance(L[k], synth.Tensor) else L[k]) for k in keys}
+    ql = [dict(f64(L, ("q", "k", "v", "dout")), window=L["window"]) for L in x["q_layers"]]
+    pl = [dict(f64(L, ("q", "k", "v", "dout")), gates=L["gates"].astype(np.float64), window=L["window"])
+          for L in x["p_layers"]]
+    store = _bf16 if wl["dtype"] == "bf16" else None
+    ref = oracle.stack_forward_backward(ql, pl, x["w_mk"].f64, x["w_mv"].f64, wl["lam"], store=store)
+    return S, ref
+
+
+def _check_all(S, ref, dt):
+    B, T, H, hd = S.B, S.T, S.H, S.hd
+    for i, L in enumerate(S.q):
+        assert_close(host(L.out), ref["q_out"][i], dt, f"Q{i} out")
+        for g in ("dq", "dk", "dv"):
+            assert_close(host(getattr(L, g)), ref["q_grads"][i][g], dt, f"Q{i} {g}")
+    for i, L in enumerate(S.p):
+        assert_close(host(L.out), ref["p_out"][i], dt, f"P{i} out")
+        for g in ("dq", "dk", "dv"):
+            assert_close(host(getattr(L, g)), ref["p_grads"][i][g], dt, f"P{i} {g}")
+        assert_close(host(L.dgate), ref["p_grads"][i]["dgate"], "f32" if dt == "f32" else dt, f"P{i} dgate")
+    assert_close(host(S.m_prime), ref["m_prime"], dt, "m'")
+    assert_close(host(S.m_shift), ref["m_shift"], dt, "m_shift")
+    assert np.all(host(S.m_shift)[:, 0] == 0), "row 0 of the shifted memory is m'_0 = 0"
+    assert_close(host(S.m), ref["m"], dt, "m")
+    assert abs(float(S.loss.item()) - ref["loss"]) <= TOL[dt] * abs(ref["loss"]), (float(S.loss.item()), ref["loss"])
+    assert_close(host(S.dm_shift), ref["dm_shift"], dt, "dm_shift")
+    assert_close(host(S.dw_mk), ref["dw_mk"], dt, "dW_mk")
+    assert_close(host(S.dw_mv), ref["dw_mv"], dt, "dW_mv")
+
+
+@pytest.mark.parametrize("T", [200, 129])
+def test_stack_bf16_small(T):
+    """SLSL prefiller (window 64 and full causal) and a 3-layer injected decoder,
+    ragged T, two heads of 128 (the tensor-core path)."""
+    wl = dict(B=2, T=T, H=2, hd=128, dtype="bf16", lam=0.1)
+    S, ref = _run(wl, 1234, [64, T, 64, T], [64, 64, 64])
+    _check_all(S, ref, "bf16")
+
+
+def test_stack_f32_small():
+    """The same stack on the fp32 path (CUDA cores), head dim 64."""
+    wl = dict(B=1, T=150, H=2, hd=64, dtype="f32", lam=1.0)
+    S, ref = _run(wl, 1235, [32, 150], [32, 32])
+    _check_all(S, ref, "f32")

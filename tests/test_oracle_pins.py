@@ -356,6 +356,90 @@ def test_mem_project_backward_matches_autograd():
     np.testing.assert_allclose(dWv, tv.grad.numpy(), rtol=1e-12)
 
 
+# ---------------------------------------------------------------- stack (Q -> memory -> P -> loss)
+def _stack(B=1, T=7, H=1, hd=4, nq=2, np_=2):
+    D = H * hd
+    ql = [dict(q=rand(B, T, H, hd), k=rand(B, T, H, hd), v=rand(B, T, H, hd), dout=rand(B, T, H, hd),
+               window=3 if i % 2 == 0 else T) for i in range(nq)]
+    pl = [dict(q=rand(B, T, H, hd), k=rand(B, T, H, hd), v=rand(B, T, H, hd), dout=rand(B, T, H, hd),
+               gates=RNG.uniform(-2, 2, (4, H)), window=3) for _ in range(np_)]
+    return ql, pl, rand(D, D) / np.sqrt(D), rand(D, D) / np.sqrt(D)
+
+
+def _stack_objective(ql, pl, wk, wv, lam):
+    r = oracle.stack_forward_backward(ql, pl, wk, wv, lam)
+    j = r["loss"]
+    for L, o in zip(ql, r["q_out"]):
+        j += np.sum(o * L["dout"])
+    for L, o in zip(pl, r["p_out"]):
+        j += np.sum(o * L["dout"])
+    return j
+
+
+def test_shift_memory_and_state():
+    m = rand(2, 5, 3)
+    s = oracle.shift_memory(m)
+    assert np.all(s[:, 0] == 0) and np.array_equal(s[:, 1:], m[:, :-1])
+    o = rand(2, 5, 6)
+    ref = F.rms_norm(torch.from_numpy(o), (6,), eps=1e-6).numpy()
+    np.testing.assert_allclose(oracle.memory_state(o), ref, rtol=1e-13)
+
+
+def test_stack_central_differences():
+    """Every gradient of the stack objective, including the path from P's loss
+    and injection back through the shift into Q's last layer."""
+    ql, pl, wk, wv = _stack()
+    lam = 0.7
+    r = oracle.stack_forward_backward(ql, pl, wk, wv, lam)
+    cases = []
+    for li in range(len(ql)):
+        for key in ("q", "k", "v"):
+            cases.append((("q", li, key), r["q_grads"][li]["d" + key]))
+    for li in range(len(pl)):
+        for key in ("q", "k", "v"):
+            cases.append((("p", li, key), r["p_grads"][li]["d" + key]))
+        cases.append((("p", li, "gates"), r["p_grads"][li]["dgate"]))
+    cases += [(("w", 0, "wk"), r["dw_mk"]), (("w", 0, "wv"), r["dw_mv"])]
+    h = 1e-6
+    for (side, li, key), grad in cases:
+        for idx in [tuple(RNG.integers(0, s) for s in grad.shape) for _ in range(3)]:
+            def j_at(delta):
+                ql2 = [{k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in L.items()} for L in ql]
+                pl2 = [{k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in L.items()} for L in pl]
+                wk2, wv2 = wk.copy(), wv.copy()
+                if side == "q":
+                    ql2[li][key][idx] += delta
+                elif side == "p":
+                    pl2[li][key][idx] += delta
+                else:
+                    (wk2 if key == "wk" else wv2)[idx] += delta
+                return _stack_objective(ql2, pl2, wk2, wv2, lam)
+            fd = (j_at(h) - j_at(-h)) / (2 * h)
+            assert abs(fd - grad[idx]) <= 1e-6 * max(1.0, abs(fd)), (side, li, key, idx, fd, grad[idx])
+
+
+def test_stack_gates_off_decouples_memory():
+    """With both recurrent gates shut (a = -inf) P ignores the memory: P's
+    outputs are plain SWA, the projection gets no gradient, and Q's last layer
+    sees only its own dout plus the loss's target term."""
+    ql, pl, wk, wv = _stack(T=9)
+    for L in pl:
+        L["gates"][1] = -np.inf
+        L["gates"][3] = -np.inf
+        L["gates"][0] = 0.0
+        L["gates"][2] = 0.0
+    r = oracle.stack_forward_backward(ql, pl, wk, wv, 0.5)
+    for L, o in zip(pl, r["p_out"]):
+        plain = oracle.inject_swa_forward(L["q"], L["k"], L["v"], None, None, None, L["window"], inject=False)
+        assert np.array_equal(o, plain["out"])
+    assert np.all(r["dw_mk"] == 0) and np.all(r["dw_mv"] == 0) and np.all(r["dm_shift"] == 0)
+    B, T, H, hd = ql[-1]["q"].shape
+    oq = r["q_out"][-1].reshape(B, T, H * hd)
+    _, _, dmp = oracle.consistency_loss(r["m"].reshape(B * T, -1), r["m_prime"].reshape(B * T, -1), 0.5)
+    want = ql[-1]["dout"] + oracle.rmsnorm_backward(oq, dmp.reshape(B, T, -1), 1e-6).reshape(B, T, H, hd)
+    np.testing.assert_allclose(r["q_grads"][-1]["dout"], want, rtol=1e-13, atol=1e-13)
+
+
 # ---------------------------------------------------------------- consistency loss
 def test_consistency_loss_closed_forms():
     rows, d = 7, 64
