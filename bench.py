@@ -35,6 +35,7 @@ import numpy as np  # noqa: E402
 METRIC = "Injected-SWA attn fwd+bwd TFLOP/s & % bf16 peak; decode tokens/s"
 LAYER = dict(B=4, T=2048, H=10, hd=128, d=1280, W=512, lam=0.1)
 DECODE = dict(B=64, L=20, H=10, hd=128, d=1280, W=512, first_pos=512)
+STACK = dict(B=8, T=2048, H=10, hd=128, L=20, W=512, lam=0.1)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per launch from ncu captures, keyed by trace name;
@@ -61,6 +62,25 @@ def layer_flops(B, T, H, hd, d, W):
             "proj_bwd": proj_bwd, "total": attn_fwd + attn_bwd + proj_fwd + proj_bwd}
 
 
+def stack_windows(c: dict):
+    """Prefiller Q alternates sliding (W) and full (T) layers; decoder P is all W."""
+    q = [c["W"] if l % 2 == 0 else c["T"] for l in range(c["L"])]
+    return q, [c["W"]] * c["L"]
+
+
+def stack_flops(c: dict) -> float:
+    """Attention fwd+bwd of every Q and P layer plus one shared projection fwd+bwd."""
+    B, T, H, hd = c["B"], c["T"], c["H"], c["hd"]
+    d = H * hd
+    q_w, p_w = stack_windows(c)
+    tot = 0.0
+    for w in q_w + p_w:
+        f = layer_flops(B, T, H, hd, d, w)
+        tot += f["attn_fwd"] + f["attn_bwd"]
+    f = layer_flops(B, T, H, hd, d, c["W"])
+    return tot + f["proj_fwd"] + f["proj_bwd"]
+
+
 def kernel_work(name: str, cfg: dict) -> tuple[float, str]:
     """Algorithmic work of one launch of a traced kernel: (amount, unit)."""
     B, T, H, hd, d, W = (cfg[k] for k in ("B", "T", "H", "hd", "d", "W"))
@@ -79,10 +99,14 @@ def kernel_work(name: str, cfg: dict) -> tuple[float, str]:
         "mem_project_tc": (f["proj_fwd"], "flop"),
         "mem_project_bwd_dm_tc": (f["proj_fwd"], "flop"),
         "mem_project_bwd_dw_tc": (f["proj_fwd"], "flop"),
+        # reads q, k, v, R_k, R_v; writes q_rot, k_bar, v_bar (bf16)
         "inject_prep": (B * T * D * 2.0 * (5 + 3), "byte"),
-        "unmix": (B * T * D * (4 * 2 + 2 * 4 + 4 * 2.0), "byte"),
-        "consistency_loss": (B * T * D * 2.0 * 3, "byte"),
-        "attn_delta": (B * T * D * 2.0 * 2, "byte"),
+        # reads dq_rot, dk_bar, dv_bar (fp32) and k, v, R_k, R_v; writes dq, dk, dv, dR_k, dR_v
+        "unmix": (B * T * D * (3 * 4 + 4 * 2 + 5 * 2.0), "byte"),
+        # reads m, m', dm; writes dm (the layer step accumulates into dO)
+        "consistency_loss": (B * T * D * 2.0 * 4, "byte"),
+        # reads O, dO (bf16); zeroes the fp32 dQ accumulator
+        "attn_delta": (B * T * D * (2.0 * 2 + 4), "byte"),
     }
     return table.get(name, (0.0, "flop"))
 
@@ -195,7 +219,12 @@ def make_layer_inputs(torch, dev, seed):
 
 
 class LayerStep:
-    """One fwd + loss + bwd step of the d20 layer through the C ABI."""
+    """One fwd + loss + bwd step of the d20 layer through the C ABI.
+
+    The loss gradient is added in place to the upstream-gradient buffer, as a
+    training step adds it to the dO it receives; the buffer is filled from the
+    seeded dO once, outside the timed region (the added ~1e-6 per element is
+    below half a bf16 ulp of the N(0,1) values, so steps do not drift)."""
 
     def __init__(self, torch, dev, inputs):
         from sliding_window_recurrent_b200.layer import InjectedSWALayer
@@ -204,11 +233,10 @@ class LayerStep:
         self.x = inputs
         self.L = InjectedSWALayer(c["B"], c["T"], c["H"], c["hd"], c["d"], c["W"], dtype="bf16", device=dev)
         self.D = c["H"] * c["hd"]
-        self.dout_total = torch.empty_like(inputs["dout"])
+        self.dout_total = inputs["dout"].clone()
 
     def __call__(self):
         x, L, D = self.x, self.L, self.D
-        self.dout_total.copy_(x["dout"])
         L.forward(x["q"], x["k"], x["v"], x["gates"], x["m_shift"], x["w_mk"], x["w_mv"])
         L.consistency(L.out.view(-1, D), x["target"].view(-1, D), LAYER["lam"],
                       dm=self.dout_total.view(-1, D), accumulate_dm=True)
@@ -299,8 +327,8 @@ def run_layer_e2e(torch, dev, steps, warmup, step):
     stream = torch.cuda.current_stream()
 
     def e2e_step():
-        for n in names:
-            x[n].copy_(host[n], non_blocking=True)
+        for n in names:  # this step's dO lands in the buffer the step accumulates into
+            (step.dout_total if n == "dout" else x[n]).copy_(host[n], non_blocking=True)
         step()
         for o, h in zip(outs, host_out):
             h.copy_(o, non_blocking=True)
@@ -315,6 +343,82 @@ def run_layer_e2e(torch, dev, steps, warmup, step):
     e1.record(stream)
     torch.cuda.synchronize()
     return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
+def run_layer_fwd_bench(torch, dev, steps, warmup, step):
+    """Forward only (projection, injection, attention) of the same layer."""
+    x, L = step.x, step.L
+
+    def fwd():
+        L.forward(x["q"], x["k"], x["v"], x["gates"], x["m_shift"], x["w_mk"], x["w_mv"])
+
+    for _ in range(warmup):
+        fwd()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fwd()
+    e1.record()
+    torch.cuda.synchronize()
+    c = LAYER
+    f = layer_flops(c["B"], c["T"], c["H"], c["hd"], c["d"], c["W"])
+    ms = e0.elapsed_time(e1) / steps
+    return {"value": round((f["attn_fwd"] + f["proj_fwd"]) / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 4), "gflop_per_step": round((f["attn_fwd"] + f["proj_fwd"]) / 1e9, 3),
+            "workload": "d20 injected-SWA layer forward: B=4 T=2048 d=1280 H=10x128 W=512, bf16"}
+
+
+def run_stack_bench(torch, dev, steps, warmup):
+    """Prefiller Q (20 SLSL layers, no injection) + decoder P (20 injected
+    layers) + shared projection + memory state + loss, fwd+bwd, B=8."""
+    import sliding_window_recurrent_b200 as mg
+    from sliding_window_recurrent_b200.stack import PrefillerDecoderStack
+    c = STACK
+    B, T, H, hd = c["B"], c["T"], c["H"], c["hd"]
+    D = H * hd
+    q_w, p_w = stack_windows(c)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(2468)
+    bf = torch.bfloat16
+    rn = lambda *s, std=1.0: (torch.randn(*s, generator=gen, device=dev) * std).to(bf)
+    qi = [(rn(B, T, H, hd), rn(B, T, H, hd), rn(B, T, H, hd)) for _ in q_w]
+    pi = [(rn(B, T, H, hd), rn(B, T, H, hd), rn(B, T, H, hd),
+           torch.rand(4, H, generator=gen, device=dev) * 4 - 2) for _ in p_w]
+    qd = [rn(B, T, H, hd) for _ in q_w]
+    pd = [rn(B, T, H, hd) for _ in p_w]
+    wk, wv = rn(D, D, std=D ** -0.5), rn(D, D, std=D ** -0.5)
+    S = PrefillerDecoderStack(B, T, H, hd, q_w, p_w, lam=c["lam"], device=dev)
+    step = lambda: S.step(qi, pi, qd, pd, wk, wv)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    n0 = mg.maglev_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    launches = mg.maglev_launch_count() - n0
+    ms = e0.elapsed_time(e1) / steps
+    mg.maglev_profile_enable(True)
+    step()
+    torch.cuda.synchronize()
+    mg.maglev_profile_enable(False)
+    prof = aggregate_profile(mg.maglev_profile_report())
+    tot = sum(v[1] for v in prof.values())
+    fl = stack_flops(c)
+    out = {"value": round(fl / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s", "ms_per_step": round(ms, 3),
+           "gflop_per_step": round(fl / 1e9, 1), "gpu_launches": launches,
+           "workload": f"prefiller Q 20 layers SLSL (W={c['W']}/{T}, no injection) + decoder P 20 injected "
+                       f"layers (W={c['W']}) + shared projection + memory state + consistency loss, fwd+bwd, "
+                       f"B={B} T={T} H={H}x{hd}, bf16",
+           "kernels": {n: {"calls": v[0], "ms_total": round(v[1], 3), "share": round(v[1] / tot, 4)}
+                       for n, v in sorted(prof.items(), key=lambda kv: -kv[1][1])}}
+    del S, qi, pi, qd, pd
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_decode_bench(torch, dev, steps, warmup, peaks):
@@ -429,6 +533,18 @@ def sample_flops(c):
     return f["total"]
 
 
+def oracle_threads() -> int:
+    """Threads the oracle's numpy BLAS runs with (its only parallel part)."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads", 1) for p in threadpool_info() if p.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return 1
+
+
 def cpu_baseline(budget_s=12.0):
     c = LAYER
     x = oracle_sample_inputs()
@@ -440,7 +556,7 @@ def cpu_baseline(budget_s=12.0):
         el = time.perf_counter() - t0
         if el >= budget_s or n >= 50:
             break
-    return {"value": round(fl * n / el / 1e12, 6), "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+    return {"value": round(fl * n / el / 1e12, 6), "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
             "sample": f"oracle fwd+loss+bwd of batch row 0, head 0 (T=2048, W=512, d=1280): {fl/1e9:.3f} GFLOP x {n} runs in {el:.1f} s"}
 
 
@@ -463,7 +579,7 @@ def reference_arm(args, rank):
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": "d20 injected-SWA layer fwd+loss+bwd, bounded sample: batch row 0, head 0, "
                                    "T=2048, W=512, d=1280 (the CPU fp64 oracle)", "seq_len": c["T"]},
-            "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+            "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
                              "sample": f"{fl/1e9:.3f} GFLOP per step (one batch row, one head)"},
             "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -478,6 +594,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--decode-steps", type=int, default=64)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--stack-steps", type=int, default=5)
+    ap.add_argument("--no-stack", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
@@ -523,6 +641,13 @@ def main():
         e2e = {"value": round(job_rate(r["flops"]["total"], world, ms_e2e) / 1e12, 3), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 4)}
 
+    fwd = run_layer_fwd_bench(torch, dev, args.steps, args.warmup, r["step"])
+    stack = None
+    if not args.no_stack:
+        stack = run_stack_bench(torch, dev, args.stack_steps, args.warmup)
+        ms_stack = max_over_ranks(dist, stack["ms_per_step"], dev)
+        stack["value"] = round(job_rate(stack_flops(STACK), world, ms_stack) / 1e12, 3)
+
     dec = None
     if not args.no_decode:
         dec = run_decode_bench(torch, dev, args.decode_steps, args.warmup, peaks)
@@ -555,6 +680,8 @@ def main():
         "e2e": e2e,
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
+        "forward": fwd,
+        "stack": stack,
         "decode": None if dec is None else {
             "value": round(dec["tokens_per_s"], 1), "unit": "tokens/s", "ms_per_step": round(dec["ms_per_step"], 4),
             "workload": dec["workload"], "roofline": dec["roofline"], "kernels": dec["kernels"]},

@@ -7,14 +7,19 @@
 //   S^T  = K Q^T,  dP^T = V dO^T                    (TMEM, fp32)
 //   P^T  = exp(S^T * scale - LSE),  dS^T = P^T (dP^T - Delta) * scale
 //   dV  += P^T dO,  dK += dS^T Q                    (TMEM accumulators)
-//   dQ_i = dS K -> fp32 vector atomics into a zeroed dQ accumulator
+//   dQ_i = dS K -> staged in shared memory, reduce-added (TMA, fp32) into a
+//                  zeroed dQ accumulator
 //   warp 0     TMA: K, V once; Q_i, dO_i per query tile
 //   warp 1     tcgen05.mma issue
 //   warps 2-9  two warps per TMEM lane quarter, each taking half of the 128
 //              query columns of a key row: masked P^T and dS^T in registers,
 //              written bf16 128B-swizzled into shared memory (K-major for the
 //              dV / dK MMAs, read back MN-major as dS for the dQ MMA); then
-//              half of the dQ drain; finally dK, dV rows stored in fp32.
+//              half of the dQ drain: TMEM -> registers (R_S released at
+//              once) -> the warp's own 4 KiB slices of the P^T / dS^T
+//              buffers (free once the dQ MMA completed) -> one TMA
+//              reduce-add per 32x32 fp32 block; finally dK, dV rows in fp32.
+//              Half-tiles inside every row's window skip the band mask.
 //              LSE and Delta of each query tile are staged in shared memory.
 // Delta = rowsum(dO * O) comes from the delta kernel. Every wait is bounded.
 #include <cuda.h>
@@ -25,6 +30,7 @@
 namespace maglev {
 
 cudaError_t make_tmap_tokens(CUtensorMap* m, const void* base, int B, int T, int H, int hd, uint32_t box_rows);
+cudaError_t make_tmap_f32_tokens(CUtensorMap* m, void* base, int B, int T, int H, int hd);
 
 namespace {
 
@@ -61,7 +67,7 @@ struct BwdParams {
   float scale, scale_log2;
   const float* lse;    // [B,H,T] natural log
   const float* delta;  // [B,H,T]
-  float* dq_acc;       // [B,T,H,hd] fp32, zeroed, rotated frame
+  float* dq_acc;       // [B,T,H,hd] fp32, zeroed, rotated frame (written through tmDQ)
   float* dk_bar;       // [B,T,H,hd] fp32
   float* dv_bar;       // [B,T,H,hd] fp32
   int64_t spin_limit;
@@ -88,7 +94,7 @@ template <int HD>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                       BwdParams p) {
+                       const __grid_constant__ CUtensorMap tmDQ, BwdParams p) {
   using C = BwdCfg<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -125,6 +131,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmDO);
+    tma_prefetch_desc(&tmDQ);
   }
   if (warp == 1) tmem_alloc(tmem_slot, 512);
   __syncthreads();
@@ -248,8 +255,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ok = ok && warp_wait(s_full, par, ab);
       if (!ok) continue;
       tc_fence_after();
+      if (i > 0) {  // the previous tile's dQ reduce has read its staging (our P^T / dS^T slices)
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+      }
       const int lo = kj - qt;  // first valid column (query >= key)
       const int hi = min(kj + p.W - 1, p.T - 1) - qt;
+      const int kw = kt + 32 * q4;  // first key row of this warp
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
         const int c = 2 * half + cc;  // 32-column chunk index
@@ -257,6 +269,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_ld32(tmem + lane_off + C::R_S + 32u * (uint32_t)c, sv);
         tmem_ld32(tmem + lane_off + C::R_DP + 32u * (uint32_t)c, dv);
         tmem_wait_ld();
+        // queries qt+32c .. +31 inside the window of each of this warp's keys
+        const int q0 = qt + 32 * c;
+        const bool full = q0 >= kw + 31 && q0 + 31 <= kw + p.W - 1 && q0 + 31 <= p.T - 1 && kw + 31 < p.T;
         float pt[32], ds[32];
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
@@ -268,8 +283,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int u = 0; u < 4; ++u) {
             const int e = 4 * e4 + u;
             const int col = 32 * c + e;
-            const bool valid = col >= lo && col <= hi && kj < p.T;
-            const float pe = valid ? exp2f(__uint_as_float(sv[e]) * p.scale_log2 - Ls[u]) : 0.f;
+            const float y = ex2_fast(fmaf(__uint_as_float(sv[e]), p.scale_log2, -Ls[u]));
+            const float pe = (full || (col >= lo && col <= hi && kj < p.T)) ? y : 0.f;
             pt[e] = pe;
             ds[e] = pe * (__uint_as_float(dv[e]) - Ds[u]) * p.scale;
           }
@@ -284,24 +299,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ok = warp_wait(dq_full, par, ab);
       if (!ok) continue;
       tc_fence_after();
-      const int qi = qt + r;
-      float* dst = p.dq_acc + (((int64_t)b * p.T + qi) * p.H + h) * HD;
-#pragma unroll 1
-      for (int c = half * (HD / 64); c < (half + 1) * (HD / 64); ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_off + C::R_S + 32u * (uint32_t)c, v);
-        tmem_wait_ld();
-        if (qi < p.T) {
+      // this warp's dQ block: query rows qt+32*q4 .. +31, channels [32*c0, 32*c0 + 32*NC)
+      constexpr int NC = HD / 64;
+      const int c0 = half * NC;
+      uint32_t v[NC][32];
 #pragma unroll
-          for (int g = 0; g < 8; ++g)
-            atomicAdd(reinterpret_cast<float4*>(dst + 32 * c + 4 * g),
-                      make_float4(__uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1]),
-                                  __uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3])));
-        }
-      }
+      for (int cc = 0; cc < NC; ++cc) tmem_ld32(tmem + lane_off + C::R_S + 32u * (uint32_t)(c0 + cc), v[cc]);
+      tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(dq_empty);
+      mbar_arrive(dq_empty);  // R_S may take S^T of the next tile
+      // stage each 32x32 fp32 block in this warp's slice of P^T (cc = 0) / dS^T
+      // (cc = 1): rows of 128 B, 16-byte chunks swizzled by row (TMA 128B swizzle)
+#pragma unroll
+      for (int cc = 0; cc < NC; ++cc) {
+        uint8_t* stage = (cc == 0 ? sPT : sDS) + half * 16384 + q4 * 4096;
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+          *reinterpret_cast<uint4*>(stage + lane * 128 + ((g ^ (lane & 7)) << 4)) =
+              make_uint4(v[cc][4 * g], v[cc][4 * g + 1], v[cc][4 * g + 2], v[cc][4 * g + 3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && qt + 32 * q4 < p.T) {
+#pragma unroll
+        for (int cc = 0; cc < NC; ++cc)
+          tma_reduce_add_4d(&tmDQ, (cc == 0 ? sPT : sDS) + half * 16384 + q4 * 4096, 32 * (c0 + cc), h,
+                            qt + 32 * q4, b);
+        bulk_commit();
+      }
     }
+    if (lane == 0) bulk_wait_all();  // dQ reductions complete before the CTA leaves
+    __syncwarp();
     if (__all_sync(0xffffffffu, ok) && n_q > 0) {
       // all MMAs are complete (dq_full of the last tile was waited): dK, dV rows
       tc_fence_after();
@@ -351,6 +379,8 @@ cudaError_t launch_attn_bwd_tc(const SwaShape& s, const void* q_rot, const void*
   if ((e = make_tmap_tokens(&tk, k_bar, s.B, s.T, s.H, s.hd, 128)) != cudaSuccess) return e;
   if ((e = make_tmap_tokens(&tv, v_bar, s.B, s.T, s.H, s.hd, 128)) != cudaSuccess) return e;
   if ((e = make_tmap_tokens(&tdo, dout, s.B, s.T, s.H, s.hd, 128)) != cudaSuccess) return e;
+  CUtensorMap tdq;
+  if ((e = make_tmap_f32_tokens(&tdq, dq_acc, s.B, s.T, s.H, s.hd)) != cudaSuccess) return e;
   BwdParams p;
   p.B = s.B;
   p.T = s.T;
@@ -370,12 +400,12 @@ cudaError_t launch_attn_bwd_tc(const SwaShape& s, const void* q_rot, const void*
     auto k = attn_bwd_tc_kernel<128>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BwdCfg<128>::SMEM);
     if (e != cudaSuccess) return e;
-    k<<<grid, NUM_THREADS, BwdCfg<128>::SMEM, st>>>(tq, tk, tv, tdo, p);
+    k<<<grid, NUM_THREADS, BwdCfg<128>::SMEM, st>>>(tq, tk, tv, tdo, tdq, p);
   } else if (s.hd == 64) {
     auto k = attn_bwd_tc_kernel<64>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BwdCfg<64>::SMEM);
     if (e != cudaSuccess) return e;
-    k<<<grid, NUM_THREADS, BwdCfg<64>::SMEM, st>>>(tq, tk, tv, tdo, p);
+    k<<<grid, NUM_THREADS, BwdCfg<64>::SMEM, st>>>(tq, tk, tv, tdo, tdq, p);
   } else {
     return cudaErrorInvalidValue;
   }
