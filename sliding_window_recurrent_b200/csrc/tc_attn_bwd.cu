@@ -31,6 +31,7 @@ namespace maglev {
 
 cudaError_t make_tmap_tokens(CUtensorMap* m, const void* base, int B, int T, int H, int hd, uint32_t box_rows);
 cudaError_t make_tmap_f32_tokens(CUtensorMap* m, void* base, int B, int T, int H, int hd);
+int num_sms();
 
 namespace {
 
@@ -368,6 +369,428 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+
+// =========================================================================== pipelined, hd = 128
+// Persistent: one CTA per SM walks units (128-key tile, head, batch row),
+// ranked by decreasing cost and dealt in a snake order. A unit visits the
+// 64-query half-tiles that see its keys (at most 10 for W = 512); g counts
+// half-tiles over all of the CTA's units.
+//   S^T_g  = K Q_g^T, dP^T_g = V dO_g^T   128 keys x 64 queries, TMEM S[g&1], DP[g&1]
+//   P^T_g, dS^T_g                          bf16, shared memory buffer g&1
+//   dV += P^T_g dO_g, dK += dS^T_g Q_g     TMEM accumulators (whole unit)
+//   dQ^T_g = K^T dS^T_g                    128 channels x 64 queries, into S[g&1]
+// The MMA warp issues S/dP of half-tile g+1 before dV/dK/dQ of g, so the
+// tensor core works on g+1 while the softmax warps work on g. The softmax
+// warps drain dQ^T_{g-1} right after producing P/dS of g: TMEM -> registers
+// (S[(g-1)&1] released at once) -> 4 KiB slices of the free P^T/dS^T buffer
+// (g-1)&1 -> one 32 x 32 fp32 TMA reduce-add per warp. Q/dO arrive through
+// a 3-deep ring; K/V once per unit.
+__device__ __forceinline__ void store_half_row(uint8_t* tile, int r, const float* x, int half) {
+  // 32 values (columns 32*half .. +31) of row r of a [rows x 64] bf16 tile in
+  // 128B-swizzled K-major layout (one 64-column chunk, 128 B per row).
+#pragma unroll
+  for (int gg = 0; gg < 4; ++gg) {
+    const int g = half * 4 + gg;
+    uint4 w;
+    w.x = pack_bf16(x[8 * gg + 0], x[8 * gg + 1]);
+    w.y = pack_bf16(x[8 * gg + 2], x[8 * gg + 3]);
+    w.z = pack_bf16(x[8 * gg + 4], x[8 * gg + 5]);
+    w.w = pack_bf16(x[8 * gg + 6], x[8 * gg + 7]);
+    *reinterpret_cast<uint4*>(tile + r * 128 + ((g ^ (r & 7)) << 4)) = w;
+  }
+}
+
+template <int HD>
+struct PipeCfg {
+  static_assert(HD == 128, "pipelined backward is written for 128 channels");
+  static constexpr int CH = HD / 64;
+  static constexpr int KV_TILE = 128 * HD * 2;  // 128 keys
+  static constexpr int KCHUNK = 128 * 128;      // 128 rows x 64 bf16
+  static constexpr int QH = 64 * HD * 2;        // 64 queries
+  static constexpr int QCHUNK = 64 * 128;       // 64 rows x 64 bf16
+  static constexpr int NQ = 3;                  // Q / dO ring depth
+  static constexpr int PH = 128 * 64 * 2;       // [128 keys x 64 queries] bf16
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = KV_TILE;
+  static constexpr int OFF_Q = 2 * KV_TILE;
+  static constexpr int OFF_DO = OFF_Q + NQ * QH;
+  static constexpr int OFF_P = OFF_DO + NQ * QH;  // [2]
+  static constexpr int OFF_DS = OFF_P + 2 * PH;   // [2]
+  static constexpr int OFF_LD = OFF_DS + 2 * PH;  // [2][128] floats: LSE*log2e (64), Delta (64)
+  static constexpr int OFF_BAR = OFF_LD + 2 * 128 * 4;
+  static constexpr size_t SMEM = OFF_BAR + 256;   // base is 1024-aligned (checked in the kernel)
+  static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 384;  // S/dP: 64 columns x 2
+};
+
+struct PipeParams {
+  BwdParams b;
+  int n_ktiles, n_units;
+};
+
+struct KUnit {
+  int kt, h, b, nh;
+};
+
+// Rank r in decreasing cost: key tiles from the first (the last tiles see
+// fewer queries); snake over the CTAs per pass. -1 past the end.
+__device__ __forceinline__ int kunit_rank(const PipeParams& p, int k) {
+  const int G = (int)gridDim.x, c = (int)blockIdx.x;
+  const int r = k * G + ((k & 1) ? G - 1 - c : c);
+  return r < p.n_units ? r : -1;
+}
+
+__device__ __forceinline__ KUnit kunit_of(const PipeParams& p, int r) {
+  KUnit x;
+  const int hb = p.b.H * p.b.B;
+  x.kt = (r / hb) * 128;
+  x.h = (r % hb) % p.b.H;
+  x.b = (r % hb) / p.b.H;
+  const int last_q = min(p.b.T - 1, x.kt + 127 + p.b.W - 1);
+  x.nh = ((last_q & ~63) - x.kt) / 64 + 1;
+  return x;
+}
+
+template <int HD>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    attn_bwd_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                         const __grid_constant__ CUtensorMap tmDQ, PipeParams pp) {
+  using C = PipeCfg<HD>;
+  const BwdParams& p = pp.b;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {  // the swizzled tiles need a 1024-byte aligned base
+    if (threadIdx.x == 0) record_error(p.err, DEV_TIMEOUT);
+    return;
+  }
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* kv_empty = bars + 1;
+  uint64_t* q_full = bars + 2;     // [3]
+  uint64_t* q_empty = bars + 5;    // [3]
+  uint64_t* s_full = bars + 8;     // [2]
+  uint64_t* p_full = bars + 10;    // [2]
+  uint64_t* dq_full = bars + 12;   // [2]
+  uint64_t* dq_empty = bars + 14;  // [2]
+  uint64_t* acc_full = bars + 16;
+  uint64_t* acc_empty = bars + 17;
+  uint64_t* drain = bars + 18;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const Abort ab{abort_flag, p.err, p.spin_limit * 1000};
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], SOFT_THREADS);
+      mbar_init(&dq_full[s], 1);
+      mbar_init(&dq_empty[s], SOFT_THREADS);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, SOFT_THREADS);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmDO);
+    tma_prefetch_desc(&tmDQ);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      uint32_t kv_armed = 0, kv_par = 0, q_armed = 0, q_par = 0;
+      int g = 0, n = 0;
+      bool ok = true;
+      for (int u = kunit_rank(pp, 0); u >= 0 && ok; u = kunit_rank(pp, ++n)) {
+        const KUnit x = kunit_of(pp, u);
+        for (int j = 0; j < x.nh; ++j, ++g) {
+          const int s = g % 3;
+          const uint32_t ph = (uint32_t)(g / 3) & 1u;
+          if (!mbar_wait(&q_empty[s], ph ^ 1u, ab)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&q_full[s], 2 * C::QH);
+          q_armed |= 1u << s;
+          q_par = (q_par & ~(1u << s)) | (ph << s);
+          const int qt = x.kt + 64 * j;
+#pragma unroll
+          for (int c = 0; c < C::CH; ++c) {
+            tma_load_4d(smem + C::OFF_Q + s * C::QH + c * C::QCHUNK, &tmQ, &q_full[s], 64 * c, x.h, qt, x.b);
+            tma_load_4d(smem + C::OFF_DO + s * C::QH + c * C::QCHUNK, &tmDO, &q_full[s], 64 * c, x.h, qt, x.b);
+          }
+          if (j == 0) {  // the unit's K/V, once the previous unit's MMAs are done with them
+            const uint32_t kph = (uint32_t)n & 1u;
+            if (!mbar_wait(kv_empty, kph ^ 1u, ab)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(kv_full, 2 * C::KV_TILE);
+            kv_armed = 1;
+            kv_par = kph;
+#pragma unroll
+            for (int c = 0; c < C::CH; ++c) {
+              tma_load_4d(smem + C::OFF_K + c * C::KCHUNK, &tmK, kv_full, 64 * c, x.h, x.kt, x.b);
+              tma_load_4d(smem + C::OFF_V + c * C::KCHUNK, &tmV, kv_full, 64 * c, x.h, x.kt, x.b);
+            }
+          }
+        }
+      }
+      if (kv_armed) mbar_drain(kv_full, kv_par, DRAIN_LIMIT_NS);
+      for (int s = 0; s < 3; ++s)
+        if (q_armed & (1u << s)) mbar_drain(&q_full[s], (q_par >> s) & 1u, DRAIN_LIMIT_NS);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      constexpr uint32_t ID_S = idesc_bf16(128, 64, false, false);  // S^T, dP^T: 128 keys x 64 queries
+      constexpr uint32_t ID_KV = idesc_bf16(128, HD, false, true);  // dV, dK: 128 keys x hd
+      constexpr uint32_t ID_DQ = idesc_bf16(HD, 64, true, true);    // dQ^T: hd x 64 queries
+      const uint32_t k_addr = smem_u32(smem + C::OFF_K);
+      const uint32_t v_addr = smem_u32(smem + C::OFF_V);
+      // S^T_gs, dP^T_gs into buffer gs&1, once that buffer's dQ^T_{gs-2} is drained
+      auto issue_sdp = [&](int gs) -> bool {
+        const int s = gs % 3, buf = gs & 1;
+        if (!mbar_wait(&q_full[s], (uint32_t)(gs / 3) & 1u, ab)) return false;
+        if (gs >= 2 && !mbar_wait(&dq_empty[buf], (uint32_t)((gs - 2) >> 1) & 1u, ab)) return false;
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(smem + C::OFF_Q + s * C::QH);
+        const uint32_t do_addr = smem_u32(smem + C::OFF_DO + s * C::QH);
+#pragma unroll
+        for (int k16 = 0; k16 < HD / 16; ++k16) {
+          const uint32_t ka = (uint32_t)(k16 >> 2) * C::KCHUNK, qa = (uint32_t)(k16 >> 2) * C::QCHUNK;
+          mma_ss(tmem + C::T_S + 64u * buf, kmajor_desc(k_addr + ka, k16 & 3), kmajor_desc(q_addr + qa, k16 & 3),
+                 ID_S, k16 > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int k16 = 0; k16 < HD / 16; ++k16) {
+          const uint32_t ka = (uint32_t)(k16 >> 2) * C::KCHUNK, qa = (uint32_t)(k16 >> 2) * C::QCHUNK;
+          mma_ss(tmem + C::T_DP + 64u * buf, kmajor_desc(v_addr + ka, k16 & 3), kmajor_desc(do_addr + qa, k16 & 3),
+                 ID_S, k16 > 0 ? 1u : 0u);
+        }
+        mma_commit(&s_full[buf]);
+        return true;
+      };
+      int g = 0, n = 0;
+      bool ok = true;
+      for (int u = kunit_rank(pp, 0); u >= 0 && ok; u = kunit_rank(pp, ++n)) {
+        const KUnit x = kunit_of(pp, u);
+        if (!mbar_wait(kv_full, (uint32_t)n & 1u, ab) || !issue_sdp(g)) break;
+        for (int j = 0; j < x.nh; ++j, ++g) {
+          if (j + 1 < x.nh && !issue_sdp(g + 1)) {
+            ok = false;
+            break;
+          }
+          const int s = g % 3, buf = g & 1;
+          if (!mbar_wait(&p_full[buf], (uint32_t)(g >> 1) & 1u, ab)) {
+            ok = false;
+            break;
+          }
+          // the first dV/dK of a unit overwrites the accumulators: the previous
+          // unit's epilogue must have read them
+          if (j == 0 && !mbar_wait(acc_empty, ((uint32_t)n & 1u) ^ 1u, ab)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t q_addr = smem_u32(smem + C::OFF_Q + s * C::QH);
+          const uint32_t do_addr = smem_u32(smem + C::OFF_DO + s * C::QH);
+          const uint32_t p_addr = smem_u32(smem + C::OFF_P + buf * C::PH);
+          const uint32_t ds_addr = smem_u32(smem + C::OFF_DS + buf * C::PH);
+#pragma unroll
+          for (int k16 = 0; k16 < 4; ++k16) {  // K = 64 queries
+            mma_ss(tmem + C::T_DV, kmajor_desc(p_addr, k16),
+                   sw128_desc(do_addr + (uint32_t)k16 * 2048u, (uint32_t)C::QCHUNK, 1024u), ID_KV,
+                   (j > 0 || k16 > 0) ? 1u : 0u);
+          }
+#pragma unroll
+          for (int k16 = 0; k16 < 4; ++k16) {
+            mma_ss(tmem + C::T_DK, kmajor_desc(ds_addr, k16),
+                   sw128_desc(q_addr + (uint32_t)k16 * 2048u, (uint32_t)C::QCHUNK, 1024u), ID_KV,
+                   (j > 0 || k16 > 0) ? 1u : 0u);
+          }
+          mma_commit(&q_empty[s]);
+#pragma unroll
+          for (int k16 = 0; k16 < 8; ++k16) {  // K = 128 keys
+            mma_ss(tmem + C::T_S + 64u * buf, sw128_desc(k_addr + (uint32_t)k16 * 2048u, (uint32_t)C::KCHUNK, 1024u),
+                   sw128_desc(ds_addr + (uint32_t)k16 * 2048u, (uint32_t)C::PH, 1024u), ID_DQ, k16 > 0 ? 1u : 0u);
+          }
+          mma_commit(&dq_full[buf]);
+          if (j + 1 == x.nh) {
+            mma_commit(acc_full);
+            mma_commit(kv_empty);
+          }
+        }
+      }
+      mma_commit(drain);
+      mbar_drain(drain, 0, DRAIN_LIMIT_NS);
+    }
+  } else {
+    // -------------------------------------------------------------- softmax-backward / drains
+    const int q4 = warp & 3;
+    const int half = (warp - 2) >> 2;  // 32 of the 64 query columns
+    const int r = q4 * 32 + lane;      // TMEM lane: key row (S^T, dV, dK) / channel (dQ^T)
+    const int st = threadIdx.x - 64;   // 0..255 among the softmax threads
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    float* lds_all = reinterpret_cast<float*>(smem + C::OFF_LD);
+    bool ok = true;
+    // LSE / Delta of half-tile g, loaded one half-tile ahead by threads 0..127
+    float pre = 0.f;
+    auto fetch = [&](const KUnit& x, int j) {
+      if (st < 128) {
+        const int qi = x.kt + 64 * j + (st & 63);
+        const int64_t lrow = ((int64_t)x.b * p.H + x.h) * p.T;
+        pre = qi < p.T ? (st < 64 ? p.lse[lrow + qi] * LOG2E : p.delta[lrow + qi]) : 0.f;
+      }
+    };
+    // dQ^T of half-tile gd (unit xd, its local index jd): lanes are channels,
+    // this warp's 32 columns are queries xd.kt + 64*jd + 32*half ...
+    auto drain_dq = [&](int gd, const KUnit& xd, int jd) {
+      const int buf = gd & 1;
+      ok = ok && warp_wait(&dq_full[buf], (uint32_t)(gd >> 1) & 1u, ab);
+      if (!ok) return;
+      tc_fence_after();
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_off + C::T_S + 64u * (uint32_t)buf + 32u * (uint32_t)half, v);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&dq_empty[buf]);  // S[buf] may take S^T of half-tile gd + 2
+      // box of 32 query rows x 32 channels (128 B rows, 16-byte chunks swizzled by row)
+      const int w8 = q4 + 4 * half;
+      uint8_t* slice = smem + (w8 < 4 ? C::OFF_P : C::OFF_DS) + buf * C::PH + (w8 & 3) * 4096;
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        *reinterpret_cast<uint32_t*>(slice + c * 128 + ((((lane >> 2) ^ (c & 7))) << 4) + (lane & 3) * 4) = v[c];
+      fence_proxy_async_smem();
+      __syncwarp();
+      const int q0 = xd.kt + 64 * jd + 32 * half;
+      if (lane == 0 && q0 < p.T) {
+        tma_reduce_add_4d(&tmDQ, slice, 32 * q4, xd.h, q0, xd.b);
+        bulk_commit();
+      }
+    };
+    int g = 0, n = 0;
+    KUnit xp{0, 0, 0, 0};  // unit of half-tile g-1
+    int jp = 0;            // its local index
+    {
+      const int u0 = kunit_rank(pp, 0);
+      if (u0 >= 0) fetch(kunit_of(pp, u0), 0);
+    }
+    for (int u = kunit_rank(pp, 0); u >= 0; u = kunit_rank(pp, ++n)) {
+      const KUnit x = kunit_of(pp, u);
+      const int kj = x.kt + r;
+      const int kw = x.kt + 32 * q4;  // first key row of this warp
+      for (int j = 0; j < x.nh; ++j, ++g) {
+        const int buf = g & 1;
+        const int qt = x.kt + 64 * j;
+        float* lds = lds_all + buf * 128;  // [0,64) LSE*log2e, [64,128) Delta
+        // the reduce-adds of half-tile g-2 have read their staging in buffer g&1
+        if (lane == 0) bulk_wait_read_all();
+        if (st < 128) lds[st] = pre;
+        // every softmax thread reaches this barrier on every half-tile, aborted or not
+        asm volatile("bar.sync 1, %0;" ::"n"(SOFT_THREADS) : "memory");
+        if (j + 1 < x.nh) {
+          fetch(x, j + 1);
+        } else {
+          const int un = kunit_rank(pp, n + 1);
+          if (un >= 0) fetch(kunit_of(pp, un), 0);
+        }
+        ok = ok && warp_wait(&s_full[buf], (uint32_t)(g >> 1) & 1u, ab);
+        if (ok) {
+          tc_fence_after();
+          uint32_t sv[32], dv[32];
+          tmem_ld32(tmem + lane_off + C::T_S + 64u * buf + 32u * half, sv);
+          tmem_ld32(tmem + lane_off + C::T_DP + 64u * buf + 32u * half, dv);
+          tmem_wait_ld();
+          const int q0 = qt + 32 * half;  // first query column of this warp
+          const int lo = kj - q0;         // query >= key
+          const int hi = min(kj + p.W - 1, p.T - 1) - q0;
+          const bool full = q0 >= kw + 31 && q0 + 31 <= kw + p.W - 1 && q0 + 31 <= p.T - 1 && kw + 31 < p.T;
+          float pt[32], ds[32];
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 L = *reinterpret_cast<const float4*>(lds + 32 * half + 4 * e4);
+            const float4 D = *reinterpret_cast<const float4*>(lds + 64 + 32 * half + 4 * e4);
+            const float Ls[4] = {L.x, L.y, L.z, L.w};
+            const float Ds[4] = {D.x, D.y, D.z, D.w};
+#pragma unroll
+            for (int uu = 0; uu < 4; ++uu) {
+              const int e = 4 * e4 + uu;
+              const float y = ex2_fast(fmaf(__uint_as_float(sv[e]), p.scale_log2, -Ls[uu]));
+              const float pe = (full || (e >= lo && e <= hi && kj < p.T)) ? y : 0.f;
+              pt[e] = pe;
+              ds[e] = pe * (__uint_as_float(dv[e]) - Ds[uu]) * p.scale;
+            }
+          }
+          // buffer g&1: its MMAs (half-tile g-2) completed before dQ^T_{g-2} was drained
+          store_half_row(smem + C::OFF_P + buf * C::PH, r, pt, half);
+          store_half_row(smem + C::OFF_DS + buf * C::PH, r, ds, half);
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(&p_full[buf]);
+        }
+        if (g >= 1) drain_dq(g - 1, xp, jp);
+        xp = x;
+        jp = j;
+      }
+      // epilogue of the unit: dK, dV rows (fp32)
+      ok = ok && warp_wait(acc_full, (uint32_t)n & 1u, ab);
+      if (ok) {
+        tc_fence_after();
+        const bool row_ok = kj < p.T;
+        const int64_t row = (((int64_t)x.b * p.T + (row_ok ? kj : 0)) * p.H + x.h) * HD;
+        uint32_t vk[2][32], vv[2][32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          tmem_ld32(tmem + lane_off + C::T_DK + 64u * (uint32_t)half + 32u * (uint32_t)c, vk[c]);
+          tmem_ld32(tmem + lane_off + C::T_DV + 64u * (uint32_t)half + 32u * (uint32_t)c, vv[c]);
+        }
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(acc_empty);
+        if (row_ok) {
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+#pragma unroll
+            for (int g4 = 0; g4 < 8; ++g4) {
+              const int col = 64 * half + 32 * c + 4 * g4;
+              *reinterpret_cast<float4*>(p.dk_bar + row + col) =
+                  make_float4(__uint_as_float(vk[c][4 * g4]), __uint_as_float(vk[c][4 * g4 + 1]),
+                              __uint_as_float(vk[c][4 * g4 + 2]), __uint_as_float(vk[c][4 * g4 + 3]));
+              *reinterpret_cast<float4*>(p.dv_bar + row + col) =
+                  make_float4(__uint_as_float(vv[c][4 * g4]), __uint_as_float(vv[c][4 * g4 + 1]),
+                              __uint_as_float(vv[c][4 * g4 + 2]), __uint_as_float(vv[c][4 * g4 + 3]));
+            }
+          }
+        }
+      }
+    }
+    if (g >= 1) drain_dq(g - 1, xp, jp);
+    if (lane == 0) bulk_wait_all();  // dQ reductions complete before the CTA leaves
+    __syncwarp();
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_attn_bwd_tc(const SwaShape& s, const void* q_rot, const void* k_bar, const void* v_bar,
@@ -397,10 +820,18 @@ cudaError_t launch_attn_bwd_tc(const SwaShape& s, const void* q_rot, const void*
   p.err = err;
   dim3 grid((unsigned)((s.T + 127) / 128), (unsigned)s.H, (unsigned)s.B);
   if (s.hd == 128) {
-    auto k = attn_bwd_tc_kernel<128>;
-    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BwdCfg<128>::SMEM);
+    CUtensorMap tq64, tdo64;  // Q / dO in 64-row boxes for the half-tiles
+    if ((e = make_tmap_tokens(&tq64, q_rot, s.B, s.T, s.H, s.hd, 64)) != cudaSuccess) return e;
+    if ((e = make_tmap_tokens(&tdo64, dout, s.B, s.T, s.H, s.hd, 64)) != cudaSuccess) return e;
+    PipeParams pp;
+    pp.b = p;
+    pp.n_ktiles = (s.T + 127) / 128;
+    pp.n_units = pp.n_ktiles * s.H * s.B;
+    const unsigned pgrid = (unsigned)(pp.n_units < num_sms() ? pp.n_units : num_sms());
+    auto k = attn_bwd_pipe_kernel<128>;
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PipeCfg<128>::SMEM);
     if (e != cudaSuccess) return e;
-    k<<<grid, NUM_THREADS, BwdCfg<128>::SMEM, st>>>(tq, tk, tv, tdo, tdq, p);
+    k<<<pgrid, NUM_THREADS, PipeCfg<128>::SMEM, st>>>(tq64, tk, tv, tdo64, tdq, pp);
   } else if (s.hd == 64) {
     auto k = attn_bwd_tc_kernel<64>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BwdCfg<64>::SMEM);
