@@ -263,7 +263,7 @@ def shift_memory(m):
 
 
 def stack_forward_backward(q_layers, p_layers, w_mk, w_mv, lam: float, rope_base: float = 10000.0,
-                           eps: float = 1e-6, store=None):
+                           eps: float = 1e-6, store=None, inv_count: float | None = None):
     """One training step of a prefiller Q and a decoder P that share a memory.
 
     Q's layers (no injection; dicts with q, k, v, dout, window) run first;
@@ -278,6 +278,9 @@ def stack_forward_backward(q_layers, p_layers, w_mk, w_mv, lam: float, rope_base
     `store` (optional) maps the combined upstream gradient of each last layer
     (its dout plus the memory's gradient) to the values kept in storage, for
     comparison with an implementation that keeps it in a narrower type.
+    `inv_count` is the loss's 1/|I| (default 1/(B*T)); batch rows are
+    independent apart from |I| and the sums over rows (loss, dW, gate grads),
+    so a slice of rows with the full batch's |I| reproduces those rows.
     """
     store = store if store is not None else (lambda x: x)
     B, T, H, hd = q_layers[-1]["q"].shape
@@ -292,7 +295,7 @@ def stack_forward_backward(q_layers, p_layers, w_mk, w_mv, lam: float, rope_base
           for L in p_layers]
     op = pf[-1]["out"].reshape(B, T, D)
     m = memory_state(op, eps)
-    loss, dm, dm_prime = consistency_loss(m.reshape(B * T, D), m_prime.reshape(B * T, D), lam)
+    loss, dm, dm_prime = consistency_loss(m.reshape(B * T, D), m_prime.reshape(B * T, D), lam, inv_count)
     dm = dm.reshape(B, T, D)
     dm_prime = dm_prime.reshape(B, T, D)
 

@@ -78,3 +78,55 @@ def test_stack_f32_small():
     wl = dict(B=1, T=150, H=2, hd=64, dtype="f32", lam=1.0)
     S, ref = _run(wl, 1235, [32, 150], [32, 32])
     _check_all(S, ref, "f32")
+
+
+def _slice_b0(L):
+    out = {}
+    for k, v in L.items():
+        if isinstance(v, synth.Tensor):
+            out[k] = v.f64[:1]
+        elif k == "gates":
+            out[k] = v.astype(np.float64)
+        else:
+            out[k] = v
+    return out
+
+
+def test_stack_full_size_batch_row_0():
+    """Every launch at the benchmark's shape (B=8, T=2048, 10 heads of 128,
+    windows 512 and full 2048): a 2-layer SL prefiller and a 2-layer decoder.
+    Batch row 0 of every output and gradient is compared with the oracle run
+    on that row alone, with the loss's |I| of the whole batch."""
+    import torch
+    from sliding_window_recurrent_b200.stack import PrefillerDecoderStack
+
+    wl = dict(synth.WORKLOADS["stack20_bf16"])
+    B, T, H, hd = wl["B"], wl["T"], wl["H"], wl["hd"]
+    q_windows, p_windows = [512, T], [512, 512]
+    x = synth.stack_inputs(wl, 1234, q_windows, p_windows)
+    S = PrefillerDecoderStack(B, T, H, hd, q_windows, p_windows, lam=wl["lam"])
+    qi = [(dev(L["q"]), dev(L["k"]), dev(L["v"])) for L in x["q_layers"]]
+    pi = [(dev(L["q"]), dev(L["k"]), dev(L["v"]), dev(L["gates"])) for L in x["p_layers"]]
+    qd = [dev(L["dout"]) for L in x["q_layers"]]
+    pd = [dev(L["dout"]) for L in x["p_layers"]]
+    S.step(qi, pi, qd, pd, dev(x["w_mk"]), dev(x["w_mv"]))
+    torch.cuda.synchronize()
+
+    ref = oracle.stack_forward_backward([_slice_b0(L) for L in x["q_layers"]],
+                                        [_slice_b0(L) for L in x["p_layers"]],
+                                        x["w_mk"].f64, x["w_mv"].f64, wl["lam"], store=_bf16,
+                                        inv_count=1.0 / (B * T))
+    h0 = lambda t: host(t[:1])
+    for i, L in enumerate(S.q):
+        assert_close(h0(L.out), ref["q_out"][i], "bf16", f"Q{i} out")
+        for g in ("dq", "dk", "dv"):
+            assert_close(h0(getattr(L, g)), ref["q_grads"][i][g], "bf16", f"Q{i} {g}")
+    for i, L in enumerate(S.p):
+        assert_close(h0(L.out), ref["p_out"][i], "bf16", f"P{i} out")
+        for g in ("dq", "dk", "dv"):
+            assert_close(h0(getattr(L, g)), ref["p_grads"][i][g], "bf16", f"P{i} {g}")
+    assert_close(h0(S.m_prime), ref["m_prime"], "bf16", "m'")
+    assert_close(h0(S.m), ref["m"], "bf16", "m")
+    assert_close(h0(S.dm_shift), ref["dm_shift"], "bf16", "dm_shift")
+    assert_close(h0(S.dR_k), ref["dR_k"], "bf16", "dR_k")
+    assert_close(h0(S.dR_v), ref["dR_v"], "bf16", "dR_v")
