@@ -13,8 +13,14 @@
 
 #include "common.cuh"
 #include "launchers.h"
+#include "tc_common.cuh"
 
 namespace maglev {
+
+cudaError_t make_tmap_bf16_2d_plain(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                                    uint32_t box_inner, uint32_t box_rows);
+int num_sms();
+
 namespace {
 
 // In place: x[b,h,:] <- RoPE_{pos[b]}(RMSNorm(x[b,h,:])); one warp per (b,h).
@@ -153,15 +159,13 @@ __global__ void __launch_bounds__(256) decode_step_kernel(
 // ---------------------------------------------------------------------------
 // Ring attention for bf16 rings, one thread-block cluster of NS CTAs per (b,h).
 // CTA `rank` owns slots [rank*C, rank*C + C), C <= 128; warp w owns 32 of
-// them. Each lane loads 16-byte pieces of its K rows straight into registers
-// (all issued before any is used, so many bytes are in flight per SM), forms
-// partial dot products reduced over the lanes of a row, then does the same
-// for its V rows while the chunk softmax is formed. Four 128-thread CTAs fit
-// per SM (128 registers per thread), which overlaps one CTA's loads with
-// another's arithmetic. Rank 0 merges the NS partial
-// (max, sum, o) triples through distributed shared memory. The CTA whose
-// chunk holds slot p mod W writes the new entry to the ring and uses it in
-// place of the stale slot.
+// them. Two bulk copies bring the chunk's K and V rows into shared memory
+// (64 KiB per CTA in flight from the first cycle, three CTAs per SM); lanes
+// form partial dot products over 16-byte pieces of a row, reduced over the
+// row's lanes, then the same for V with the chunk softmax weights. Rank 0
+// merges the NS partial (max, sum, o) triples through distributed shared
+// memory. The CTA whose chunk holds slot p mod W writes the new entry to the
+// ring once its copies have landed and uses it in place of the stale slot.
 // ---------------------------------------------------------------------------
 constexpr int RING_ROWS = 128;  // slots per CTA at most
 constexpr int RING_THREADS = 128;
@@ -169,16 +173,21 @@ constexpr int RING_WARPS = RING_THREADS / 32;
 constexpr int ROWS_PER_WARP = RING_ROWS / RING_WARPS;
 
 template <int HD>
-__global__ void __launch_bounds__(RING_THREADS) decode_ring_kernel(
+__global__ void __launch_bounds__(RING_THREADS) decode_ring_bulk_kernel(
     DecShape s, int ns, int chunk, const int64_t* __restrict__ pos, const bf16* __restrict__ q,
     const bf16* __restrict__ k, const bf16* __restrict__ v, const bf16* __restrict__ krec,
     const bf16* __restrict__ vrec, const float* __restrict__ gates, bf16* __restrict__ kring,
-    bf16* __restrict__ vring, bf16* __restrict__ out, float scale) {
+    bf16* __restrict__ vring, bf16* __restrict__ out, float scale, int64_t limit_ns, int* err) {
   namespace cg = cooperative_groups;
   constexpr int HALF = HD / 2;
   constexpr int LPR = HD / 8;     // lanes per row (16 B each)
-  constexpr int RPW = 32 / LPR;   // rows per warp load step
-  constexpr int STEPS = ROWS_PER_WARP / RPW;  // load steps for the warp's rows
+  constexpr int RPW = 32 / LPR;   // rows per warp step
+  constexpr int STEPS = ROWS_PER_WARP / RPW;
+  extern __shared__ __align__(128) uint8_t dsm[];
+  bf16* ks = reinterpret_cast<bf16*>(dsm);                         // [RING_ROWS][HD]
+  bf16* vs = reinterpret_cast<bf16*>(dsm + RING_ROWS * HD * 2);    // [RING_ROWS][HD]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(dsm + 2 * RING_ROWS * HD * 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 1);
   __shared__ float qs[HD], kn[HD], vn[HD];
   __shared__ float sc[RING_ROWS];
   __shared__ float part_o[RING_WARPS][HD];
@@ -198,14 +207,18 @@ __global__ void __launch_bounds__(RING_THREADS) decode_ring_kernel(
   const int nlive = !valid_pos ? 0 : (p >= W - 1 ? W : (int)p + 1);
   const int live_rows = max(0, min(rows, nlive - r0));
   const int sub = lane / LPR, cl = (lane % LPR) * 8;
+  const tc::Abort ab{abort_flag, err, limit_ns};
 
-  // K rows of this warp -> registers (issued first, consumed after the new entry)
-  uint4 kv[STEPS];
-#pragma unroll
-  for (int i = 0; i < STEPS; ++i) {
-    const int r = warp * ROWS_PER_WARP + i * RPW + sub;
-    kv[i] = r < live_rows ? __ldg(reinterpret_cast<const uint4*>(kring + ring + (int64_t)(r0 + r) * HD + cl))
-                          : make_uint4(0, 0, 0, 0);
+  if (tid == 0) {
+    tc::mbar_init(bar, 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+    if (live_rows > 0) {
+      const uint32_t bytes = (uint32_t)live_rows * HD * 2;
+      tc::mbar_arrive_expect_tx(bar, 2 * bytes);
+      tc::bulk_load(ks, kring + ring + (int64_t)r0 * HD, bytes, bar);
+      tc::bulk_load(vs, vring + ring + (int64_t)r0 * HD, bytes, bar);
+    }
   }
   if (tid < HALF && valid_pos) {
     const int c = tid;
@@ -230,9 +243,12 @@ __global__ void __launch_bounds__(RING_THREADS) decode_ring_kernel(
     vn[c] = to_f(from_f<bf16>(v1));
     vn[c + HALF] = to_f(from_f<bf16>(v2));
   }
-  __syncthreads();
+  __syncthreads();  // barrier initialised, new entry formed
+  // the chunk has landed (or the wait gave up: scores of a failed chunk are not used)
+  const bool landed = live_rows == 0 || tc::mbar_wait(bar, 0, ab);
+  const int use_rows = landed ? live_rows : 0;
   const bool owner = valid_pos && slot >= r0 && slot < r0 + rows;
-  if (owner && tid < HD) {
+  if (owner && tid < HD) {  // the copy of this slot has completed: overwrite it in the ring
     kring[ring + (int64_t)slot * HD + tid] = from_f<bf16>(kn[tid]);
     vring[ring + (int64_t)slot * HD + tid] = from_f<bf16>(vn[tid]);
   }
@@ -246,8 +262,9 @@ __global__ void __launch_bounds__(RING_THREADS) decode_ring_kernel(
     if (r0 + r == slot) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) d = fmaf(qv[e], kn[cl + e], d);
-    } else {
-      const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&kv[i]);
+    } else if (r < use_rows) {
+      const uint4 u = *reinterpret_cast<const uint4*>(ks + r * HD + cl);
+      const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 f = __bfloat1622float2(hv[e]);
@@ -257,14 +274,7 @@ __global__ void __launch_bounds__(RING_THREADS) decode_ring_kernel(
     }
 #pragma unroll
     for (int o = LPR / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-    if ((lane % LPR) == 0) sc[r] = r < live_rows ? d * scale : -INFINITY;
-  }
-  // V rows of this warp -> registers while the chunk softmax is formed
-#pragma unroll
-  for (int i = 0; i < STEPS; ++i) {
-    const int r = warp * ROWS_PER_WARP + i * RPW + sub;
-    kv[i] = r < live_rows ? __ldg(reinterpret_cast<const uint4*>(vring + ring + (int64_t)(r0 + r) * HD + cl))
-                          : make_uint4(0, 0, 0, 0);
+    if ((lane % LPR) == 0) sc[r] = r < use_rows ? d * scale : -INFINITY;
   }
   __syncthreads();
   if (warp == 0) {
@@ -288,12 +298,14 @@ __global__ void __launch_bounds__(RING_THREADS) decode_ring_kernel(
 #pragma unroll
   for (int i = 0; i < STEPS; ++i) {
     const int r = warp * ROWS_PER_WARP + i * RPW + sub;
-    const float pr = r < live_rows ? sc[r] : 0.f;
     if (r0 + r == slot) {
+      const float pr = sc[r];
 #pragma unroll
       for (int e = 0; e < 8; ++e) o[e] = fmaf(pr, vn[cl + e], o[e]);
-    } else {
-      const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&kv[i]);
+    } else if (r < use_rows) {
+      const float pr = sc[r];
+      const uint4 u = *reinterpret_cast<const uint4*>(vs + r * HD + cl);
+      const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 f = __bfloat1622float2(hv[e]);
@@ -328,9 +340,277 @@ __global__ void __launch_bounds__(RING_THREADS) decode_ring_kernel(
       L += w * cluster.map_shared_rank(stat, r)[1];
       O += w * cluster.map_shared_rank(&part_o[0][0], r)[tid];
     }
-    out[tok + tid] = from_f<bf16>(valid_pos ? O / L : 0.f);
+    out[tok + tid] = from_f<bf16>(valid_pos && L > 0.f ? O / L : 0.f);
   }
   cluster.sync();  // remote reads done before any CTA of the cluster exits
+}
+
+// ---------------------------------------------------------------------------
+// Streaming ring attention for bf16 rings: persistent, one CTA per SM walks
+// (b,h) pairs with a stride of the grid and reads each window once. A
+// producer warp streams 128-slot chunks of K and V through a ring of
+// shared-memory stages with tiled TMA copies (a 2-D view of the ring, boxes of
+// 64 channels x 128 slots, alternating K_c, V_c), running on into the next
+// pair while the current one finishes; sixteen compute warps each own 8 rows
+// of every chunk and keep an online softmax (running max, sum and output,
+// log2 units) over their rows, merged at the end of the pair. The new entry
+// is formed at the start of the pair, used in place of slot p mod W, and
+// written to the ring after the pair's copies have landed.
+// ---------------------------------------------------------------------------
+constexpr int ST_ROWS = 128;          // slots per chunk
+constexpr int ST_WARPS = 16;          // compute warps
+constexpr int ST_THREADS = 32 * (ST_WARPS + 1);
+
+template <int HD>
+struct StreamCfg {
+  static constexpr int CH = HD / 64;                         // 64-channel boxes per row
+  static constexpr int BOX_BYTES = ST_ROWS * 64 * 2;         // 16 KiB
+  static constexpr int CHUNK_BYTES = CH * BOX_BYTES;         // one K or V chunk
+  static constexpr int NSTAGE = HD == 128 ? 6 : 12;          // 192 KiB
+  static constexpr int OFF_BAR = NSTAGE * CHUNK_BYTES;
+  static constexpr size_t SMEM = OFF_BAR + 256;
+};
+
+template <int HD>
+__global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
+    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, DecShape s,
+    const int64_t* __restrict__ pos, const bf16* __restrict__ q, const bf16* __restrict__ k,
+    const bf16* __restrict__ v, const bf16* __restrict__ krec, const bf16* __restrict__ vrec,
+    const float* __restrict__ gates, bf16* __restrict__ kring, bf16* __restrict__ vring, bf16* __restrict__ out,
+    float scale_log2, int64_t limit_ns, int* err) {
+  using C = StreamCfg<HD>;
+  constexpr int HALF = HD / 2;
+  constexpr int LPR = HD / 8;                // lanes per row (16 B each)
+  constexpr int RPS = 32 / LPR;              // rows per warp step
+  constexpr int WROWS = ST_ROWS / ST_WARPS;  // rows of a chunk per warp
+  constexpr int STEPS = WROWS / RPS;
+  constexpr int CT = 32 * ST_WARPS;          // compute threads
+  extern __shared__ __align__(1024) uint8_t dsm[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(dsm + C::OFF_BAR);   // [NSTAGE]
+  uint64_t* empty = full + C::NSTAGE;                                 // [NSTAGE]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + C::NSTAGE);
+  __shared__ float qs[HD], kn[HD], vn[HD];
+  __shared__ float wm[ST_WARPS], wl[ST_WARPS];
+  __shared__ float wo[ST_WARPS][HD];
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int W = s.W;
+  const int npairs = s.B * s.H;
+  const tc::Abort ab{abort_flag, err, limit_ns};
+  // live slots of pair bh: positions max(0, p-W+1)..p
+  auto live_of = [&](int bh) -> int {
+    const int64_t p = pos[bh / s.H];
+    return p < 0 ? 0 : (p >= W - 1 ? W : (int)p + 1);
+  };
+
+  if (tid == 0) {
+    for (int i = 0; i < C::NSTAGE; ++i) {
+      tc::mbar_init(&full[i], 1);
+      tc::mbar_init(&empty[i], ST_WARPS);
+    }
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+    tc::tma_prefetch_desc(&tmK);
+    tc::tma_prefetch_desc(&tmV);
+  }
+  __syncthreads();
+
+  if (warp == ST_WARPS) {
+    // ------------------------------------------------------------ producer
+    // streams K_c, V_c of every chunk of every pair of this CTA, in order
+    if (lane == 0) {
+      uint32_t armed = 0, par = 0;
+      int L = 0;
+      bool ok = true;
+      for (int bh = blockIdx.x; bh < npairs && ok; bh += gridDim.x) {
+        const int nchunks = (live_of(bh) + ST_ROWS - 1) / ST_ROWS;
+        for (int j = 0; j < 2 * nchunks; ++j, ++L) {  // j = 2c: K_c, j = 2c+1: V_c
+          const int st = L % C::NSTAGE;
+          const uint32_t ph = (uint32_t)(L / C::NSTAGE) & 1u;
+          if (!tc::mbar_wait(&empty[st], ph ^ 1u, ab)) {
+            ok = false;
+            break;
+          }
+          tc::mbar_arrive_expect_tx(&full[st], C::CHUNK_BYTES);
+          armed |= 1u << st;
+          par = (par & ~(1u << st)) | (ph << st);
+          const int row = bh * W + (j >> 1) * ST_ROWS;  // rows past the tensor arrive as zeros
+#pragma unroll
+          for (int c = 0; c < C::CH; ++c)
+            tc::tma_load_2d(dsm + st * C::CHUNK_BYTES + c * C::BOX_BYTES, (j & 1) ? &tmV : &tmK, &full[st], 64 * c,
+                            row);
+        }
+      }
+      // copies in flight land before the CTA leaves (needed only after an abort)
+      for (int st = 0; st < C::NSTAGE; ++st)
+        if (armed & (1u << st)) tc::mbar_drain(&full[st], (par >> st) & 1u, tc::DRAIN_LIMIT_NS);
+    }
+    return;  // takes no part in the compute warps' barriers
+  }
+  // ------------------------------------------------------------ compute warps
+  const int sub = lane / LPR, cl = (lane % LPR) * 8;
+  const int boff = (cl / 64) * C::BOX_BYTES + (cl % 64) * 2;  // byte offset of this lane's piece in a row
+  int L = 0;
+  bool ok = true;
+  for (int bh = blockIdx.x; bh < npairs; bh += gridDim.x) {
+    const int b = bh / s.H, h = bh % s.H;
+    const int64_t p = pos[b];
+    const int64_t tok = (int64_t)bh * HD;
+    const int64_t ring = (int64_t)bh * W * HD;
+    const bool valid_pos = p >= 0;
+    const int slot = valid_pos ? (int)(p % W) : -1;
+    const int nlive = live_of(bh);
+    const int nchunks = (nlive + ST_ROWS - 1) / ST_ROWS;
+    if (tid < HALF && valid_pos) {
+      const int c = tid;
+      float cs, sn;
+      rope_cos_sin(p, c, HD, s.log2_base, &cs, &sn);
+      const float q1 = to_f(q[tok + c]), q2 = to_f(q[tok + c + HALF]);
+      qs[c] = (q1 * cs - q2 * sn) * scale_log2;  // scores come out in log2 units
+      qs[c + HALF] = (q1 * sn + q2 * cs) * scale_log2;
+      const float k1 = to_f(k[tok + c]), k2 = to_f(k[tok + c + HALF]);
+      float a1 = k1 * cs - k2 * sn, a2 = k1 * sn + k2 * cs;
+      float v1 = to_f(v[tok + c]), v2 = to_f(v[tok + c + HALF]);
+      if (s.inject) {
+        const float gkl = gate_value(gates[0 * s.H + h]), gkr = gate_value(gates[1 * s.H + h]);
+        const float gvl = gate_value(gates[2 * s.H + h]), gvr = gate_value(gates[3 * s.H + h]);
+        a1 = gkl * a1 + gkr * to_f(krec[tok + c]);
+        a2 = gkl * a2 + gkr * to_f(krec[tok + c + HALF]);
+        v1 = gvl * v1 + gvr * to_f(vrec[tok + c]);
+        v2 = gvl * v2 + gvr * to_f(vrec[tok + c + HALF]);
+      }
+      kn[c] = to_f(from_f<bf16>(a1));  // the step attends to exactly what it stores
+      kn[c + HALF] = to_f(from_f<bf16>(a2));
+      vn[c] = to_f(from_f<bf16>(v1));
+      vn[c + HALF] = to_f(from_f<bf16>(v2));
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(CT) : "memory");  // the pair's q and new entry are ready
+    float qv[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) qv[e] = qs[cl + e];
+    float m = -INFINITY, l = 0.f;  // log2 units, over the rows this lane-group has seen
+    float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int c = 0; c < nchunks; ++c, L += 2) {
+      if (!ok) continue;  // after an abort the remaining chunks are skipped
+      const int sk = L % C::NSTAGE, sv = (L + 1) % C::NSTAGE;
+      if (!tc::mbar_wait(&full[sk], (uint32_t)(L / C::NSTAGE) & 1u, ab)) {
+        ok = false;
+        continue;
+      }
+      const uint8_t* kc = dsm + sk * C::CHUNK_BYTES + boff;
+      float sc[STEPS];
+      float cmax = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < STEPS; ++i) {
+        const int r = warp * WROWS + i * RPS + sub;  // row within the chunk
+        const int gr = c * ST_ROWS + r;              // ring slot
+        float d0 = 0.f, d1 = 0.f;
+        if (gr == slot) {
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            d0 = fmaf(qv[e], kn[cl + e], d0);
+            d1 = fmaf(qv[e + 1], kn[cl + e + 1], d1);
+          }
+        } else {
+          const uint4 u = *reinterpret_cast<const uint4*>(kc + r * 128);
+          const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(hv[e]);
+            d0 = fmaf(qv[2 * e], f.x, d0);
+            d1 = fmaf(qv[2 * e + 1], f.y, d1);
+          }
+        }
+        float d = d0 + d1;
+#pragma unroll
+        for (int off = LPR / 2; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+        sc[i] = gr < nlive ? d : -INFINITY;
+        cmax = fmaxf(cmax, sc[i]);
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&empty[sk]);  // K_c read by this warp
+      // online softmax over this lane-group's rows (log2 units)
+      const float mn = fmaxf(m, cmax);
+      const float alpha = (m == -INFINITY) ? 0.f : tc::ex2_fast(m - mn);
+      const float nm = mn == -INFINITY ? 0.f : -mn;
+      float pr[STEPS];
+      float ps = 0.f;
+#pragma unroll
+      for (int i = 0; i < STEPS; ++i) {
+        pr[i] = tc::ex2_fast(sc[i] + nm);  // -inf gives 0
+        ps += pr[i];
+      }
+      l = l * alpha + ps;
+      m = mn;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] *= alpha;
+      if (!tc::mbar_wait(&full[sv], (uint32_t)((L + 1) / C::NSTAGE) & 1u, ab)) {
+        ok = false;
+        continue;
+      }
+      const uint8_t* vc = dsm + sv * C::CHUNK_BYTES + boff;
+#pragma unroll
+      for (int i = 0; i < STEPS; ++i) {
+        const int r = warp * WROWS + i * RPS + sub;
+        const int gr = c * ST_ROWS + r;
+        if (gr == slot) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[e] = fmaf(pr[i], vn[cl + e], o[e]);
+        } else if (gr < nlive) {  // dead slots may hold anything, NaN included
+          const uint4 u = *reinterpret_cast<const uint4*>(vc + r * 128);
+          const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(hv[e]);
+            o[2 * e] = fmaf(pr[i], f.x, o[2 * e]);
+            o[2 * e + 1] = fmaf(pr[i], f.y, o[2 * e + 1]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&empty[sv]);  // V_c read by this warp
+    }
+    // merge the RPS lane-groups of the warp (same channels, different rows)
+#pragma unroll
+    for (int off = LPR; off < 32; off <<= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+      const float l2 = __shfl_xor_sync(0xffffffffu, l, off);
+      const float mn = fmaxf(m, m2);
+      const float a1 = m == -INFINITY ? 0.f : tc::ex2_fast(m - mn);
+      const float a2 = m2 == -INFINITY ? 0.f : tc::ex2_fast(m2 - mn);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = o[e] * a1 + __shfl_xor_sync(0xffffffffu, o[e], off) * a2;
+      l = l * a1 + l2 * a2;
+      m = mn;
+    }
+    if (lane < LPR) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) wo[warp][cl + e] = o[e];
+    }
+    if (lane == 0) {
+      wm[warp] = ok ? m : -INFINITY;
+      wl[warp] = ok ? l : 0.f;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(CT) : "memory");  // every warp's partial is in
+    // merge the warps; write the new entry now that the pair's copies have landed
+    if (tid < HD) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < ST_WARPS; ++w) M = fmaxf(M, wm[w]);
+      float Ls = 0.f, O = 0.f;
+#pragma unroll
+      for (int w = 0; w < ST_WARPS; ++w) {
+        const float a = wm[w] == -INFINITY ? 0.f : tc::ex2_fast(wm[w] - M);
+        Ls += a * wl[w];
+        O += a * wo[w][tid];
+      }
+      out[tok + tid] = from_f<bf16>(valid_pos && Ls > 0.f ? O / Ls : 0.f);
+      if (valid_pos && ok) {
+        kring[ring + (int64_t)slot * HD + tid] = from_f<bf16>(kn[tid]);
+        vring[ring + (int64_t)slot * HD + tid] = from_f<bf16>(vn[tid]);
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(CT) : "memory");  // q, new entry, partials free again
+  }
 }
 
 }  // namespace
@@ -357,15 +637,47 @@ cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void
                                const float* gates, void* k_ring, void* v_ring, void* out,
                                int64_t limit_us, int* err, cudaStream_t st) {
   const float scale = 1.0f / sqrtf((float)s.hd);
-  if (s.dtype == 1 && (s.hd == 128 || s.hd == 64) && s.W <= 8 * RING_ROWS) {
-    (void)limit_us;  // the ring kernel has no asynchronous waits
-    (void)err;
+  if (s.dtype == 1 && (s.hd == 128 || s.hd == 64)) {
+    const int64_t limit_ns = (limit_us > 0 ? limit_us : DEFAULT_SPIN_LIMIT) * 1000;
+    if (s.B * s.H == 0) return cudaSuccess;
+    // the rings as 2-D [B*H*W, hd] tensors, boxes of 64 channels x 128 slots
+    CUtensorMap tk, tv;
+    const uint64_t nrows = (uint64_t)s.B * s.H * s.W;
+    cudaError_t te = make_tmap_bf16_2d_plain(&tk, k_ring, (uint64_t)s.hd, nrows, 64, ST_ROWS);
+    if (te != cudaSuccess) return te;
+    te = make_tmap_bf16_2d_plain(&tv, v_ring, (uint64_t)s.hd, nrows, 64, ST_ROWS);
+    if (te != cudaSuccess) return te;
+    const float scale_log2 = 1.4426950408889634f * scale;
+    const unsigned grid = (unsigned)(s.B * s.H < num_sms() ? s.B * s.H : num_sms());  // persistent
+    if (s.hd == 128) {
+      auto kern = decode_stream_kernel<128>;
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)StreamCfg<128>::SMEM);
+      if (e != cudaSuccess) return e;
+      kern<<<grid, ST_THREADS, StreamCfg<128>::SMEM, st>>>(tk, tv, s, pos, (const bf16*)q, (const bf16*)k,
+                                                               (const bf16*)v, (const bf16*)krec, (const bf16*)vrec,
+                                                               gates, (bf16*)k_ring, (bf16*)v_ring, (bf16*)out,
+                                                               scale_log2, limit_ns, err);
+    } else {
+      auto kern = decode_stream_kernel<64>;
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)StreamCfg<64>::SMEM);
+      if (e != cudaSuccess) return e;
+      kern<<<grid, ST_THREADS, StreamCfg<64>::SMEM, st>>>(tk, tv, s, pos, (const bf16*)q, (const bf16*)k,
+                                                              (const bf16*)v, (const bf16*)krec, (const bf16*)vrec,
+                                                              gates, (bf16*)k_ring, (bf16*)v_ring, (bf16*)out,
+                                                              scale_log2, limit_ns, err);
+    }
+    return cudaGetLastError();
+  }
+  if (false) {
     const int ns = (s.W + RING_ROWS - 1) / RING_ROWS;
     const int chunk = (s.W + ns - 1) / ns;
+    const size_t dyn = 2 * (size_t)RING_ROWS * s.hd * 2 + 64;  // K and V chunk, barrier, abort flag
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(s.B * s.H * ns));
     cfg.blockDim = dim3(RING_THREADS);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = dyn;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -374,13 +686,21 @@ cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (s.hd == 128)
-      return cudaLaunchKernelEx(&cfg, decode_ring_kernel<128>, s, ns, chunk, pos, (const bf16*)q, (const bf16*)k,
-                                (const bf16*)v, (const bf16*)krec, (const bf16*)vrec, gates, (bf16*)k_ring,
-                                (bf16*)v_ring, (bf16*)out, scale);
-    return cudaLaunchKernelEx(&cfg, decode_ring_kernel<64>, s, ns, chunk, pos, (const bf16*)q, (const bf16*)k,
+    const int64_t limit_ns = (limit_us > 0 ? limit_us : DEFAULT_SPIN_LIMIT) * 1000;
+    if (s.hd == 128) {
+      cudaError_t e = cudaFuncSetAttribute(decode_ring_bulk_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)dyn);
+      if (e != cudaSuccess) return e;
+      return cudaLaunchKernelEx(&cfg, decode_ring_bulk_kernel<128>, s, ns, chunk, pos, (const bf16*)q,
+                                (const bf16*)k, (const bf16*)v, (const bf16*)krec, (const bf16*)vrec, gates,
+                                (bf16*)k_ring, (bf16*)v_ring, (bf16*)out, scale, limit_ns, err);
+    }
+    cudaError_t e = cudaFuncSetAttribute(decode_ring_bulk_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)dyn);
+    if (e != cudaSuccess) return e;
+    return cudaLaunchKernelEx(&cfg, decode_ring_bulk_kernel<64>, s, ns, chunk, pos, (const bf16*)q, (const bf16*)k,
                               (const bf16*)v, (const bf16*)krec, (const bf16*)vrec, gates, (bf16*)k_ring,
-                              (bf16*)v_ring, (bf16*)out, scale);
+                              (bf16*)v_ring, (bf16*)out, scale, limit_ns, err);
   }
   const size_t smem = (size_t)s.W * sizeof(float);
   MAGLEV_DISPATCH2(s.dtype, s.hd, {

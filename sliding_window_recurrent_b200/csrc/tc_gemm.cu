@@ -306,6 +306,28 @@ cudaError_t make_tmap_tokens(CUtensorMap* m, const void* base, int B, int T, int
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// bf16 [rows, inner] row-major tensor without swizzle (the box lands row-major
+// in shared memory), box {box_inner, box_rows}; inner * 2 bytes per row.
+cudaError_t make_tmap_bf16_2d_plain(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                                    uint32_t box_inner, uint32_t box_rows) {
+  std::call_once(g_encode_once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  if (!g_encode) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // fp32 [B,T,H,hd] token tensor, box {32 channels, 1 head, 32 rows, 1}, 128B
 // swizzle: the target of the dQ reduce-add of the attention backward.
 cudaError_t make_tmap_f32_tokens(CUtensorMap* m, void* base, int B, int T, int H, int hd) {
