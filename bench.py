@@ -41,7 +41,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) per launch from ncu captures, keyed by trace name;
 # each entry records the sha256 of the kernel source it was taken on, and is
 # ignored once that source changes.
-NCU_TRAFFIC: dict[str, dict] = {}
+NCU_TRAFFIC: dict[str, dict] = {
+    # ncu --set full on the timed step's launches (profiles/ncu_attn_layer_bf16.md)
+    "attn_bwd_tc": {"bytes": 204036864, "src": "tc_attn_bwd.cu", "src_sha": "ee73a005eb511859"},
+    "attn_fwd_tc": {"bytes": 68504064, "src": "tc_attn_fwd.cu", "src_sha": "599bc5b79289372c"},
+    # one launch of the 64 x 10 x 512 x 128 ring step (profiles/ncu_decode_step.md)
+    "decode_step": {"bytes": 172343552, "src": "decode.cu", "src_sha": "ab1ab99dee605d36"},
+}
 
 
 # --------------------------------------------------------------------------- work model
@@ -496,9 +502,11 @@ def run_decode_bench(torch, dev, steps, warmup, peaks):
         calls, tot, _ = prof["decode_step"]
         avg = tot / calls
         gbs = ring_bytes / (avg * 1e-3) / 1e9
+        tr = NCU_TRAFFIC.get("decode_step")
         roof = {"kernel": "decode_step", "bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4), "avg_launch_ms": round(avg, 5),
-                "bytes_per_launch": ring_bytes}
+                "bytes_per_launch": ring_bytes,
+                "traffic": tr["bytes"] if tr and tr.get("src_sha") == src_sha(tr.get("src", "")) else None}
     return {"tokens_per_s": B * 1000.0 / ms, "ms_per_step": ms, "roofline": roof,
             "kernels": {n: {"calls": v[0], "ms_total": round(v[1], 4)} for n, v in prof.items()},
             "workload": f"decode B={B} L={L} H={H}x{hd} d={d} ring W={W}, pos from {c['first_pos']}, CUDA graph"}

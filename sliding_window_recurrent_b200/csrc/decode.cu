@@ -11,6 +11,8 @@
 // attends over the live slots (positions max(0, p-W+1)..p).
 #include <cooperative_groups.h>
 
+#include <cmath>
+
 #include "common.cuh"
 #include "launchers.h"
 #include "tc_common.cuh"
@@ -357,6 +359,11 @@ __global__ void __launch_bounds__(RING_THREADS) decode_ring_bulk_kernel(
 // is formed at the start of the pair, used in place of slot p mod W, and
 // written to the ring after the pair's copies have landed.
 // ---------------------------------------------------------------------------
+// RoPE frequencies base^(-2c/hd), computed once on the host (double).
+struct RopeFreq {
+  double inv_freq[64];
+};
+
 constexpr int ST_ROWS = 128;          // slots per chunk
 constexpr int ST_WARPS = 16;          // compute warps
 constexpr int ST_THREADS = 32 * (ST_WARPS + 1);
@@ -377,7 +384,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
     const int64_t* __restrict__ pos, const bf16* __restrict__ q, const bf16* __restrict__ k,
     const bf16* __restrict__ v, const bf16* __restrict__ krec, const bf16* __restrict__ vrec,
     const float* __restrict__ gates, bf16* __restrict__ kring, bf16* __restrict__ vring, bf16* __restrict__ out,
-    float scale_log2, int64_t limit_ns, int* err) {
+    float scale_log2, int64_t limit_ns, int* err, const __grid_constant__ RopeFreq rf) {
   using C = StreamCfg<HD>;
   constexpr int HALF = HD / 2;
   constexpr int LPR = HD / 8;                // lanes per row (16 B each)
@@ -462,8 +469,11 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
     const int nchunks = (nlive + ST_ROWS - 1) / ST_ROWS;
     if (tid < HALF && valid_pos) {
       const int c = tid;
+      // angle p * theta_c reduced to [-pi, pi] in double before the float sincos
+      double ang = (double)p * rf.inv_freq[c];
+      ang -= 6.283185307179586476925286766559 * rint(ang * 0.15915494309189533577);
       float cs, sn;
-      rope_cos_sin(p, c, HD, s.log2_base, &cs, &sn);
+      sincosf((float)ang, &sn, &cs);
       const float q1 = to_f(q[tok + c]), q2 = to_f(q[tok + c + HALF]);
       qs[c] = (q1 * cs - q2 * sn) * scale_log2;  // scores come out in log2 units
       qs[c + HALF] = (q1 * sn + q2 * cs) * scale_log2;
@@ -648,6 +658,9 @@ cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void
     te = make_tmap_bf16_2d_plain(&tv, v_ring, (uint64_t)s.hd, nrows, 64, ST_ROWS);
     if (te != cudaSuccess) return te;
     const float scale_log2 = 1.4426950408889634f * scale;
+    RopeFreq rf{};
+    const double base = std::exp2(s.log2_base);
+    for (int c = 0; c < s.hd / 2 && c < 64; ++c) rf.inv_freq[c] = std::pow(base, -2.0 * c / s.hd);
     const unsigned grid = (unsigned)(s.B * s.H < num_sms() ? s.B * s.H : num_sms());  // persistent
     if (s.hd == 128) {
       auto kern = decode_stream_kernel<128>;
@@ -657,7 +670,7 @@ cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void
       kern<<<grid, ST_THREADS, StreamCfg<128>::SMEM, st>>>(tk, tv, s, pos, (const bf16*)q, (const bf16*)k,
                                                                (const bf16*)v, (const bf16*)krec, (const bf16*)vrec,
                                                                gates, (bf16*)k_ring, (bf16*)v_ring, (bf16*)out,
-                                                               scale_log2, limit_ns, err);
+                                                               scale_log2, limit_ns, err, rf);
     } else {
       auto kern = decode_stream_kernel<64>;
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -666,7 +679,7 @@ cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void
       kern<<<grid, ST_THREADS, StreamCfg<64>::SMEM, st>>>(tk, tv, s, pos, (const bf16*)q, (const bf16*)k,
                                                               (const bf16*)v, (const bf16*)krec, (const bf16*)vrec,
                                                               gates, (bf16*)k_ring, (bf16*)v_ring, (bf16*)out,
-                                                              scale_log2, limit_ns, err);
+                                                              scale_log2, limit_ns, err, rf);
     }
     return cudaGetLastError();
   }
