@@ -747,38 +747,51 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         xp = x;
         jp = j;
       }
-      // epilogue of the unit: dK, dV rows (fp32)
+      // epilogue of the unit: dK, dV rows (fp32). Each warp's 32 rows x 64
+      // columns go through its own 8 KiB of the P^T / dS^T buffers (free: the
+      // unit's MMAs are complete and the pending dQ reduce-adds have read their
+      // staging), so that every global store covers two whole 256-byte row pieces.
       ok = ok && warp_wait(acc_full, (uint32_t)n & 1u, ab);
+      if (lane == 0) bulk_wait_read_all();
+      asm volatile("bar.sync 1, %0;" ::"n"(SOFT_THREADS) : "memory");  // reached by every softmax thread
       if (ok) {
         tc_fence_after();
-        const bool row_ok = kj < p.T;
-        const int64_t row = (((int64_t)x.b * p.T + (row_ok ? kj : 0)) * p.H + x.h) * HD;
-        uint32_t vk[2][32], vv[2][32];
+        uint8_t* stg = smem + C::OFF_P + (q4 + 4 * half) * 8192;  // [32 rows][64 fp32], 16-byte chunks swizzled
+        const int64_t tstride = (int64_t)p.H * HD;                // floats between consecutive tokens
+        const int64_t col0 = (int64_t)x.h * HD + 64 * half;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          tmem_ld32(tmem + lane_off + C::T_DK + 64u * (uint32_t)half + 32u * (uint32_t)c, vk[c]);
-          tmem_ld32(tmem + lane_off + C::T_DV + 64u * (uint32_t)half + 32u * (uint32_t)c, vv[c]);
-        }
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(acc_empty);
-        if (row_ok) {
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-#pragma unroll
-            for (int g4 = 0; g4 < 8; ++g4) {
-              const int col = 64 * half + 32 * c + 4 * g4;
-              *reinterpret_cast<float4*>(p.dk_bar + row + col) =
-                  make_float4(__uint_as_float(vk[c][4 * g4]), __uint_as_float(vk[c][4 * g4 + 1]),
-                              __uint_as_float(vk[c][4 * g4 + 2]), __uint_as_float(vk[c][4 * g4 + 3]));
-              *reinterpret_cast<float4*>(p.dv_bar + row + col) =
-                  make_float4(__uint_as_float(vv[c][4 * g4]), __uint_as_float(vv[c][4 * g4 + 1]),
-                              __uint_as_float(vv[c][4 * g4 + 2]), __uint_as_float(vv[c][4 * g4 + 3]));
-            }
+        for (int t = 0; t < 2; ++t) {  // dK, then dV
+          uint32_t v[2][32];
+          const uint32_t tcol = (t == 0 ? C::T_DK : C::T_DV) + 64u * (uint32_t)half;
+          tmem_ld32(tmem + lane_off + tcol, v[0]);
+          tmem_ld32(tmem + lane_off + tcol + 32u, v[1]);
+          tmem_wait_ld();
+          if (t == 1) {  // both accumulators are in registers or stored: the next unit may overwrite them
+            tc_fence_before();
+            mbar_arrive(acc_empty);
           }
+#pragma unroll
+          for (int c4 = 0; c4 < 16; ++c4)
+            *reinterpret_cast<uint4*>(stg + lane * 256 + ((c4 ^ (lane & 15)) << 4)) =
+                make_uint4(v[c4 >> 3][4 * (c4 & 7)], v[c4 >> 3][4 * (c4 & 7) + 1], v[c4 >> 3][4 * (c4 & 7) + 2],
+                           v[c4 >> 3][4 * (c4 & 7) + 3]);
+          __syncwarp();
+          float* dst = t == 0 ? p.dk_bar : p.dv_bar;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int r = 2 * i + (lane >> 4), ch = lane & 15;
+            const uint4 w = *reinterpret_cast<const uint4*>(stg + r * 256 + ((ch ^ (r & 15)) << 4));
+            const int key = x.kt + 32 * q4 + r;
+            if (key < p.T)
+              *reinterpret_cast<uint4*>(dst + ((int64_t)x.b * p.T + key) * tstride + col0 + 4 * ch) = w;
+          }
+          __syncwarp();
         }
       }
     }
+    // the last drain stages into buffers the epilogue staged through: every warp
+    // must be done with its epilogue first
+    asm volatile("bar.sync 1, %0;" ::"n"(SOFT_THREADS) : "memory");
     if (g >= 1) drain_dq(g - 1, xp, jp);
     if (lane == 0) bulk_wait_all();  // dQ reductions complete before the CTA leaves
     __syncwarp();
