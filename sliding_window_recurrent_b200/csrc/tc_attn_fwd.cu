@@ -375,7 +375,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
       }
       tc_fence_after();
       const float inv = 1.f / l;
-      bf16* dst = static_cast<bf16*>(p.out) + (((int64_t)x.b * p.T + i) * p.H + x.h) * HD;
+      // 64 columns at a time through this warp's own 32 rows of the P buffer
+      // (free: the unit's last PV has completed; only this warp writes them
+      // next), read back so that each warp-wide store covers four whole
+      // 128-byte row pieces
+      uint8_t* stg = sP + q * 4096;
+      const int64_t tstride = (int64_t)p.H * HD;  // elements between consecutive tokens
+      bf16* obase = static_cast<bf16*>(p.out) + ((int64_t)x.b * p.T + i_lo) * tstride + (int64_t)x.h * HD;
 #pragma unroll 1
       for (int c = 0; c < HD / 64; ++c) {
         uint32_t o2[2][32];
@@ -387,17 +393,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
           tc_fence_before();
           mbar_arrive(o_empty);
         }
-        if (i < p.T) {
 #pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8) {
-            uint4 w;
-            w.x = pack_bf16(__uint_as_float(o[8 * c8 + 0]) * inv, __uint_as_float(o[8 * c8 + 1]) * inv);
-            w.y = pack_bf16(__uint_as_float(o[8 * c8 + 2]) * inv, __uint_as_float(o[8 * c8 + 3]) * inv);
-            w.z = pack_bf16(__uint_as_float(o[8 * c8 + 4]) * inv, __uint_as_float(o[8 * c8 + 5]) * inv);
-            w.w = pack_bf16(__uint_as_float(o[8 * c8 + 6]) * inv, __uint_as_float(o[8 * c8 + 7]) * inv);
-            *reinterpret_cast<uint4*>(dst + 64 * c + 8 * c8) = w;
-          }
+        for (int c8 = 0; c8 < 8; ++c8) {
+          uint4 w;
+          w.x = pack_bf16(__uint_as_float(o[8 * c8 + 0]) * inv, __uint_as_float(o[8 * c8 + 1]) * inv);
+          w.y = pack_bf16(__uint_as_float(o[8 * c8 + 2]) * inv, __uint_as_float(o[8 * c8 + 3]) * inv);
+          w.z = pack_bf16(__uint_as_float(o[8 * c8 + 4]) * inv, __uint_as_float(o[8 * c8 + 5]) * inv);
+          w.w = pack_bf16(__uint_as_float(o[8 * c8 + 6]) * inv, __uint_as_float(o[8 * c8 + 7]) * inv);
+          *reinterpret_cast<uint4*>(stg + lane * 128 + ((c8 ^ (lane & 7)) << 4)) = w;
         }
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int rr = 4 * k + (lane >> 3), j = lane & 7;  // row of the warp's 32, 16-byte chunk
+          const uint4 w = *reinterpret_cast<const uint4*>(stg + rr * 128 + ((j ^ (rr & 7)) << 4));
+          if (i_lo + rr < p.T) *reinterpret_cast<uint4*>(obase + rr * tstride + 64 * c + 8 * j) = w;
+        }
+        __syncwarp();
       }
       if (i < p.T) p.lse[((int64_t)x.b * p.H + x.h) * p.T + i] = (m_ref + log2f(l)) * 0.69314718055994531f;
     }

@@ -47,7 +47,8 @@ struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
   static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+  static constexpr int OFF_EPI = STAGES * STAGE_BYTES + 256;  // 4 warps x [32 rows x 128 B] output staging
+  static constexpr size_t SMEM = 1024 + (size_t)OFF_EPI + 4 * 4096;
 };
 
 template <int BN, bool A_MN, bool B_MN>
@@ -201,8 +202,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // -------------------------------------------------------------- epilogue
+    // 64 columns at a time: TMEM -> bf16 -> the warp's 4 KiB of staging
+    // (16-byte chunks swizzled by row) -> read back so that each warp-wide
+    // store covers four whole 128-byte row pieces.
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;
+    uint8_t* stg = smem + C::OFF_EPI + q * 4096;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
@@ -223,24 +228,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       const int n_lim = (p.out_switch_n > 0 && n0 < p.out_switch_n) ? p.out_switch_n : p.N;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c0), r);
+      for (int c0 = 0; c0 < BN; c0 += 64) {
+        uint32_t r[2][32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c0), r[0]);
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c0 + 32), r[1]);
         tmem_wait_ld();
-        if (gm < p.M && n0 + c0 < n_lim) {
-          bf16* dst = out + (int64_t)om * p.ldo + on0 + c0;
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            if (n0 + c0 + 8 * g < n_lim) {
-              uint4 v;
-              v.x = pack_bf16(__uint_as_float(r[8 * g + 0]), __uint_as_float(r[8 * g + 1]));
-              v.y = pack_bf16(__uint_as_float(r[8 * g + 2]), __uint_as_float(r[8 * g + 3]));
-              v.z = pack_bf16(__uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5]));
-              v.w = pack_bf16(__uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7]));
-              *reinterpret_cast<uint4*>(dst + 8 * g) = v;
-            }
-          }
+        for (int j = 0; j < 8; ++j) {
+          uint4 v;
+          v.x = pack_bf16(__uint_as_float(r[j >> 2][8 * (j & 3) + 0]), __uint_as_float(r[j >> 2][8 * (j & 3) + 1]));
+          v.y = pack_bf16(__uint_as_float(r[j >> 2][8 * (j & 3) + 2]), __uint_as_float(r[j >> 2][8 * (j & 3) + 3]));
+          v.z = pack_bf16(__uint_as_float(r[j >> 2][8 * (j & 3) + 4]), __uint_as_float(r[j >> 2][8 * (j & 3) + 5]));
+          v.w = pack_bf16(__uint_as_float(r[j >> 2][8 * (j & 3) + 6]), __uint_as_float(r[j >> 2][8 * (j & 3) + 7]));
+          *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) = v;
         }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 4 * i + (lane >> 3), j = lane & 7;  // row of the warp's 32, 16-byte chunk
+          const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 128 + ((j ^ (rr & 7)) << 4));
+          const int col = n0 + c0 + 8 * j;
+          if (m0 + q * 32 + rr < p.M && col + 8 <= n_lim)
+            *reinterpret_cast<uint4*>(out + (int64_t)(om - lane + rr) * p.ldo + on0 + c0 + 8 * j) = v;
+        }
+        __syncwarp();
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
