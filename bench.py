@@ -107,8 +107,8 @@ def kernel_work(name: str, cfg: dict) -> tuple[float, str]:
         "mem_project_bwd_dw_tc": (f["proj_fwd"], "flop"),
         # reads q, k, v, R_k, R_v; writes q_rot, k_bar, v_bar (bf16)
         "inject_prep": (B * T * D * 2.0 * (5 + 3), "byte"),
-        # reads dq_rot, dk_bar, dv_bar (fp32) and k, v, R_k, R_v; writes dq, dk, dv, dR_k, dR_v
-        "unmix": (B * T * D * (3 * 4 + 4 * 2 + 5 * 2.0), "byte"),
+        # reads dq_rot (fp32), dk_bar, dv_bar, k, v, R_k, R_v (bf16); writes dq, dk, dv, dR_k, dR_v
+        "unmix": (B * T * D * (4 + 6 * 2 + 5 * 2.0), "byte"),
         # reads m, m', dm; writes dm (the layer step accumulates into dO)
         "consistency_loss": (B * T * D * 2.0 * 4, "byte"),
         # reads O, dO (bf16); zeroes the fp32 dQ accumulator

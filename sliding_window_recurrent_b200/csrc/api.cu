@@ -151,9 +151,10 @@ struct BwdLayout {
 BwdLayout bwd_layout(const maglev_swa_desc* d) {
   BwdLayout L;
   const size_t n = (size_t)d->B * d->T * d->H * d->hd;
+  const size_t elt = d->dtype == MAGLEV_BF16 ? 2 : 4;  // dk_bar, dv_bar in the activation type
   L.dkb = 0;
-  L.dvb = L.dkb + align256(n * 4);
-  L.delta = L.dvb + align256(n * 4);
+  L.dvb = L.dkb + align256(n * elt);
+  L.delta = L.dvb + align256(n * elt);
   L.gpart = L.delta + align256((size_t)d->B * d->H * d->T * 4);
   L.dq_acc = L.gpart + align256((size_t)d->B * d->T * 4 * d->H * 4);
   L.total = L.dq_acc + (d->dtype == MAGLEV_BF16 ? align256(n * 4) : 0);
@@ -478,8 +479,8 @@ maglev_status maglev_inject_swa_bwd(const maglev_swa_desc* d, const void* k, con
   const void* kb = at<char>(saved, L.k);
   const void* vb = at<char>(saved, L.v);
   float* delta = at<float>(workspace, Wk.delta);
-  float* dkb = at<float>(workspace, Wk.dkb);
-  float* dvb = at<float>(workspace, Wk.dvb);
+  void* dkb = at<char>(workspace, Wk.dkb);
+  void* dvb = at<char>(workspace, Wk.dvb);
   float* gpart = at<float>(workspace, Wk.gpart);
   float* dq_acc = d->dtype == MAGLEV_BF16 ? at<float>(workspace, Wk.dq_acc) : nullptr;
   MAGLEV_LAUNCH(1, s, launch_attn_delta(sh, out, dout, delta, dq_acc, s), "attn_delta");

@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(256) prep_vec_kernel(SwaShape s, RopeTable rt,
 
 template <typename T, int HD>
 __global__ void __launch_bounds__(256) unmix_vec_kernel(
-    SwaShape s, RopeTable rt, const float* __restrict__ dkb, const float* __restrict__ dvb,
+    SwaShape s, RopeTable rt, const T* __restrict__ dkb, const T* __restrict__ dvb,
     const T* __restrict__ k, const T* __restrict__ v, const T* __restrict__ Rk, const T* __restrict__ Rv,
     const float* __restrict__ gates, T* __restrict__ dk, T* __restrict__ dv, T* __restrict__ dRk,
     T* __restrict__ dRv, int accumulate, float* __restrict__ gpart, const float* __restrict__ dq_acc,
@@ -396,14 +396,14 @@ cudaError_t launch_prep(const SwaShape& s, const void* q, const void* k, const v
   return cudaGetLastError();
 }
 
-cudaError_t launch_unmix(const SwaShape& s, const float* dk_bar, const float* dv_bar, const void* k,
+cudaError_t launch_unmix(const SwaShape& s, const void* dk_bar, const void* dv_bar, const void* k,
                          const void* v, const void* Rk, const void* Rv, const float* gates, void* dk, void* dv,
                          void* dRk, void* dRv, int accumulate, float* gpart, const float* dq_acc, void* dq,
                          cudaStream_t st) {
   const RopeTable rt = rope_table(s);
   MAGLEV_EW_DISPATCH(s.dtype, s.hd,
                      unmix_vec_kernel<T, HD><<<blocks_for(s, HD / 16), 256, 0, st>>>(
-                         s, rt, dk_bar, dv_bar, (const T*)k, (const T*)v, (const T*)Rk, (const T*)Rv, gates,
+                         s, rt, (const T*)dk_bar, (const T*)dv_bar, (const T*)k, (const T*)v, (const T*)Rk, (const T*)Rv, gates,
                          (T*)dk, (T*)dv, (T*)dRk, (T*)dRv, accumulate, gpart, dq_acc, (T*)dq));
   return cudaGetLastError();
 }

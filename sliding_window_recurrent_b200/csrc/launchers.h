@@ -40,14 +40,14 @@ cudaError_t launch_attn_delta(const SwaShape& s, const void* out, const void* do
 cudaError_t launch_attn_bwd_dq_simt(const SwaShape& s, const void* q_rot, const void* k_bar,
                                     const void* v_bar, const void* dout, const float* lse,
                                     const float* delta, void* dq, cudaStream_t st);
-// dk_bar, dv_bar in fp32.
+// dk_bar, dv_bar in the activation type.
 cudaError_t launch_attn_bwd_dkdv_simt(const SwaShape& s, const void* q_rot, const void* k_bar,
                                       const void* v_bar, const void* dout, const float* lse,
-                                      const float* delta, float* dk_bar, float* dv_bar,
+                                      const float* delta, void* dk_bar, void* dv_bar,
                                       cudaStream_t st);
 // dk, dv, dR_k, dR_v (and dq from dq_acc when non-null) and per-row gate
-// partials gpart[(g*H + h) * B*T + row] from dk_bar, dv_bar.
-cudaError_t launch_unmix(const SwaShape& s, const float* dk_bar, const float* dv_bar,
+// partials gpart[(g*H + h) * B*T + row] from dk_bar, dv_bar (activation type).
+cudaError_t launch_unmix(const SwaShape& s, const void* dk_bar, const void* dv_bar,
                          const void* k, const void* v, const void* Rk, const void* Rv,
                          const float* gates, void* dk, void* dv, void* dRk, void* dRv,
                          int accumulate, float* gpart, const float* dq_acc, void* dq,
@@ -96,11 +96,12 @@ cudaError_t launch_proj_bwd_dw_tc(int64_t M, int D, int d, const void* dRk, cons
                                   int* err, cudaStream_t s);
 int num_sms();
 
-// tcgen05 banded attention backward: dk_bar, dv_bar (fp32) and the rotated-frame
-// dq accumulated with fp32 atomics into dq_acc (zeroed by the launcher).
+// tcgen05 banded attention backward: dk_bar, dv_bar (bf16, rounded from the
+// fp32 accumulators) and the rotated-frame dq reduce-added in fp32 into dq_acc
+// (zeroed beforehand).
 cudaError_t launch_attn_bwd_tc(const SwaShape& s, const void* q_rot, const void* k_bar, const void* v_bar,
                                const void* dout, const float* lse, const float* delta, float* dq_acc,
-                               float* dk_bar, float* dv_bar, int64_t spin_limit, int* err, cudaStream_t st);
+                               void* dk_bar, void* dv_bar, int64_t spin_limit, int* err, cudaStream_t st);
 
 // tcgen05 banded attention forward on the saved bf16 q_rot / k_bar / v_bar.
 cudaError_t launch_attn_fwd_tc(const SwaShape& s, const void* q_rot, const void* k_bar, const void* v_bar,

@@ -175,13 +175,13 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(
 
 // ---------------------------------------------------------------------------
 // a6 backward, dk_bar and dv_bar: warp per key row j, 8 keys per block sharing
-// 32-query tiles of [j0, j0+7+W-1]; fp32 results for the un-mix.
+// 32-query tiles of [j0, j0+7+W-1]; results in the activation type for the un-mix.
 // ---------------------------------------------------------------------------
 template <typename T, int HD>
 __global__ void __launch_bounds__(256) attn_bwd_dkdv_kernel(
     SwaShape s, const T* __restrict__ qr, const T* __restrict__ kb, const T* __restrict__ vb,
     const T* __restrict__ dout, const float* __restrict__ lse, const float* __restrict__ delta,
-    float* __restrict__ dkb, float* __restrict__ dvb, float scale) {
+    T* __restrict__ dkb, T* __restrict__ dvb, float scale) {
   constexpr int NC = HD / 32;
   __shared__ float Qs[32][HD + 1];
   __shared__ float Gs[32][HD + 1];
@@ -250,8 +250,8 @@ __global__ void __launch_bounds__(256) attn_bwd_dkdv_kernel(
   if (j < T_) {
 #pragma unroll
     for (int r = 0; r < NC; ++r) {
-      dkb[rowp(j) + lane + 32 * r] = ak[r] * scale;
-      dvb[rowp(j) + lane + 32 * r] = av[r];
+      dkb[rowp(j) + lane + 32 * r] = from_f<T>(ak[r] * scale);
+      dvb[rowp(j) + lane + 32 * r] = from_f<T>(av[r]);
     }
   }
 }
@@ -293,14 +293,14 @@ cudaError_t launch_attn_bwd_dq_simt(const SwaShape& s, const void* q_rot, const 
 
 cudaError_t launch_attn_bwd_dkdv_simt(const SwaShape& s, const void* q_rot, const void* k_bar,
                                       const void* v_bar, const void* dout, const float* lse,
-                                      const float* delta, float* dk_bar, float* dv_bar,
+                                      const float* delta, void* dk_bar, void* dv_bar,
                                       cudaStream_t st) {
   dim3 grid((unsigned)((s.T + 7) / 8), (unsigned)s.H, (unsigned)s.B);
   const float scale = 1.0f / sqrtf((float)s.hd);
   MAGLEV_DISPATCH(s.dtype, s.hd,
                   attn_bwd_dkdv_kernel<T, HD><<<grid, 256, 0, st>>>(
                       s, (const T*)q_rot, (const T*)k_bar, (const T*)v_bar, (const T*)dout, lse,
-                      delta, dk_bar, dv_bar, scale));
+                      delta, (T*)dk_bar, (T*)dv_bar, scale));
   return cudaGetLastError();
 }
 

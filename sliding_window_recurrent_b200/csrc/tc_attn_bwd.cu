@@ -69,8 +69,8 @@ struct BwdParams {
   const float* lse;    // [B,H,T] natural log
   const float* delta;  // [B,H,T]
   float* dq_acc;       // [B,T,H,hd] fp32, zeroed, rotated frame (written through tmDQ)
-  float* dk_bar;       // [B,T,H,hd] fp32
-  float* dv_bar;       // [B,T,H,hd] fp32
+  bf16* dk_bar;        // [B,T,H,hd] bf16 (rounded from the fp32 accumulators)
+  bf16* dv_bar;        // [B,T,H,hd] bf16
   int64_t spin_limit;
   int* err;
 };
@@ -340,23 +340,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll 1
       for (int c = half * (HD / 64); c < (half + 1) * (HD / 64); ++c) {
         uint32_t v[32];
-        tmem_ld32(tmem + lane_off + C::R_DK + 32u * (uint32_t)c, v);
-        tmem_wait_ld();
-        if (row_ok) {
 #pragma unroll
-          for (int g = 0; g < 8; ++g)
-            *reinterpret_cast<float4*>(p.dk_bar + row + 32 * c + 4 * g) =
-                make_float4(__uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1]),
-                            __uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3]));
-        }
-        tmem_ld32(tmem + lane_off + C::R_DV + 32u * (uint32_t)c, v);
-        tmem_wait_ld();
-        if (row_ok) {
+        for (int t = 0; t < 2; ++t) {  // dK, then dV
+          tmem_ld32(tmem + lane_off + (t == 0 ? C::R_DK : C::R_DV) + 32u * (uint32_t)c, v);
+          tmem_wait_ld();
+          bf16* dst = (t == 0 ? p.dk_bar : p.dv_bar) + row + 32 * c;
+          if (row_ok) {
 #pragma unroll
-          for (int g = 0; g < 8; ++g)
-            *reinterpret_cast<float4*>(p.dv_bar + row + 32 * c + 4 * g) =
-                make_float4(__uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1]),
-                            __uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3]));
+            for (int g = 0; g < 4; ++g)
+              *reinterpret_cast<uint4*>(dst + 8 * g) = make_uint4(
+                  pack_bf16(__uint_as_float(v[8 * g + 0]), __uint_as_float(v[8 * g + 1])),
+                  pack_bf16(__uint_as_float(v[8 * g + 2]), __uint_as_float(v[8 * g + 3])),
+                  pack_bf16(__uint_as_float(v[8 * g + 4]), __uint_as_float(v[8 * g + 5])),
+                  pack_bf16(__uint_as_float(v[8 * g + 6]), __uint_as_float(v[8 * g + 7])));
+          }
         }
       }
     }
@@ -747,17 +744,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         xp = x;
         jp = j;
       }
-      // epilogue of the unit: dK, dV rows (fp32). Each warp's 32 rows x 64
-      // columns go through its own 8 KiB of the P^T / dS^T buffers (free: the
-      // unit's MMAs are complete and the pending dQ reduce-adds have read their
-      // staging), so that every global store covers two whole 256-byte row pieces.
+      // epilogue of the unit: dK, dV rows, rounded to bf16. Each warp's 32 rows
+      // x 64 columns go through its own 4 KiB of the P^T / dS^T buffers (free:
+      // the unit's MMAs are complete and the pending dQ reduce-adds have read
+      // their staging), so that every global store covers four whole 128-byte
+      // row pieces.
       ok = ok && warp_wait(acc_full, (uint32_t)n & 1u, ab);
       if (lane == 0) bulk_wait_read_all();
       asm volatile("bar.sync 1, %0;" ::"n"(SOFT_THREADS) : "memory");  // reached by every softmax thread
       if (ok) {
         tc_fence_after();
-        uint8_t* stg = smem + C::OFF_P + (q4 + 4 * half) * 8192;  // [32 rows][64 fp32], 16-byte chunks swizzled
-        const int64_t tstride = (int64_t)p.H * HD;                // floats between consecutive tokens
+        uint8_t* stg = smem + C::OFF_P + (q4 + 4 * half) * 4096;  // [32 rows][64 bf16], 16-byte chunks swizzled
+        const int64_t tstride = (int64_t)p.H * HD;                // elements between consecutive tokens
         const int64_t col0 = (int64_t)x.h * HD + 64 * half;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {  // dK, then dV
@@ -771,19 +769,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_arrive(acc_empty);
           }
 #pragma unroll
-          for (int c4 = 0; c4 < 16; ++c4)
-            *reinterpret_cast<uint4*>(stg + lane * 256 + ((c4 ^ (lane & 15)) << 4)) =
-                make_uint4(v[c4 >> 3][4 * (c4 & 7)], v[c4 >> 3][4 * (c4 & 7) + 1], v[c4 >> 3][4 * (c4 & 7) + 2],
-                           v[c4 >> 3][4 * (c4 & 7) + 3]);
+          for (int c8 = 0; c8 < 8; ++c8) {
+            const uint32_t* a = &v[c8 >> 2][8 * (c8 & 3)];
+            *reinterpret_cast<uint4*>(stg + lane * 128 + ((c8 ^ (lane & 7)) << 4)) = make_uint4(
+                pack_bf16(__uint_as_float(a[0]), __uint_as_float(a[1])),
+                pack_bf16(__uint_as_float(a[2]), __uint_as_float(a[3])),
+                pack_bf16(__uint_as_float(a[4]), __uint_as_float(a[5])),
+                pack_bf16(__uint_as_float(a[6]), __uint_as_float(a[7])));
+          }
           __syncwarp();
-          float* dst = t == 0 ? p.dk_bar : p.dv_bar;
+          bf16* dst = t == 0 ? p.dk_bar : p.dv_bar;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int r = 2 * i + (lane >> 4), ch = lane & 15;
-            const uint4 w = *reinterpret_cast<const uint4*>(stg + r * 256 + ((ch ^ (r & 15)) << 4));
+          for (int i = 0; i < 8; ++i) {
+            const int r = 4 * i + (lane >> 3), ch = lane & 7;  // row of the warp's 32, 16-byte chunk
+            const uint4 w = *reinterpret_cast<const uint4*>(stg + r * 128 + ((ch ^ (r & 7)) << 4));
             const int key = x.kt + 32 * q4 + r;
             if (key < p.T)
-              *reinterpret_cast<uint4*>(dst + ((int64_t)x.b * p.T + key) * tstride + col0 + 4 * ch) = w;
+              *reinterpret_cast<uint4*>(dst + ((int64_t)x.b * p.T + key) * tstride + col0 + 8 * ch) = w;
           }
           __syncwarp();
         }
@@ -808,7 +810,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 cudaError_t launch_attn_bwd_tc(const SwaShape& s, const void* q_rot, const void* k_bar, const void* v_bar,
                                const void* dout, const float* lse, const float* delta, float* dq_acc,
-                               float* dk_bar, float* dv_bar, int64_t spin_limit, int* err, cudaStream_t st) {
+                               void* dk_bar, void* dv_bar, int64_t spin_limit, int* err, cudaStream_t st) {
   CUtensorMap tq, tk, tv, tdo;
   cudaError_t e;
   if ((e = make_tmap_tokens(&tq, q_rot, s.B, s.T, s.H, s.hd, 128)) != cudaSuccess) return e;
@@ -827,8 +829,8 @@ cudaError_t launch_attn_bwd_tc(const SwaShape& s, const void* q_rot, const void*
   p.lse = lse;
   p.delta = delta;
   p.dq_acc = dq_acc;
-  p.dk_bar = dk_bar;
-  p.dv_bar = dv_bar;
+  p.dk_bar = static_cast<bf16*>(dk_bar);
+  p.dv_bar = static_cast<bf16*>(dv_bar);
   p.spin_limit = spin_limit;
   p.err = err;
   dim3 grid((unsigned)((s.T + 127) / 128), (unsigned)s.H, (unsigned)s.B);
