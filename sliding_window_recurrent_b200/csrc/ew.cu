@@ -56,14 +56,38 @@ __device__ __forceinline__ void store8(float* p, const V8& v) {
   *reinterpret_cast<float4*>(p) = make_float4(v.x[0], v.x[1], v.x[2], v.x[3]);
   *reinterpret_cast<float4*>(p + 4) = make_float4(v.x[4], v.x[5], v.x[6], v.x[7]);
 }
+// A 16-byte (bf16) or 32-byte (fp32) load kept in its stored form until used,
+// so that a thread can put all its loads in flight before any arithmetic.
 template <typename T>
-__device__ __forceinline__ void store8_acc(T* p, V8 v, int accumulate) {
-  if (accumulate) {
-    const V8 o = load8(p);
+struct Raw8;
+template <>
+struct Raw8<bf16> {
+  uint4 u;
+};
+template <>
+struct Raw8<float> {
+  float4 a, b;
+};
+__device__ __forceinline__ Raw8<bf16> raw8(const bf16* p) { return {*reinterpret_cast<const uint4*>(p)}; }
+__device__ __forceinline__ Raw8<float> raw8(const float* p) {
+  return {*reinterpret_cast<const float4*>(p), *reinterpret_cast<const float4*>(p + 4)};
+}
+__device__ __forceinline__ V8 cvt8(const Raw8<bf16>& r) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r.u);
+  V8 x;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) v.x[e] += o.x[e];
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    x.x[2 * i] = f.x;
+    x.x[2 * i + 1] = f.y;
   }
-  store8(p, v);
+  return x;
+}
+__device__ __forceinline__ V8 cvt8(const Raw8<float>& r) {
+  V8 x;
+  x.x[0] = r.a.x; x.x[1] = r.a.y; x.x[2] = r.a.z; x.x[3] = r.a.w;
+  x.x[4] = r.b.x; x.x[5] = r.b.y; x.x[6] = r.b.z; x.x[7] = r.b.w;
+  return x;
 }
 
 // Sum over the TPR lanes that share a row (TPR a power of two <= 32, aligned).
@@ -171,7 +195,7 @@ __global__ void __launch_bounds__(256) prep_vec_kernel(SwaShape s, RopeTable rt,
 }
 
 template <typename T, int HD>
-__global__ void __launch_bounds__(256) unmix_vec_kernel(
+__global__ void __launch_bounds__(256, sizeof(T) == 2 ? 2 : 1) unmix_vec_kernel(
     SwaShape s, RopeTable rt, const T* __restrict__ dkb, const T* __restrict__ dvb,
     const T* __restrict__ k, const T* __restrict__ v, const T* __restrict__ Rk, const T* __restrict__ Rv,
     const float* __restrict__ gates, T* __restrict__ dk, T* __restrict__ dv, T* __restrict__ dRk,
@@ -189,10 +213,41 @@ __global__ void __launch_bounds__(256) unmix_vec_kernel(
   const int t = (int)(bt % s.T);
   const int64_t p = (int64_t)s.pos0 + t;
   const int64_t b1 = rr * HD + 8 * u, b2 = b1 + HALF;
+  // every load first; the RoPE angles are computed while they are in flight
+  Raw8<T> d1r{}, d2r{}, e1r{}, e2r{}, k1r{}, k2r{}, r1r{}, r2r{}, v1r{}, v2r{}, w1r{}, w2r{};
+  Raw8<T> pk1{}, pk2{}, pv1{}, pv2{};
+  Raw8<float> x1r{}, x2r{};
+  const bool with_dq = dq_acc != nullptr;
+  if (live) {
+    d1r = raw8(dkb + b1);
+    d2r = raw8(dkb + b2);
+    e1r = raw8(dvb + b1);
+    e2r = raw8(dvb + b2);
+    if (with_dq) {
+      x1r = raw8(dq_acc + b1);
+      x2r = raw8(dq_acc + b2);
+    }
+    if (s.inject) {
+      k1r = raw8(k + b1);
+      k2r = raw8(k + b2);
+      r1r = raw8(Rk + b1);
+      r2r = raw8(Rk + b2);
+      v1r = raw8(v + b1);
+      v2r = raw8(v + b2);
+      w1r = raw8(Rv + b1);
+      w2r = raw8(Rv + b2);
+      if (accumulate) {
+        pk1 = raw8(dRk + b1);
+        pk2 = raw8(dRk + b2);
+        pv1 = raw8(dRv + b1);
+        pv2 = raw8(dRv + b2);
+      }
+    }
+  }
   float cs[8], sn[8];
   rope8(p, rt.inv_freq, 8 * u, cs, sn);
-  if (live && dq_acc) {
-    const V8 x1 = load8(dq_acc + b1), x2 = load8(dq_acc + b2);
+  if (live && with_dq) {  // dq = RoPE^T(dq_rot)
+    const V8 x1 = cvt8(x1r), x2 = cvt8(x2r);
     V8 o1, o2;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -202,11 +257,7 @@ __global__ void __launch_bounds__(256) unmix_vec_kernel(
     store8(dq + b1, o1);
     store8(dq + b2, o2);
   }
-  V8 d1 = {}, d2 = {};
-  if (live) {
-    d1 = load8(dkb + b1);
-    d2 = load8(dkb + b2);
-  }
+  const V8 d1 = cvt8(d1r), d2 = cvt8(d2r);
   // RoPE^T of dk_bar
   V8 bk1, bk2;
 #pragma unroll
@@ -218,20 +269,14 @@ __global__ void __launch_bounds__(256) unmix_vec_kernel(
     if (live) {
       store8(dk + b1, bk1);
       store8(dk + b2, bk2);
-      store8(dv + b1, load8(dvb + b1));
-      store8(dv + b2, load8(dvb + b2));
+      store8(dv + b1, cvt8(e1r));
+      store8(dv + b2, cvt8(e2r));
     }
     return;
   }
   const float gkl = gate_value(gates[0 * s.H + h]), gkr = gate_value(gates[1 * s.H + h]);
   const float gvl = gate_value(gates[2 * s.H + h]), gvr = gate_value(gates[3 * s.H + h]);
-  V8 r1 = {}, r2 = {}, k1 = {}, k2 = {};
-  if (live) {
-    r1 = load8(Rk + b1);
-    r2 = load8(Rk + b2);
-    k1 = load8(k + b1);
-    k2 = load8(k + b2);
-  }
+  const V8 r1 = cvt8(r1r), r2 = cvt8(r2r), k1 = cvt8(k1r), k2 = cvt8(k2r);
   float ss = 0.f;
 #pragma unroll
   for (int e = 0; e < 8; ++e) ss += r1.x[e] * r1.x[e] + r2.x[e] * r2.x[e];
@@ -252,15 +297,7 @@ __global__ void __launch_bounds__(256) unmix_vec_kernel(
     s_ndn += n1.x[e] * dn1.x[e] + n2.x[e] * dn2.x[e];
   }
   const float mean_ndn = row_sum<TPR>(s_ndn) / HD;
-  V8 dv1 = {}, dv2 = {}, va = {}, vc = {}, ra = {}, rc = {};
-  if (live) {
-    dv1 = load8(dvb + b1);
-    dv2 = load8(dvb + b2);
-    va = load8(v + b1);
-    vc = load8(v + b2);
-    ra = load8(Rv + b1);
-    rc = load8(Rv + b2);
-  }
+  const V8 dv1 = cvt8(e1r), dv2 = cvt8(e2r), va = cvt8(v1r), vc = cvt8(v2r), ra = cvt8(w1r), rc = cvt8(w2r);
   float s_vl = 0.f, s_vr = 0.f;
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
@@ -280,13 +317,16 @@ __global__ void __launch_bounds__(256) unmix_vec_kernel(
   }
   store8(dk + b1, o1);
   store8(dk + b2, o2);
+  {
+    const V8 a1 = cvt8(pk1), a2 = cvt8(pk2);  // zero unless accumulating
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    o1.x[e] = (dn1.x[e] - n1.x[e] * mean_ndn) * rinv;
-    o2.x[e] = (dn2.x[e] - n2.x[e] * mean_ndn) * rinv;
+    for (int e = 0; e < 8; ++e) {
+      o1.x[e] = (dn1.x[e] - n1.x[e] * mean_ndn) * rinv + a1.x[e];
+      o2.x[e] = (dn2.x[e] - n2.x[e] * mean_ndn) * rinv + a2.x[e];
+    }
   }
-  store8_acc(dRk + b1, o1, accumulate);
-  store8_acc(dRk + b2, o2, accumulate);
+  store8(dRk + b1, o1);
+  store8(dRk + b2, o2);
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     o1.x[e] = gvl * dv1.x[e];
@@ -294,13 +334,16 @@ __global__ void __launch_bounds__(256) unmix_vec_kernel(
   }
   store8(dv + b1, o1);
   store8(dv + b2, o2);
+  {
+    const V8 a1 = cvt8(pv1), a2 = cvt8(pv2);
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    o1.x[e] = gvr * dv1.x[e];
-    o2.x[e] = gvr * dv2.x[e];
+    for (int e = 0; e < 8; ++e) {
+      o1.x[e] = gvr * dv1.x[e] + a1.x[e];
+      o2.x[e] = gvr * dv2.x[e] + a2.x[e];
+    }
   }
-  store8_acc(dRv + b1, o1, accumulate);
-  store8_acc(dRv + b2, o2, accumulate);
+  store8(dRv + b1, o1);
+  store8(dRv + b2, o2);
   if (u == 0) {  // column-contiguous partials: gpart[(g*H + h) * rows + bt]
     const int64_t rows = (int64_t)s.B * s.T;
     gpart[(0 * s.H + h) * rows + bt] = s_kl;
