@@ -42,11 +42,13 @@ struct TcGemmParams {
 
 template <int BN, bool A_MN, bool B_MN>
 struct Cfg {
+  static_assert(BN % 64 == 0 && BN <= 256, "N tiles are whole 64-column blocks");
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
   static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
+  static constexpr int ACC_STRIDE = TMEM_COLS / 2;  // column of the second accumulator
   static constexpr int OFF_EPI = STAGES * STAGE_BYTES + 256;  // 4 warps x [32 rows x 128 B] output staging
   static constexpr size_t SMEM = 1024 + (size_t)OFF_EPI + 4 * 4096;
 };
@@ -168,7 +170,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, ab)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * C::ACC_STRIDE);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&full[stage], phase, ab)) {
             ok = false;
@@ -230,8 +232,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 64) {
         uint32_t r[2][32];
-        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c0), r[0]);
-        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c0 + 32), r[1]);
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::ACC_STRIDE + c0), r[0]);
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::ACC_STRIDE + c0 + 32), r[1]);
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -442,10 +444,14 @@ cudaError_t launch_proj_bwd_dm_tc(int64_t M, int D, int d, const void* dRk, cons
 }
 
 // dW_mk | dW_mv [D, d] = dR^T [D, M] m_shift [M, d] (A and B both M-contiguous in memory).
+// 128 x 192 tiles: at D = d = 1280 that is 20 x 7 = 140 tiles, one per SM in a
+// single wave (128 x 256 would give 100 tiles and leave a third of the SMs idle);
+// N = 192 still keeps the shared-memory operand traffic of an MMA under the
+// per-cycle limit.
 cudaError_t launch_proj_bwd_dw_tc(int64_t M, int D, int d, const void* dRk, const void* dRv,
                                   const void* m_shift, void* dwk, void* dwv, int64_t spin_limit,
                                   int* err, cudaStream_t s) {
-  constexpr int BN = 256;
+  constexpr int BN = 192;
   CUtensorMap a0, a1, b;
   cudaError_t e;
   if ((e = make_tmap_bf16_2d(&a0, dRk, D, M, (uint64_t)D * 2, 64, 64)) != cudaSuccess) return e;
