@@ -43,8 +43,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ignored once that source changes.
 NCU_TRAFFIC: dict[str, dict] = {
     # ncu --set full on the timed step's launches (profiles/ncu_attn_layer_bf16.md)
-    "attn_bwd_tc": {"bytes": 204036864, "src": "tc_attn_bwd.cu", "src_sha": "ee73a005eb511859"},
-    "attn_fwd_tc": {"bytes": 68504064, "src": "tc_attn_fwd.cu", "src_sha": "599bc5b79289372c"},
+    "attn_bwd_tc": {"bytes": 162984960, "src": "tc_attn_bwd.cu", "src_sha": "fe20220f81eacb39"},
+    "attn_fwd_tc": {"bytes": 68273920, "src": "tc_attn_fwd.cu", "src_sha": "e2b9ee99ddfc1ff6"},
     # one launch of the 64 x 10 x 512 x 128 ring step (profiles/ncu_decode_step.md)
     "decode_step": {"bytes": 172343552, "src": "decode.cu", "src_sha": "ab1ab99dee605d36"},
 }
