@@ -159,195 +159,6 @@ __global__ void __launch_bounds__(256) decode_step_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Ring attention for bf16 rings, one thread-block cluster of NS CTAs per (b,h).
-// CTA `rank` owns slots [rank*C, rank*C + C), C <= 128; warp w owns 32 of
-// them. Two bulk copies bring the chunk's K and V rows into shared memory
-// (64 KiB per CTA in flight from the first cycle, three CTAs per SM); lanes
-// form partial dot products over 16-byte pieces of a row, reduced over the
-// row's lanes, then the same for V with the chunk softmax weights. Rank 0
-// merges the NS partial (max, sum, o) triples through distributed shared
-// memory. The CTA whose chunk holds slot p mod W writes the new entry to the
-// ring once its copies have landed and uses it in place of the stale slot.
-// ---------------------------------------------------------------------------
-constexpr int RING_ROWS = 128;  // slots per CTA at most
-constexpr int RING_THREADS = 128;
-constexpr int RING_WARPS = RING_THREADS / 32;
-constexpr int ROWS_PER_WARP = RING_ROWS / RING_WARPS;
-
-template <int HD>
-__global__ void __launch_bounds__(RING_THREADS) decode_ring_bulk_kernel(
-    DecShape s, int ns, int chunk, const int64_t* __restrict__ pos, const bf16* __restrict__ q,
-    const bf16* __restrict__ k, const bf16* __restrict__ v, const bf16* __restrict__ krec,
-    const bf16* __restrict__ vrec, const float* __restrict__ gates, bf16* __restrict__ kring,
-    bf16* __restrict__ vring, bf16* __restrict__ out, float scale, int64_t limit_ns, int* err) {
-  namespace cg = cooperative_groups;
-  constexpr int HALF = HD / 2;
-  constexpr int LPR = HD / 8;     // lanes per row (16 B each)
-  constexpr int RPW = 32 / LPR;   // rows per warp step
-  constexpr int STEPS = ROWS_PER_WARP / RPW;
-  extern __shared__ __align__(128) uint8_t dsm[];
-  bf16* ks = reinterpret_cast<bf16*>(dsm);                         // [RING_ROWS][HD]
-  bf16* vs = reinterpret_cast<bf16*>(dsm + RING_ROWS * HD * 2);    // [RING_ROWS][HD]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(dsm + 2 * RING_ROWS * HD * 2);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 1);
-  __shared__ float qs[HD], kn[HD], vn[HD];
-  __shared__ float sc[RING_ROWS];
-  __shared__ float part_o[RING_WARPS][HD];
-  __shared__ float stat[2];  // chunk max, chunk sum
-  cg::cluster_group cluster = cg::this_cluster();
-  const int rank = (int)cluster.block_rank();
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int bh = blockIdx.x / ns, b = bh / s.H, h = bh % s.H;
-  const int W = s.W;
-  const int64_t p = pos[b];
-  const int64_t tok = (int64_t)bh * HD;
-  const int64_t ring = (int64_t)bh * W * HD;
-  const int r0 = rank * chunk;
-  const int rows = max(0, min(W, r0 + chunk) - r0);
-  const bool valid_pos = p >= 0;
-  const int slot = valid_pos ? (int)(p % W) : -1;
-  const int nlive = !valid_pos ? 0 : (p >= W - 1 ? W : (int)p + 1);
-  const int live_rows = max(0, min(rows, nlive - r0));
-  const int sub = lane / LPR, cl = (lane % LPR) * 8;
-  const tc::Abort ab{abort_flag, err, limit_ns};
-
-  if (tid == 0) {
-    tc::mbar_init(bar, 1);
-    *abort_flag = 0;
-    tc::fence_mbar_init();
-    if (live_rows > 0) {
-      const uint32_t bytes = (uint32_t)live_rows * HD * 2;
-      tc::mbar_arrive_expect_tx(bar, 2 * bytes);
-      tc::bulk_load(ks, kring + ring + (int64_t)r0 * HD, bytes, bar);
-      tc::bulk_load(vs, vring + ring + (int64_t)r0 * HD, bytes, bar);
-    }
-  }
-  if (tid < HALF && valid_pos) {
-    const int c = tid;
-    float cs, sn;
-    rope_cos_sin(p, c, HD, s.log2_base, &cs, &sn);
-    const float q1 = to_f(q[tok + c]), q2 = to_f(q[tok + c + HALF]);
-    qs[c] = q1 * cs - q2 * sn;
-    qs[c + HALF] = q1 * sn + q2 * cs;
-    const float k1 = to_f(k[tok + c]), k2 = to_f(k[tok + c + HALF]);
-    float a1 = k1 * cs - k2 * sn, a2 = k1 * sn + k2 * cs;
-    float v1 = to_f(v[tok + c]), v2 = to_f(v[tok + c + HALF]);
-    if (s.inject) {
-      const float gkl = gate_value(gates[0 * s.H + h]), gkr = gate_value(gates[1 * s.H + h]);
-      const float gvl = gate_value(gates[2 * s.H + h]), gvr = gate_value(gates[3 * s.H + h]);
-      a1 = gkl * a1 + gkr * to_f(krec[tok + c]);
-      a2 = gkl * a2 + gkr * to_f(krec[tok + c + HALF]);
-      v1 = gvl * v1 + gvr * to_f(vrec[tok + c]);
-      v2 = gvl * v2 + gvr * to_f(vrec[tok + c + HALF]);
-    }
-    kn[c] = to_f(from_f<bf16>(a1));  // the step attends to exactly what it stores
-    kn[c + HALF] = to_f(from_f<bf16>(a2));
-    vn[c] = to_f(from_f<bf16>(v1));
-    vn[c + HALF] = to_f(from_f<bf16>(v2));
-  }
-  __syncthreads();  // barrier initialised, new entry formed
-  // the chunk has landed (or the wait gave up: scores of a failed chunk are not used)
-  const bool landed = live_rows == 0 || tc::mbar_wait(bar, 0, ab);
-  const int use_rows = landed ? live_rows : 0;
-  const bool owner = valid_pos && slot >= r0 && slot < r0 + rows;
-  if (owner && tid < HD) {  // the copy of this slot has completed: overwrite it in the ring
-    kring[ring + (int64_t)slot * HD + tid] = from_f<bf16>(kn[tid]);
-    vring[ring + (int64_t)slot * HD + tid] = from_f<bf16>(vn[tid]);
-  }
-  float qv[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) qv[e] = qs[cl + e];
-#pragma unroll
-  for (int i = 0; i < STEPS; ++i) {
-    const int r = warp * ROWS_PER_WARP + i * RPW + sub;
-    float d = 0.f;
-    if (r0 + r == slot) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) d = fmaf(qv[e], kn[cl + e], d);
-    } else if (r < use_rows) {
-      const uint4 u = *reinterpret_cast<const uint4*>(ks + r * HD + cl);
-      const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(hv[e]);
-        d = fmaf(qv[2 * e], f.x, d);
-        d = fmaf(qv[2 * e + 1], f.y, d);
-      }
-    }
-#pragma unroll
-    for (int o = LPR / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-    if ((lane % LPR) == 0) sc[r] = r < use_rows ? d * scale : -INFINITY;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    float mx = -INFINITY;
-    for (int r = lane; r < RING_ROWS; r += 32) mx = fmaxf(mx, sc[r]);
-    mx = warp_max(mx);
-    float l = 0.f;
-    for (int r = lane; r < RING_ROWS; r += 32) {
-      const float e = mx == -INFINITY ? 0.f : expf(sc[r] - mx);
-      sc[r] = e;
-      l += e;
-    }
-    l = warp_sum(l);
-    if (lane == 0) {
-      stat[0] = mx;
-      stat[1] = l;
-    }
-  }
-  __syncthreads();
-  float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int i = 0; i < STEPS; ++i) {
-    const int r = warp * ROWS_PER_WARP + i * RPW + sub;
-    if (r0 + r == slot) {
-      const float pr = sc[r];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) o[e] = fmaf(pr, vn[cl + e], o[e]);
-    } else if (r < use_rows) {
-      const float pr = sc[r];
-      const uint4 u = *reinterpret_cast<const uint4*>(vs + r * HD + cl);
-      const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(hv[e]);
-        o[2 * e] = fmaf(pr, f.x, o[2 * e]);
-        o[2 * e + 1] = fmaf(pr, f.y, o[2 * e + 1]);
-      }
-    }
-  }
-#pragma unroll
-  for (int e = 0; e < 8; ++e)
-#pragma unroll
-    for (int off = 16; off >= LPR; off >>= 1) o[e] += __shfl_xor_sync(0xffffffffu, o[e], off);
-  if (lane < LPR) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) part_o[warp][cl + e] = o[e];
-  }
-  __syncthreads();
-  if (tid < HD) {
-    float acc = 0.f;
-#pragma unroll
-    for (int w = 0; w < RING_WARPS; ++w) acc += part_o[w][tid];
-    part_o[0][tid] = acc;
-  }
-  cluster.sync();
-  if (rank == 0 && tid < HD) {
-    float M = -INFINITY;
-    for (int r = 0; r < ns; ++r) M = fmaxf(M, cluster.map_shared_rank(stat, r)[0]);
-    float L = 0.f, O = 0.f;
-    for (int r = 0; r < ns; ++r) {
-      const float mr = cluster.map_shared_rank(stat, r)[0];
-      const float w = mr == -INFINITY ? 0.f : expf(mr - M);
-      L += w * cluster.map_shared_rank(stat, r)[1];
-      O += w * cluster.map_shared_rank(&part_o[0][0], r)[tid];
-    }
-    out[tok + tid] = from_f<bf16>(valid_pos && L > 0.f ? O / L : 0.f);
-  }
-  cluster.sync();  // remote reads done before any CTA of the cluster exits
-}
-
-// ---------------------------------------------------------------------------
 // Streaming ring attention for bf16 rings: persistent, one CTA per SM walks
 // (b,h) pairs with a stride of the grid and reads each window once. A
 // producer warp streams 128-slot chunks of K and V through a ring of
@@ -355,9 +166,11 @@ __global__ void __launch_bounds__(RING_THREADS) decode_ring_bulk_kernel(
 // 64 channels x 128 slots, alternating K_c, V_c), running on into the next
 // pair while the current one finishes; sixteen compute warps each own 8 rows
 // of every chunk and keep an online softmax (running max, sum and output,
-// log2 units) over their rows, merged at the end of the pair. The new entry
-// is formed at the start of the pair, used in place of slot p mod W, and
-// written to the ring after the pair's copies have landed.
+// log2 units) over their rows, merged at the end of the pair. A prep warp
+// forms each pair's rotated q and new entry one pair ahead, into a double
+// buffer, so the compute warps never wait on that arithmetic; the new entry
+// is used in place of slot p mod W and written to the ring after the pair's
+// copies have landed.
 // ---------------------------------------------------------------------------
 // RoPE frequencies base^(-2c/hd), computed once on the host (double).
 struct RopeFreq {
@@ -366,7 +179,7 @@ struct RopeFreq {
 
 constexpr int ST_ROWS = 128;          // slots per chunk
 constexpr int ST_WARPS = 16;          // compute warps
-constexpr int ST_THREADS = 32 * (ST_WARPS + 1);
+constexpr int ST_THREADS = 32 * (ST_WARPS + 2);  // + producer warp + prep warp
 
 template <int HD>
 struct StreamCfg {
@@ -396,7 +209,10 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
   uint64_t* full = reinterpret_cast<uint64_t*>(dsm + C::OFF_BAR);   // [NSTAGE]
   uint64_t* empty = full + C::NSTAGE;                                 // [NSTAGE]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + C::NSTAGE);
-  __shared__ float qs[HD], kn[HD], vn[HD];
+  uint64_t* prep_full = empty + C::NSTAGE + 1;  // [2]
+  uint64_t* prep_empty = prep_full + 2;         // [2]
+  __shared__ float qs[2][HD], kn[2][HD], vn[2][HD];  // per pair, double-buffered
+  __shared__ long long ppos[2];
   __shared__ float wm[ST_WARPS], wl[ST_WARPS];
   __shared__ float wo[ST_WARPS][HD];
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -413,6 +229,10 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
     for (int i = 0; i < C::NSTAGE; ++i) {
       tc::mbar_init(&full[i], 1);
       tc::mbar_init(&empty[i], ST_WARPS);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&prep_full[i], 32);
+      tc::mbar_init(&prep_empty[i], 1);
     }
     *abort_flag = 0;
     tc::fence_mbar_init();
@@ -453,50 +273,72 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
     }
     return;  // takes no part in the compute warps' barriers
   }
+  if (warp == ST_WARPS + 1) {
+    // ------------------------------------------------------------ prep
+    // pair i's position, q rotated and scaled to log2 units, and its new K/V
+    // entry (RoPE of the local key, gated mix), into buffer i&1 once the
+    // compute warps are done with pair i-2
+    int i = 0;
+    for (int bh = blockIdx.x; bh < npairs; bh += gridDim.x, ++i) {
+      const int buf = i & 1;
+      if (i >= 2 && !tc::warp_wait(&prep_empty[buf], (uint32_t)((i - 2) >> 1) & 1u, ab)) break;
+      const int h = bh % s.H;
+      const int64_t p = pos[bh / s.H];
+      const int64_t tok = (int64_t)bh * HD;
+      if (p >= 0) {
+        for (int c = lane; c < HALF; c += 32) {
+          // angle p * theta_c reduced to [-pi, pi] in double before the float sincos
+          double ang = (double)p * rf.inv_freq[c];
+          ang -= 6.283185307179586476925286766559 * rint(ang * 0.15915494309189533577);
+          float cs, sn;
+          sincosf((float)ang, &sn, &cs);
+          const float q1 = to_f(q[tok + c]), q2 = to_f(q[tok + c + HALF]);
+          qs[buf][c] = (q1 * cs - q2 * sn) * scale_log2;  // scores come out in log2 units
+          qs[buf][c + HALF] = (q1 * sn + q2 * cs) * scale_log2;
+          const float k1 = to_f(k[tok + c]), k2 = to_f(k[tok + c + HALF]);
+          float a1 = k1 * cs - k2 * sn, a2 = k1 * sn + k2 * cs;
+          float v1 = to_f(v[tok + c]), v2 = to_f(v[tok + c + HALF]);
+          if (s.inject) {
+            const float gkl = gate_value(gates[0 * s.H + h]), gkr = gate_value(gates[1 * s.H + h]);
+            const float gvl = gate_value(gates[2 * s.H + h]), gvr = gate_value(gates[3 * s.H + h]);
+            a1 = gkl * a1 + gkr * to_f(krec[tok + c]);
+            a2 = gkl * a2 + gkr * to_f(krec[tok + c + HALF]);
+            v1 = gvl * v1 + gvr * to_f(vrec[tok + c]);
+            v2 = gvl * v2 + gvr * to_f(vrec[tok + c + HALF]);
+          }
+          kn[buf][c] = to_f(from_f<bf16>(a1));  // the step attends to exactly what it stores
+          kn[buf][c + HALF] = to_f(from_f<bf16>(a2));
+          vn[buf][c] = to_f(from_f<bf16>(v1));
+          vn[buf][c + HALF] = to_f(from_f<bf16>(v2));
+        }
+      }
+      if (lane == 0) ppos[buf] = p;
+      tc::mbar_arrive(&prep_full[buf]);  // each lane releases its own writes
+    }
+    return;  // takes no part in the compute warps' barriers
+  }
   // ------------------------------------------------------------ compute warps
   const int sub = lane / LPR, cl = (lane % LPR) * 8;
   const int boff = (cl / 64) * C::BOX_BYTES + (cl % 64) * 2;  // byte offset of this lane's piece in a row
   int L = 0;
   bool ok = true;
-  for (int bh = blockIdx.x; bh < npairs; bh += gridDim.x) {
-    const int b = bh / s.H, h = bh % s.H;
-    const int64_t p = pos[b];
+  int i = 0;
+  for (int bh = blockIdx.x; bh < npairs; bh += gridDim.x, ++i) {
+    const int buf = i & 1;
+    // the pair's q and new entry are ready (after an abort the pair is skipped)
+    ok = ok && tc::mbar_wait(&prep_full[buf], (uint32_t)(i >> 1) & 1u, ab);
+    const int64_t p = ok ? (int64_t)ppos[buf] : -1;
     const int64_t tok = (int64_t)bh * HD;
     const int64_t ring = (int64_t)bh * W * HD;
     const bool valid_pos = p >= 0;
     const int slot = valid_pos ? (int)(p % W) : -1;
-    const int nlive = live_of(bh);
-    const int nchunks = (nlive + ST_ROWS - 1) / ST_ROWS;
-    if (tid < HALF && valid_pos) {
-      const int c = tid;
-      // angle p * theta_c reduced to [-pi, pi] in double before the float sincos
-      double ang = (double)p * rf.inv_freq[c];
-      ang -= 6.283185307179586476925286766559 * rint(ang * 0.15915494309189533577);
-      float cs, sn;
-      sincosf((float)ang, &sn, &cs);
-      const float q1 = to_f(q[tok + c]), q2 = to_f(q[tok + c + HALF]);
-      qs[c] = (q1 * cs - q2 * sn) * scale_log2;  // scores come out in log2 units
-      qs[c + HALF] = (q1 * sn + q2 * cs) * scale_log2;
-      const float k1 = to_f(k[tok + c]), k2 = to_f(k[tok + c + HALF]);
-      float a1 = k1 * cs - k2 * sn, a2 = k1 * sn + k2 * cs;
-      float v1 = to_f(v[tok + c]), v2 = to_f(v[tok + c + HALF]);
-      if (s.inject) {
-        const float gkl = gate_value(gates[0 * s.H + h]), gkr = gate_value(gates[1 * s.H + h]);
-        const float gvl = gate_value(gates[2 * s.H + h]), gvr = gate_value(gates[3 * s.H + h]);
-        a1 = gkl * a1 + gkr * to_f(krec[tok + c]);
-        a2 = gkl * a2 + gkr * to_f(krec[tok + c + HALF]);
-        v1 = gvl * v1 + gvr * to_f(vrec[tok + c]);
-        v2 = gvl * v2 + gvr * to_f(vrec[tok + c + HALF]);
-      }
-      kn[c] = to_f(from_f<bf16>(a1));  // the step attends to exactly what it stores
-      kn[c + HALF] = to_f(from_f<bf16>(a2));
-      vn[c] = to_f(from_f<bf16>(v1));
-      vn[c + HALF] = to_f(from_f<bf16>(v2));
-    }
-    asm volatile("bar.sync 1, %0;" ::"n"(CT) : "memory");  // the pair's q and new entry are ready
+    const int nlive = valid_pos ? (p >= W - 1 ? W : (int)p + 1) : 0;
+    const int nchunks = (nlive + ST_ROWS - 1) / ST_ROWS;  // as the producer counts them
+    const float* kn_b = kn[buf];
+    const float* vn_b = vn[buf];
     float qv[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) qv[e] = qs[cl + e];
+    for (int e = 0; e < 8; ++e) qv[e] = qs[buf][cl + e];
     float m = -INFINITY, l = 0.f;  // log2 units, over the rows this lane-group has seen
     float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int c = 0; c < nchunks; ++c, L += 2) {
@@ -517,8 +359,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
         if (gr == slot) {
 #pragma unroll
           for (int e = 0; e < 8; e += 2) {
-            d0 = fmaf(qv[e], kn[cl + e], d0);
-            d1 = fmaf(qv[e + 1], kn[cl + e + 1], d1);
+            d0 = fmaf(qv[e], kn_b[cl + e], d0);
+            d1 = fmaf(qv[e + 1], kn_b[cl + e + 1], d1);
           }
         } else {
           const uint4 u = *reinterpret_cast<const uint4*>(kc + r * 128);
@@ -564,7 +406,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
         const int gr = c * ST_ROWS + r;
         if (gr == slot) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) o[e] = fmaf(pr[i], vn[cl + e], o[e]);
+          for (int e = 0; e < 8; ++e) o[e] = fmaf(pr[i], vn_b[cl + e], o[e]);
         } else if (gr < nlive) {  // dead slots may hold anything, NaN included
           const uint4 u = *reinterpret_cast<const uint4*>(vc + r * 128);
           const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&u);
@@ -615,11 +457,12 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
       }
       out[tok + tid] = from_f<bf16>(valid_pos && Ls > 0.f ? O / Ls : 0.f);
       if (valid_pos && ok) {
-        kring[ring + (int64_t)slot * HD + tid] = from_f<bf16>(kn[tid]);
-        vring[ring + (int64_t)slot * HD + tid] = from_f<bf16>(vn[tid]);
+        kring[ring + (int64_t)slot * HD + tid] = from_f<bf16>(kn_b[tid]);
+        vring[ring + (int64_t)slot * HD + tid] = from_f<bf16>(vn_b[tid]);
       }
     }
     asm volatile("bar.sync 1, %0;" ::"n"(CT) : "memory");  // q, new entry, partials free again
+    if (tid == 0) tc::mbar_arrive(&prep_empty[buf]);           // the prep warp may refill buffer buf
   }
 }
 
@@ -682,38 +525,6 @@ cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void
                                                               scale_log2, limit_ns, err, rf);
     }
     return cudaGetLastError();
-  }
-  if (false) {
-    const int ns = (s.W + RING_ROWS - 1) / RING_ROWS;
-    const int chunk = (s.W + ns - 1) / ns;
-    const size_t dyn = 2 * (size_t)RING_ROWS * s.hd * 2 + 64;  // K and V chunk, barrier, abort flag
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(s.B * s.H * ns));
-    cfg.blockDim = dim3(RING_THREADS);
-    cfg.dynamicSmemBytes = dyn;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)ns;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const int64_t limit_ns = (limit_us > 0 ? limit_us : DEFAULT_SPIN_LIMIT) * 1000;
-    if (s.hd == 128) {
-      cudaError_t e = cudaFuncSetAttribute(decode_ring_bulk_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)dyn);
-      if (e != cudaSuccess) return e;
-      return cudaLaunchKernelEx(&cfg, decode_ring_bulk_kernel<128>, s, ns, chunk, pos, (const bf16*)q,
-                                (const bf16*)k, (const bf16*)v, (const bf16*)krec, (const bf16*)vrec, gates,
-                                (bf16*)k_ring, (bf16*)v_ring, (bf16*)out, scale, limit_ns, err);
-    }
-    cudaError_t e = cudaFuncSetAttribute(decode_ring_bulk_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)dyn);
-    if (e != cudaSuccess) return e;
-    return cudaLaunchKernelEx(&cfg, decode_ring_bulk_kernel<64>, s, ns, chunk, pos, (const bf16*)q, (const bf16*)k,
-                              (const bf16*)v, (const bf16*)krec, (const bf16*)vrec, gates, (bf16*)k_ring,
-                              (bf16*)v_ring, (bf16*)out, scale, limit_ns, err);
   }
   const size_t smem = (size_t)s.W * sizeof(float);
   MAGLEV_DISPATCH2(s.dtype, s.hd, {
