@@ -279,6 +279,42 @@ def test_decode_full_shape():
     assert_close(host(S.krec), krec, "bf16", "krec_rot")
 
 
+def test_decode_full_shape_mixed_positions():
+    """640 (sequence, head) pairs, so each persistent CTA walks several pairs in a
+    row, with positions that change from pair to pair: negative (no write, zero
+    output), partial rings (p < W-1), p = W-1, wrapped rings. Every slot of both
+    rings is checked: the new entry against the oracle, all others bit-exact."""
+    B, H, hd, d, W = 64, 10, 128, 1280, 512
+    cycle = [-1, 0, 1, 37, 255, 510, 511, 512, 1000, 4607, -5, 2047, 300]
+    pos = [cycle[b % len(cycle)] for b in range(B)]
+    x = synth.decode_inputs(23, B, H, hd, d, W, pos, dtype="bf16")
+    S = DecodeLayerState(B, H, hd, d, W, dtype="bf16")
+    pos_t = torch.from_numpy(x["pos"]).cuda()
+    kr, vr = dev(x["k_ring"]), dev(x["v_ring"])
+    S.mem_project(pos_t, dev(x["m_prev"]), dev(x["w_mk"]), dev(x["w_mv"]))
+    S.step(pos_t, dev(x["q"]), dev(x["k"]), dev(x["v"]), dev(x["gates"]), kr, vr)
+    torch.cuda.synchronize()
+    kr, vr, out = host(kr), host(vr), host(S.out)
+    ok = [b for b in range(B) if pos[b] >= 0]
+    bad = [b for b in range(B) if pos[b] < 0]
+    sub = lambda t: t.f64[ok]
+    krec, vrec = oracle.decode_mem_project(x["pos"][ok], sub(x["m_prev"]), x["w_mk"].f64, x["w_mv"].f64, H)
+    o_ref, kr2, vr2 = oracle.decode_step(x["pos"][ok], sub(x["q"]), sub(x["k"]), sub(x["v"]), krec, vrec,
+                                         x["gates"].astype(np.float64), sub(x["k_ring"]), sub(x["v_ring"]))
+    assert_close(out[ok], o_ref, "bf16", "out")
+    assert np.all(out[bad] == 0), "a negative position writes zeros to out"
+    for b in bad:  # ring untouched
+        np.testing.assert_array_equal(kr[b], x["k_ring"].f64[b])
+        np.testing.assert_array_equal(vr[b], x["v_ring"].f64[b])
+    for i, b in enumerate(ok):
+        s_ = pos[b] % W
+        keep = [j for j in range(W) if j != s_]
+        np.testing.assert_array_equal(kr[b][:, keep], x["k_ring"].f64[b][:, keep])
+        np.testing.assert_array_equal(vr[b][:, keep], x["v_ring"].f64[b][:, keep])
+        assert normwise(kr[b][:, s_], kr2[i][:, s_]) <= TOL["bf16"], (b, pos[b])
+        assert normwise(vr[b][:, s_], vr2[i][:, s_]) <= TOL["bf16"], (b, pos[b])
+
+
 def test_decode_matches_training_row():
     """Ring filled with the forward's mixed entries: decode at p equals forward row p."""
     wl = wl_of("layer_bf16", B=1, T=700, H=2, hd=128, d=128, W=512, dtype="f32")
