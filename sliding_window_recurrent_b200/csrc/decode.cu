@@ -172,6 +172,24 @@ __global__ void __launch_bounds__(256) decode_step_kernel(
 // is used in place of slot p mod W and written to the ring after the pair's
 // copies have landed.
 // ---------------------------------------------------------------------------
+// x[c0 .. c0+N) and x[c0+half .. c0+half+N) of one bf16 row, as floats
+// (one 4-byte load per half when N == 2).
+template <int N>
+__device__ __forceinline__ void load_pairs(const bf16* x, int c0, int half, float* a, float* b) {
+  if constexpr (N == 2) {
+    const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(x + c0));
+    const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(x + c0 + half));
+    a[0] = fa.x; a[1] = fa.y;
+    b[0] = fb.x; b[1] = fb.y;
+  } else {
+#pragma unroll
+    for (int e = 0; e < N; ++e) {
+      a[e] = to_f(x[c0 + e]);
+      b[e] = to_f(x[c0 + half + e]);
+    }
+  }
+}
+
 // RoPE frequencies base^(-2c/hd), computed once on the host (double).
 struct RopeFreq {
   double inv_freq[64];
@@ -283,28 +301,44 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
       const int buf = i & 1;
       if (i >= 2 && !tc::warp_wait(&prep_empty[buf], (uint32_t)((i - 2) >> 1) & 1u, ab)) break;
       const int h = bh % s.H;
-      const int64_t p = pos[bh / s.H];
       const int64_t tok = (int64_t)bh * HD;
+      // every load of the pair at once (none depends on p): at kernel start they
+      // queue behind the ring fill of every SM, so one round trip, not three
+      constexpr int NPL = HALF / 32;  // channel pairs per lane (2 or 1), contiguous
+      const int c0 = lane * NPL;
+      float qa[NPL], qb[NPL], ka[NPL], kb[NPL], va[NPL], vb[NPL], ra[NPL], rb[NPL], wa[NPL], wb[NPL];
+      load_pairs<NPL>(q + tok, c0, HALF, qa, qb);
+      load_pairs<NPL>(k + tok, c0, HALF, ka, kb);
+      load_pairs<NPL>(v + tok, c0, HALF, va, vb);
+      float ga = 0.f, gb = 0.f, gc = 0.f, gd = 0.f;
+      if (s.inject) {  // the memory inputs and gates may be NULL without injection
+        load_pairs<NPL>(krec + tok, c0, HALF, ra, rb);
+        load_pairs<NPL>(vrec + tok, c0, HALF, wa, wb);
+        ga = gates[0 * s.H + h];
+        gb = gates[1 * s.H + h];
+        gc = gates[2 * s.H + h];
+        gd = gates[3 * s.H + h];
+      }
+      const int64_t p = pos[bh / s.H];
       if (p >= 0) {
-        for (int c = lane; c < HALF; c += 32) {
+        const float gkl = gate_value(ga), gkr = gate_value(gb), gvl = gate_value(gc), gvr = gate_value(gd);
+#pragma unroll
+        for (int e = 0; e < NPL; ++e) {
+          const int c = c0 + e;
           // angle p * theta_c reduced to [-pi, pi] in double before the float sincos
           double ang = (double)p * rf.inv_freq[c];
           ang -= 6.283185307179586476925286766559 * rint(ang * 0.15915494309189533577);
           float cs, sn;
           sincosf((float)ang, &sn, &cs);
-          const float q1 = to_f(q[tok + c]), q2 = to_f(q[tok + c + HALF]);
-          qs[buf][c] = (q1 * cs - q2 * sn) * scale_log2;  // scores come out in log2 units
-          qs[buf][c + HALF] = (q1 * sn + q2 * cs) * scale_log2;
-          const float k1 = to_f(k[tok + c]), k2 = to_f(k[tok + c + HALF]);
-          float a1 = k1 * cs - k2 * sn, a2 = k1 * sn + k2 * cs;
-          float v1 = to_f(v[tok + c]), v2 = to_f(v[tok + c + HALF]);
+          qs[buf][c] = (qa[e] * cs - qb[e] * sn) * scale_log2;  // scores come out in log2 units
+          qs[buf][c + HALF] = (qa[e] * sn + qb[e] * cs) * scale_log2;
+          float a1 = ka[e] * cs - kb[e] * sn, a2 = ka[e] * sn + kb[e] * cs;
+          float v1 = va[e], v2 = vb[e];
           if (s.inject) {
-            const float gkl = gate_value(gates[0 * s.H + h]), gkr = gate_value(gates[1 * s.H + h]);
-            const float gvl = gate_value(gates[2 * s.H + h]), gvr = gate_value(gates[3 * s.H + h]);
-            a1 = gkl * a1 + gkr * to_f(krec[tok + c]);
-            a2 = gkl * a2 + gkr * to_f(krec[tok + c + HALF]);
-            v1 = gvl * v1 + gvr * to_f(vrec[tok + c]);
-            v2 = gvl * v2 + gvr * to_f(vrec[tok + c + HALF]);
+            a1 = gkl * a1 + gkr * ra[e];
+            a2 = gkl * a2 + gkr * rb[e];
+            v1 = gvl * v1 + gvr * wa[e];
+            v2 = gvl * v2 + gvr * wb[e];
           }
           kn[buf][c] = to_f(from_f<bf16>(a1));  // the step attends to exactly what it stores
           kn[buf][c + HALF] = to_f(from_f<bf16>(a2));
