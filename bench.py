@@ -43,7 +43,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ignored once that source changes.
 NCU_TRAFFIC: dict[str, dict] = {
     # ncu --set full on the timed step's launches (profiles/ncu_attn_layer_bf16.md)
-    "attn_bwd_tc": {"bytes": 162984960, "src": "tc_attn_bwd.cu", "src_sha": "fe20220f81eacb39"},
+    "attn_bwd_tc": {"bytes": 162984960, "src": "tc_attn_bwd.cu", "src_sha": "ff592e916e291f26"},
     "attn_fwd_tc": {"bytes": 68273920, "src": "tc_attn_fwd.cu", "src_sha": "e2b9ee99ddfc1ff6"},
     # one launch of the 64 x 10 x 512 x 128 ring step (profiles/ncu_decode_step.md)
     "decode_step": {"bytes": 172034048, "src": "decode.cu", "src_sha": "3d9fef6b5a1a20e3"},

@@ -2,8 +2,9 @@
 // rule of the forward in tc_attn_fwd.cu ("Maglev: Sliding Recurrent Memory",
 // paper.rainbus.top, 方法步骤详情; window of W keys, self included).
 //
-// One CTA per (128-key tile, head, batch row), looping over the 128-query
-// tiles that see those keys (at most 5 for W = 512):
+// Head dim 64: one CTA per (128-key tile, head, batch row), looping over the
+// 128-query tiles that see those keys (at most 5 for W = 512); head dim 128
+// uses the persistent pipelined kernel further down.
 //   S^T  = K Q^T,  dP^T = V dO^T                    (TMEM, fp32)
 //   P^T  = exp(S^T * scale - LSE),  dS^T = P^T (dP^T - Delta) * scale
 //   dV  += P^T dO,  dK += dS^T Q                    (TMEM accumulators)
@@ -18,7 +19,8 @@
 //              half of the dQ drain: TMEM -> registers (R_S released at
 //              once) -> the warp's own 4 KiB slices of the P^T / dS^T
 //              buffers (free once the dQ MMA completed) -> one TMA
-//              reduce-add per 32x32 fp32 block; finally dK, dV rows in fp32.
+//              reduce-add per 32x32 fp32 block; finally dK, dV rows, rounded
+//              to bf16.
 //              Half-tiles inside every row's window skip the band mask.
 //              LSE and Delta of each query tile are staged in shared memory.
 // Delta = rowsum(dO * O) comes from the delta kernel. Every wait is bounded.
