@@ -568,6 +568,16 @@ def cpu_baseline(budget_s=12.0):
             "sample": f"oracle fwd+loss+bwd of batch row 0, head 0 (T=2048, W=512, d=1280): {fl/1e9:.3f} GFLOP x {n} runs in {el:.1f} s"}
 
 
+def layer_config(world: int) -> dict:
+    """`config` of the headline line, the same for both arms."""
+    c = LAYER
+    return {"workload": "d20 injected-SWA layer fwd+consistency loss+bwd: B=4 T=2048 d=1280 H=10x128 "
+                        "W=512 lambda=0.1, bf16 storage, fp32 accumulation",
+            "global_batch": c["B"] * world, "seq_len": c["T"], "parallelism": f"replicas x{world} (no collective)",
+            "l2": "no flush: each step touches ~0.4 GB > 126 MB L2",
+            "gflop_per_step": round(layer_flops(c["B"], c["T"], c["H"], c["hd"], c["d"], c["W"])["total"] / 1e9, 3)}
+
+
 def reference_arm(args, rank):
     if rank != 0:
         return
@@ -585,10 +595,10 @@ def reference_arm(args, rank):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "d20 injected-SWA layer fwd+loss+bwd, bounded sample: batch row 0, head 0, "
-                                   "T=2048, W=512, d=1280 (the CPU fp64 oracle)", "seq_len": c["T"]},
+            "config": layer_config(args.gpus),
             "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
-                             "sample": f"{fl/1e9:.3f} GFLOP per step (one batch row, one head)"},
+                             "sample": f"the CPU fp64 oracle's fwd+loss+bwd of batch row 0, head 0 of that "
+                                       f"workload (T=2048, W=512, d=1280): {fl/1e9:.3f} GFLOP per step"},
             "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -670,17 +680,12 @@ def main():
         dist.destroy_process_group()
     if rank != 0:
         return
-    c = LAYER
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r["ms"], 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: seeded N(0,1) inputs of the d20 shapes (stand-in for FineWeb-Edu activations)",
-        "config": {"workload": "d20 injected-SWA layer fwd+consistency loss+bwd: B=4 T=2048 d=1280 H=10x128 "
-                               "W=512 lambda=0.1, bf16 storage, fp32 accumulation",
-                   "global_batch": c["B"] * world, "seq_len": c["T"], "parallelism": f"replicas x{world} (no collective)",
-                   "l2": "no flush: each step touches ~0.4 GB > 126 MB L2",
-                   "gflop_per_step": round(r["flops"]["total"] / 1e9, 3)},
+        "config": layer_config(world),
         "frac_of_bf16_peak": round(value / world / peaks["bf16_tflops"], 5),
         "roofline": r["roofline"],
         "kernels": r["kernels"],
