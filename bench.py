@@ -38,16 +38,26 @@ DECODE = dict(B=64, L=20, H=10, hd=128, d=1280, W=512, first_pos=512)
 STACK = dict(B=8, T=2048, H=10, hd=128, L=20, W=512, lam=0.1)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes (read + write) per launch from ncu captures, keyed by trace name;
-# each entry records the sha256 of the kernel source it was taken on, and is
-# ignored once that source changes.
+# Datasheet dense peaks of one B200 (context beside the measured peaks).
+SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+
+# DRAM bytes (read + write) per launch, as stored from an ncu capture of the
+# kernel at the benchmark's shape (dram__bytes_read.sum + dram__bytes_write.sum);
+# each entry records the sha256 of the kernel source it was taken on and is
+# ignored (traffic null) once that source changes. The bench line marks these
+# figures "traffic_source": "stored ncu capture", since they are not measured
+# during the run.
 NCU_TRAFFIC: dict[str, dict] = {
-    # ncu --set full on the timed step's launches (profiles/ncu_attn_layer_bf16.md)
     "attn_bwd_tc": {"bytes": 162984960, "src": "tc_attn_bwd.cu", "src_sha": "ff592e916e291f26"},
     "attn_fwd_tc": {"bytes": 68273920, "src": "tc_attn_fwd.cu", "src_sha": "e2b9ee99ddfc1ff6"},
-    # one launch of the 64 x 10 x 512 x 128 ring step (profiles/ncu_decode_step.md)
     "decode_step": {"bytes": 172034048, "src": "decode.cu", "src_sha": "3d9fef6b5a1a20e3"},
 }
+
+
+def stored_traffic(name: str):
+    """The stored ncu DRAM bytes of `name` if taken on its current source, else None."""
+    tr = NCU_TRAFFIC.get(name)
+    return tr["bytes"] if tr and tr.get("src_sha") == src_sha(tr.get("src", "")) else None
 
 
 # --------------------------------------------------------------------------- work model
@@ -308,9 +318,12 @@ def run_layer_bench(torch, dist, rank, world, dev, steps, warmup, peaks, peaks_s
             peak = peaks["hbm_gbs"]
             roof = {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                     "unit": "GB/s", "frac": round(achieved / peak, 5)}
-        tr = NCU_TRAFFIC.get(name)
-        roof["traffic"] = tr["bytes"] if tr and tr.get("src_sha") == src_sha(tr.get("src", "")) else None
+        roof["traffic"] = stored_traffic(name)
+        roof["traffic_source"] = "stored ncu capture of this kernel's current source" if roof["traffic"] else None
         roof["peak_source"] = f"{peaks_src} burst (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback"
+        key = "bf16_tflops" if unit == "flop" else "hbm_gbs"
+        roof["spec_peak"] = SPEC_PEAKS[key]
+        roof["frac_of_spec"] = round(roof["achieved"] / SPEC_PEAKS[key], 5)
         roof["avg_launch_ms"] = round(avg_ms, 5)
         roof["work_per_launch"] = work
     kernels = {n: {"calls": v[0], "ms_total": round(v[1], 4), "share": round(v[1] / sum(w[1] for w in prof.values()), 4)}
@@ -502,14 +515,16 @@ def run_decode_bench(torch, dev, steps, warmup, peaks):
         calls, tot, _ = prof["decode_step"]
         avg = tot / calls
         gbs = ring_bytes / (avg * 1e-3) / 1e9
-        tr = NCU_TRAFFIC.get("decode_step")
+        traffic = stored_traffic("decode_step")
         roof = {"kernel": "decode_step", "bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4), "avg_launch_ms": round(avg, 5),
-                "bytes_per_launch": ring_bytes,
-                "traffic": tr["bytes"] if tr and tr.get("src_sha") == src_sha(tr.get("src", "")) else None}
+                "bytes_per_launch": ring_bytes, "traffic": traffic,
+                "traffic_source": "stored ncu capture of this kernel's current source" if traffic else None,
+                "spec_peak": SPEC_PEAKS["hbm_gbs"], "frac_of_spec": round(gbs / SPEC_PEAKS["hbm_gbs"], 4)}
     return {"tokens_per_s": B * 1000.0 / ms, "ms_per_step": ms, "roofline": roof,
             "kernels": {n: {"calls": v[0], "ms_total": round(v[1], 4)} for n, v in prof.items()},
-            "workload": f"decode B={B} L={L} H={H}x{hd} d={d} ring W={W}, pos from {c['first_pos']}, CUDA graph"}
+            "workload": f"decode B={B} L={L} H={H}x{hd} d={d} ring W={W}, {steps} token steps from pos "
+                        f"{c['first_pos']} (after {warmup + 3} warm-up steps), CUDA graph"}
 
 
 # --------------------------------------------------------------------------- oracle arm
@@ -610,7 +625,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--decode-steps", type=int, default=64)
+    ap.add_argument("--decode-steps", type=int, default=4096)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--stack-steps", type=int, default=5)
     ap.add_argument("--no-stack", action="store_true")
@@ -687,6 +702,7 @@ def main():
         "data": "synthetic: seeded N(0,1) inputs of the d20 shapes (stand-in for FineWeb-Edu activations)",
         "config": layer_config(world),
         "frac_of_bf16_peak": round(value / world / peaks["bf16_tflops"], 5),
+        "frac_of_spec_bf16_peak": round(value / world / SPEC_PEAKS["bf16_tflops"], 5),
         "roofline": r["roofline"],
         "kernels": r["kernels"],
         "cpu_baseline": cpu,

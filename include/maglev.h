@@ -137,25 +137,45 @@ maglev_status maglev_inject_swa_fwd(const maglev_swa_desc* desc, const void* q, 
                                     const float* gate_logits, void* out, float* lse, void* saved,
                                     void* stream);
 
+/* How maglev_inject_swa_bwd stores dL/dR of the shared projection. The layers
+ * of a decoder share W^rec ([rainbus] 方法步骤详情: one projection for all
+ * layers), so its gradient is the sum of every layer's dL/dR. The sum is kept
+ * in fp32 running sums (dR_acc_k, dR_acc_v) and rounded to the activation type
+ * once, by the last layer of the backward sweep:
+ *   MAGLEV_DR_WRITE  dR (dtype) = this layer's dL/dR (a single layer)
+ *   MAGLEV_DR_FIRST  dR_acc (fp32) = this layer's dL/dR (first layer of a sweep)
+ *   MAGLEV_DR_ADD    dR_acc (fp32) += this layer's dL/dR
+ *   MAGLEV_DR_LAST   dR (dtype) = dR_acc + this layer's dL/dR (last layer) */
+typedef enum {
+  MAGLEV_DR_WRITE = 0,
+  MAGLEV_DR_FIRST = 1,
+  MAGLEV_DR_ADD = 2,
+  MAGLEV_DR_LAST = 3
+} maglev_dr_mode;
+
 /* a6 -- backward of maglev_inject_swa_fwd (chain rule of the forward above).
  *   Inputs: the forward's k, v, R_k, R_v, gate_logits, out, lse, saved, and
  *   dout [B,T,H,hd] = dL/dout.
  *   dq, dk, dv [B,T,H,hd] (out, overwritten).
- *   dR_k, dR_v [B,T,D] (out): dL/dR; overwritten, or added to when
- *     accumulate_dR != 0 (summing the shared projection's gradient over layers).
- *     May be NULL when inject == 0.
+ *   dR_k, dR_v [B,T,D] of dtype (out): written in modes WRITE and LAST; may be
+ *     NULL in modes FIRST and ADD, and when inject == 0.
+ *   dR_acc_k, dR_acc_v [B,T,D] fp32: the running sums, written (FIRST), updated
+ *     (ADD) or read (LAST); unused (may be NULL) in mode WRITE.
+ *   dR_mode: a maglev_dr_mode value.
  *   dgate_logits [4,H] fp32 (out, overwritten); NULL when inject == 0.
  *   m_shift, w_mk, w_mv, dm_shift, dw_mk, dw_mv: if m_shift != NULL the call
- *     finishes with maglev_mem_project_bwd on the (accumulated) dR_k, dR_v.
- *   workspace: maglev_swa_bwd_workspace_bytes(desc) bytes of scratch. */
+ *     finishes with maglev_mem_project_bwd on dR_k, dR_v (modes WRITE and LAST).
+ *   workspace: maglev_swa_bwd_workspace_bytes(desc) bytes of scratch.
+ * Errors: INVALID_ARG for a bad dR_mode, for m_shift != NULL in modes FIRST or
+ * ADD, and for a NULL pointer the mode needs. */
 maglev_status maglev_inject_swa_bwd(const maglev_swa_desc* desc, const void* k, const void* v,
                                     const void* R_k, const void* R_v, const float* gate_logits,
                                     const void* out, const float* lse, const void* saved,
                                     const void* dout, void* dq, void* dk, void* dv, void* dR_k,
-                                    void* dR_v, int accumulate_dR, float* dgate_logits,
-                                    const void* m_shift, const void* w_mk, const void* w_mv,
-                                    void* dm_shift, void* dw_mk, void* dw_mv, void* workspace,
-                                    void* stream);
+                                    void* dR_v, float* dR_acc_k, float* dR_acc_v, int dR_mode,
+                                    float* dgate_logits, const void* m_shift, const void* w_mk,
+                                    const void* w_mv, void* dm_shift, void* dw_mk, void* dw_mv,
+                                    void* workspace, void* stream);
 
 /* a6 -- backward of the shared memory projection.
  *   dm_shift [B,T,d_mem] = dR_k W_mk + dR_v W_mv (overwritten);
@@ -216,7 +236,10 @@ maglev_status maglev_consistency_loss(const void* m, const void* m_target, int64
  * Limit: rows * d <= 67,108,864 elements; larger inputs return
  * MAGLEV_ERR_UNSUPPORTED with a message. The first call on each device looks
  * up the array's device address (cudaGetSymbolAddress) with that device
- * current: make that first call before any stream capture. All calls share
+ * current: make that first call before any stream capture (a first call
+ * inside a capture returns MAGLEV_ERR_CUDA). Every later call whose stream is
+ * not being captured looks the address up again, so a device reset (which
+ * reloads the library's device code) leaves no stale address. All calls share
  * the array and each call overwrites the partials it reads, so nothing needs
  * clearing, but calls that overlap on the GPU race and must be serialised.
  * The call allocates no memory. */

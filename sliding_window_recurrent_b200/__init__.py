@@ -19,6 +19,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "maglev.h")
 
 MAGLEV_OK, MAGLEV_ERR_INVALID_ARG, MAGLEV_ERR_UNSUPPORTED, MAGLEV_ERR_CUDA, MAGLEV_ERR_TIMEOUT = range(5)
 MAGLEV_F32, MAGLEV_BF16 = 0, 1
+MAGLEV_DR_WRITE, MAGLEV_DR_FIRST, MAGLEV_DR_ADD, MAGLEV_DR_LAST = range(4)
 
 
 class MaglevError(RuntimeError):
@@ -64,7 +65,7 @@ _SIGS = {
     "maglev_consistency_workspace_bytes": ([_I64, _I], _SZ),
     "maglev_mem_project": ([ctypes.POINTER(SwaDesc)] + [_P] * 6, _I),
     "maglev_inject_swa_fwd": ([ctypes.POINTER(SwaDesc)] + [_P] * 13, _I),
-    "maglev_inject_swa_bwd": ([ctypes.POINTER(SwaDesc)] + [_P] * 14 + [_I] + [_P] * 9, _I),
+    "maglev_inject_swa_bwd": ([ctypes.POINTER(SwaDesc)] + [_P] * 16 + [_I] + [_P] * 9, _I),
     "maglev_mem_project_bwd": ([ctypes.POINTER(SwaDesc)] + [_P] * 9, _I),
     "maglev_consistency_loss": ([_P, _P, _I64, _I, _I, _F, _F, _P, _P, _P, _I, _P, _P], _I),
     "maglev_consistency_loss_noalloc": ([_P, _P, _I64, _I, _I, _F, _F, _P, _P, _P, _I, _P], _I),
@@ -184,13 +185,13 @@ def maglev_inject_swa_fwd(desc, q, k, v, m_shift, w_mk, w_mv, R_k, R_v, gate_log
 
 
 def maglev_inject_swa_bwd(desc, k, v, R_k, R_v, gate_logits, out, lse, saved, dout, dq, dk, dv,
-                          dR_k, dR_v, accumulate_dR, dgate_logits, m_shift, w_mk, w_mv, dm_shift,
-                          dw_mk, dw_mv, workspace, stream=None):
+                          dR_k, dR_v, dR_acc_k, dR_acc_v, dR_mode, dgate_logits, m_shift, w_mk, w_mv,
+                          dm_shift, dw_mk, dw_mv, workspace, stream=None):
     _check(_lib.maglev_inject_swa_bwd(
         ctypes.byref(desc), _ptr(k), _ptr(v), _ptr(R_k), _ptr(R_v), _ptr(gate_logits), _ptr(out),
         _ptr(lse), _ptr(saved), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dR_k), _ptr(dR_v),
-        int(accumulate_dR), _ptr(dgate_logits), _ptr(m_shift), _ptr(w_mk), _ptr(w_mv),
-        _ptr(dm_shift), _ptr(dw_mk), _ptr(dw_mv), _ptr(workspace), _stream(stream)))
+        _ptr(dR_acc_k), _ptr(dR_acc_v), int(dR_mode), _ptr(dgate_logits), _ptr(m_shift), _ptr(w_mk),
+        _ptr(w_mv), _ptr(dm_shift), _ptr(dw_mk), _ptr(dw_mv), _ptr(workspace), _stream(stream)))
 
 
 def maglev_mem_project_bwd(desc, m_shift, w_mk, w_mv, dR_k, dR_v, dm_shift, dw_mk, dw_mv, stream=None):

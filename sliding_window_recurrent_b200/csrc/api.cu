@@ -170,7 +170,7 @@ const P* at(const void* base, size_t off) {
   return reinterpret_cast<const P*>(static_cast<const char*>(base) + off);
 }
 
-maglev_status status_word(int** out);
+maglev_status status_word(int** out, cudaStream_t s);
 
 int64_t spin_limit_of(int64_t v) { return v > 0 ? v : DEFAULT_SPIN_LIMIT; }
 
@@ -179,7 +179,7 @@ maglev_status run_mem_project(const maglev_swa_desc* d, const void* m, const voi
   const int64_t M = (int64_t)d->B * d->T, D = (int64_t)d->H * d->hd, K = d->d_mem;
   if (d->dtype == MAGLEV_BF16 && K % 8 == 0 && D % 256 == 0) {
     int* err = nullptr;
-    maglev_status s = status_word(&err);
+    maglev_status s = status_word(&err, st);
     if (s != MAGLEV_OK) return s;
     MAGLEV_LAUNCH(1, st, launch_proj_fwd_tc(M, (int)D, (int)K, m, wk, wv, Rk, Rv,
                                             spin_limit_of(d->spin_limit), err, st),
@@ -213,7 +213,7 @@ maglev_status run_mem_project_bwd(const maglev_swa_desc* d, const void* m, const
                                   void* dwk, void* dwv, cudaStream_t st) {
   const int64_t M = (int64_t)d->B * d->T, D = (int64_t)d->H * d->hd, K = d->d_mem;
   int* err = nullptr;
-  maglev_status stw = status_word(&err);
+  maglev_status stw = status_word(&err, st);
   if (stw != MAGLEV_OK) return stw;
   const bool tc = d->dtype == MAGLEV_BF16 && K % 8 == 0;
   if (dm && tc && D % 64 == 0) {
@@ -281,12 +281,20 @@ __device__ int g_device_status_word;
 std::mutex g_status_mu;
 int* g_status_ptr[128];
 
-maglev_status status_word(int** out) {
+// Device address of the status word on the current device: looked up on the
+// first call and again on every call whose stream is not being captured (a
+// device reset reloads the module, possibly at another address); calls made
+// during stream capture use the address cached by an earlier call.
+maglev_status status_word(int** out, cudaStream_t s) {
   int dev = 0;
   MAGLEV_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
   if (dev < 0 || dev >= 128) return fail(MAGLEV_ERR_UNSUPPORTED, "device index %d", dev);
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  const bool capturing = cudaStreamIsCapturing(s, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone;
   std::lock_guard<std::mutex> lock(g_status_mu);
-  if (!g_status_ptr[dev]) {
+  if (!capturing || !g_status_ptr[dev]) {
+    if (capturing)
+      return fail(MAGLEV_ERR_CUDA, "the first call of this library on a device must come before any stream capture");
     void* p = nullptr;
     MAGLEV_CUDA(cudaGetSymbolAddress(&p, g_device_status_word), "cudaGetSymbolAddress");
     g_status_ptr[dev] = static_cast<int*>(p);
@@ -344,9 +352,9 @@ size_t maglev_last_error(char* buf, size_t n) {
 maglev_status maglev_device_status(void* stream, int* code) {
   if (!code) return fail(MAGLEV_ERR_INVALID_ARG, "code must not be NULL");
   int* w = nullptr;
-  maglev_status st = status_word(&w);
-  if (st != MAGLEV_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  maglev_status st = status_word(&w, s);
+  if (st != MAGLEV_OK) return st;
   int host = 0;
   MAGLEV_CUDA(cudaMemcpyAsync(&host, w, sizeof(int), cudaMemcpyDeviceToHost, s), "read status");
   MAGLEV_CUDA(cudaMemsetAsync(w, 0, sizeof(int), s), "clear status");
@@ -420,7 +428,7 @@ maglev_status maglev_inject_swa_fwd(const maglev_swa_desc* d, const void* q, con
                 "inject_prep");
   if (d->dtype == MAGLEV_BF16) {
     int* err = nullptr;
-    st = status_word(&err);
+    st = status_word(&err, s);
     if (st != MAGLEV_OK) return st;
     MAGLEV_LAUNCH(1, s, launch_attn_fwd_tc(sh, at<char>(saved, L.q), at<char>(saved, L.k),
                                             at<char>(saved, L.v), out, lse, spin_limit_of(d->spin_limit),
@@ -438,10 +446,10 @@ maglev_status maglev_inject_swa_bwd(const maglev_swa_desc* d, const void* k, con
                                     const void* R_k, const void* R_v, const float* gate_logits,
                                     const void* out, const float* lse, const void* saved,
                                     const void* dout, void* dq, void* dk, void* dv, void* dR_k,
-                                    void* dR_v, int accumulate_dR, float* dgate_logits,
-                                    const void* m_shift, const void* w_mk, const void* w_mv,
-                                    void* dm_shift, void* dw_mk, void* dw_mv, void* workspace,
-                                    void* stream) {
+                                    void* dR_v, float* dR_acc_k, float* dR_acc_v, int dR_mode,
+                                    float* dgate_logits, const void* m_shift, const void* w_mk,
+                                    const void* w_mv, void* dm_shift, void* dw_mk, void* dw_mv,
+                                    void* workspace, void* stream) {
   maglev_status st = check_swa(d);
   if (st != MAGLEV_OK) return st;
   NEED_PTR(k);
@@ -454,13 +462,27 @@ maglev_status maglev_inject_swa_bwd(const maglev_swa_desc* d, const void* k, con
   NEED_PTR(dk);
   NEED_PTR(dv);
   NEED_PTR(workspace);
+  if (dR_mode < MAGLEV_DR_WRITE || dR_mode > MAGLEV_DR_LAST)
+    return fail(MAGLEV_ERR_INVALID_ARG, "dR_mode %d is not a maglev_dr_mode", dR_mode);
+  if (!d->inject) dR_mode = MAGLEV_DR_WRITE;
+  const bool dr_out = dR_mode == MAGLEV_DR_WRITE || dR_mode == MAGLEV_DR_LAST;
   if (d->inject) {
     NEED_PTR(R_k);
     NEED_PTR(R_v);
     NEED_PTR(gate_logits);
-    NEED_PTR(dR_k);
-    NEED_PTR(dR_v);
     NEED_PTR(dgate_logits);
+    if (dr_out) {
+      NEED_PTR(dR_k);
+      NEED_PTR(dR_v);
+    }
+    if (dR_mode != MAGLEV_DR_WRITE) {
+      NEED_PTR(dR_acc_k);
+      NEED_PTR(dR_acc_v);
+    }
+    if (m_shift && !dr_out)
+      return fail(MAGLEV_ERR_INVALID_ARG,
+                  "m_shift given in dR_mode %d: the projection backward needs the finished dR (WRITE or LAST)",
+                  dR_mode);
     if (m_shift) {
       NEED_PTR(m_shift);
       NEED_PTR(w_mk);
@@ -486,7 +508,7 @@ maglev_status maglev_inject_swa_bwd(const maglev_swa_desc* d, const void* k, con
   MAGLEV_LAUNCH(1, s, launch_attn_delta(sh, out, dout, delta, dq_acc, s), "attn_delta");
   if (d->dtype == MAGLEV_BF16) {
     int* err = nullptr;
-    st = status_word(&err);
+    st = status_word(&err, s);
     if (st != MAGLEV_OK) return st;
     MAGLEV_LAUNCH(1, s, launch_attn_bwd_tc(sh, qr, kb, vb, dout, lse, delta, dq_acc, dkb, dvb,
                                            spin_limit_of(d->spin_limit), err, s),
@@ -497,7 +519,7 @@ maglev_status maglev_inject_swa_bwd(const maglev_swa_desc* d, const void* k, con
                   "attn_bwd_dkdv");
   }
   MAGLEV_LAUNCH(1, s, launch_unmix(sh, dkb, dvb, k, v, R_k, R_v, gate_logits, dk, dv, dR_k, dR_v,
-                                   accumulate_dR ? 1 : 0, gpart, dq_acc, dq, s),
+                                   dR_acc_k, dR_acc_v, dR_mode, gpart, dq_acc, dq, s),
                 "unmix");
   if (d->inject) {
     MAGLEV_LAUNCH(1, s, launch_gate_reduce((int64_t)d->B * d->T, d->H, gpart, gate_logits, dgate_logits, s),
@@ -641,7 +663,7 @@ maglev_status maglev_decode_mem_project(const maglev_decode_desc* d, const int64
   const int64_t D = (int64_t)d->H * d->hd, K = d->d_mem;
   if (d->dtype == MAGLEV_BF16 && K % 8 == 0 && D % 256 == 0) {
     int* err = nullptr;
-    st = status_word(&err);
+    st = status_word(&err, s);
     if (st != MAGLEV_OK) return st;
     MAGLEV_LAUNCH(1, s, launch_proj_fwd_tc(d->B, (int)D, (int)K, m_prev, w_mk, w_mv, krec_rot, vrec,
                                            spin_limit_of(d->spin_limit), err, s),
@@ -691,7 +713,7 @@ maglev_status maglev_decode_step(const maglev_decode_desc* d, const int64_t* pos
   if (d->B == 0) return MAGLEV_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* err = nullptr;
-  st = status_word(&err);
+  st = status_word(&err, s);
   if (st != MAGLEV_OK) return st;
   MAGLEV_LAUNCH(1, s, launch_decode_step(dec_shape(d), pos, q, k, v, krec_rot, vrec, gate_logits, k_ring,
                                           v_ring, out, spin_limit_of(d->spin_limit), err, s),

@@ -3,7 +3,9 @@
 //          v_bar = g_vl v + g_vr R_v                       (forward, a2-a4)
 //   unmix  dq = RoPE^T(dq_rot); dk = g_kl RoPE^T(dk_bar);
 //          dR_k = RMSNorm'(R_k, RoPE^T(g_kr dk_bar)); dv = g_vl dv_bar;
-//          dR_v = g_vr dv_bar; per-row partial sums of the four gate gradients
+//          dR_v = g_vr dv_bar; per-row partial sums of the four gate gradients.
+//          dR is written in the activation type, or summed over the layers
+//          that share W^rec in fp32 running sums (rounded once, by the last)
 //   delta  Delta_i = dout_i . out_i (and zeroes the dq accumulator)
 //   gate   dgate[g,h] = sum over rows of the partials * dg/da
 // Source: "Maglev: Sliding Recurrent Memory", paper.rainbus.top, 方法步骤详情
@@ -199,8 +201,8 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 2 : 1) unmix_vec_kernel(
     SwaShape s, RopeTable rt, const T* __restrict__ dkb, const T* __restrict__ dvb,
     const T* __restrict__ k, const T* __restrict__ v, const T* __restrict__ Rk, const T* __restrict__ Rv,
     const float* __restrict__ gates, T* __restrict__ dk, T* __restrict__ dv, T* __restrict__ dRk,
-    T* __restrict__ dRv, int accumulate, float* __restrict__ gpart, const float* __restrict__ dq_acc,
-    T* __restrict__ dq) {
+    T* __restrict__ dRv, float* __restrict__ accRk, float* __restrict__ accRv, int dr_mode,
+    float* __restrict__ gpart, const float* __restrict__ dq_acc, T* __restrict__ dq) {
   constexpr int HALF = HD / 2, TPR = HD / 16;
   const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t row = gid / TPR;
@@ -215,8 +217,9 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 2 : 1) unmix_vec_kernel(
   const int64_t b1 = rr * HD + 8 * u, b2 = b1 + HALF;
   // every load first; the RoPE angles are computed while they are in flight
   Raw8<T> d1r{}, d2r{}, e1r{}, e2r{}, k1r{}, k2r{}, r1r{}, r2r{}, v1r{}, v2r{}, w1r{}, w2r{};
-  Raw8<T> pk1{}, pk2{}, pv1{}, pv2{};
+  Raw8<float> pk1{}, pk2{}, pv1{}, pv2{};  // fp32 running sums of dR over earlier layers
   Raw8<float> x1r{}, x2r{};
+  const bool read_acc = dr_mode == DR_ADD || dr_mode == DR_LAST;
   const bool with_dq = dq_acc != nullptr;
   if (live) {
     d1r = raw8(dkb + b1);
@@ -236,11 +239,11 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 2 : 1) unmix_vec_kernel(
       v2r = raw8(v + b2);
       w1r = raw8(Rv + b1);
       w2r = raw8(Rv + b2);
-      if (accumulate) {
-        pk1 = raw8(dRk + b1);
-        pk2 = raw8(dRk + b2);
-        pv1 = raw8(dRv + b1);
-        pv2 = raw8(dRv + b2);
+      if (read_acc) {
+        pk1 = raw8(accRk + b1);
+        pk2 = raw8(accRk + b2);
+        pv1 = raw8(accRv + b1);
+        pv2 = raw8(accRv + b2);
       }
     }
   }
@@ -317,16 +320,22 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 2 : 1) unmix_vec_kernel(
   }
   store8(dk + b1, o1);
   store8(dk + b2, o2);
+  const bool to_acc = dr_mode == DR_FIRST || dr_mode == DR_ADD;
   {
-    const V8 a1 = cvt8(pk1), a2 = cvt8(pk2);  // zero unless accumulating
+    const V8 a1 = cvt8(pk1), a2 = cvt8(pk2);  // zero unless a running sum is read
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       o1.x[e] = (dn1.x[e] - n1.x[e] * mean_ndn) * rinv + a1.x[e];
       o2.x[e] = (dn2.x[e] - n2.x[e] * mean_ndn) * rinv + a2.x[e];
     }
   }
-  store8(dRk + b1, o1);
-  store8(dRk + b2, o2);
+  if (to_acc) {
+    store8(accRk + b1, o1);
+    store8(accRk + b2, o2);
+  } else {
+    store8(dRk + b1, o1);
+    store8(dRk + b2, o2);
+  }
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     o1.x[e] = gvl * dv1.x[e];
@@ -342,8 +351,13 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 2 : 1) unmix_vec_kernel(
       o2.x[e] = gvr * dv2.x[e] + a2.x[e];
     }
   }
-  store8(dRv + b1, o1);
-  store8(dRv + b2, o2);
+  if (to_acc) {
+    store8(accRv + b1, o1);
+    store8(accRv + b2, o2);
+  } else {
+    store8(dRv + b1, o1);
+    store8(dRv + b2, o2);
+  }
   if (u == 0) {  // column-contiguous partials: gpart[(g*H + h) * rows + bt]
     const int64_t rows = (int64_t)s.B * s.T;
     gpart[(0 * s.H + h) * rows + bt] = s_kl;
@@ -441,13 +455,13 @@ cudaError_t launch_prep(const SwaShape& s, const void* q, const void* k, const v
 
 cudaError_t launch_unmix(const SwaShape& s, const void* dk_bar, const void* dv_bar, const void* k,
                          const void* v, const void* Rk, const void* Rv, const float* gates, void* dk, void* dv,
-                         void* dRk, void* dRv, int accumulate, float* gpart, const float* dq_acc, void* dq,
-                         cudaStream_t st) {
+                         void* dRk, void* dRv, float* accRk, float* accRv, int dr_mode, float* gpart,
+                         const float* dq_acc, void* dq, cudaStream_t st) {
   const RopeTable rt = rope_table(s);
   MAGLEV_EW_DISPATCH(s.dtype, s.hd,
                      unmix_vec_kernel<T, HD><<<blocks_for(s, HD / 16), 256, 0, st>>>(
                          s, rt, (const T*)dk_bar, (const T*)dv_bar, (const T*)k, (const T*)v, (const T*)Rk, (const T*)Rv, gates,
-                         (T*)dk, (T*)dv, (T*)dRk, (T*)dRv, accumulate, gpart, dq_acc, (T*)dq));
+                         (T*)dk, (T*)dv, (T*)dRk, (T*)dRv, accRk, accRv, dr_mode, gpart, dq_acc, (T*)dq));
   return cudaGetLastError();
 }
 

@@ -45,13 +45,17 @@ cudaError_t launch_attn_bwd_dkdv_simt(const SwaShape& s, const void* q_rot, cons
                                       const void* v_bar, const void* dout, const float* lse,
                                       const float* delta, void* dk_bar, void* dv_bar,
                                       cudaStream_t st);
+// How unmix stores dL/dR (values of maglev_dr_mode): DR_WRITE dR = g (dtype);
+// DR_FIRST acc = g; DR_ADD acc += g; DR_LAST dR = acc + g (dtype), with the
+// running sums acc in fp32.
+constexpr int DR_WRITE = 0, DR_FIRST = 1, DR_ADD = 2, DR_LAST = 3;
 // dk, dv, dR_k, dR_v (and dq from dq_acc when non-null) and per-row gate
 // partials gpart[(g*H + h) * B*T + row] from dk_bar, dv_bar (activation type).
 cudaError_t launch_unmix(const SwaShape& s, const void* dk_bar, const void* dv_bar,
                          const void* k, const void* v, const void* Rk, const void* Rv,
                          const float* gates, void* dk, void* dv, void* dRk, void* dRv,
-                         int accumulate, float* gpart, const float* dq_acc, void* dq,
-                         cudaStream_t st);
+                         float* accRk, float* accRv, int dr_mode, float* gpart,
+                         const float* dq_acc, void* dq, cudaStream_t st);
 cudaError_t launch_gate_reduce(int64_t rows, int H, const float* gpart, const float* gates,
                                float* dgate, cudaStream_t st);
 

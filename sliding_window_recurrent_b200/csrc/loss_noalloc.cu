@@ -39,12 +39,33 @@ __global__ void __launch_bounds__(NOALLOC_THREADS) noalloc_partial_kernel(
   const int64_t lo = (int64_t)blockIdx.x * NOALLOC_CHUNK;
   const int64_t hi = min(n, lo + NOALLOC_CHUNK);
   float acc = 0.f;
-  for (int64_t i = lo + threadIdx.x; i < hi; i += NOALLOC_THREADS) {
-    const float diff = to_f(m[i]) - to_f(mt[i]);
-    acc = fmaf(diff, diff, acc);
-    const float g = scale_grad * diff;
-    if (dm) dm[i] = from_f<T>(accumulate ? to_f(dm[i]) + g : g);
-    if (dmt) dmt[i] = from_f<T>(-g);
+  if ((n & 7) == 0) {
+    // 8 elements (16 or 32 bytes) per thread and step; NOALLOC_CHUNK is a
+    // multiple of 8, so every vector lies inside one chunk
+    for (int64_t i = lo + 8 * threadIdx.x; i < hi; i += 8 * NOALLOC_THREADS) {
+      float a[8], b[8], d[8];
+      load8f(m + i, a);
+      load8f(mt + i, b);
+      if (dm && accumulate) load8f(dm + i, d);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float diff = a[e] - b[e];
+        acc = fmaf(diff, diff, acc);
+        const float g = scale_grad * diff;
+        a[e] = (dm && accumulate) ? d[e] + g : g;
+        b[e] = -g;
+      }
+      if (dm) store8f(dm + i, a);
+      if (dmt) store8f(dmt + i, b);
+    }
+  } else {
+    for (int64_t i = lo + threadIdx.x; i < hi; i += NOALLOC_THREADS) {
+      const float diff = to_f(m[i]) - to_f(mt[i]);
+      acc = fmaf(diff, diff, acc);
+      const float g = scale_grad * diff;
+      if (dm) dm[i] = from_f<T>(accumulate ? to_f(dm[i]) + g : g);
+      if (dmt) dmt[i] = from_f<T>(-g);
+    }
   }
   acc = warp_sum(acc);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x / 32] = acc;
@@ -71,19 +92,25 @@ __global__ void __launch_bounds__(NOALLOC_THREADS) noalloc_final_kernel(
   }
 }
 
-// Device address of g_loss_scratch on the current device, looked up once per
-// device with that device current. In host code the symbol itself is only a
-// host-side stand-in and must never be handed to a kernel.
+// Device address of g_loss_scratch on the current device. In host code the
+// symbol itself is only a host-side stand-in and must never be handed to a
+// kernel. The address is looked up with the device current on the first call
+// and again on every call whose stream is not being captured (a device reset
+// reloads the module, possibly at another address); a call made during stream
+// capture uses the address cached by an earlier call on that device.
 std::mutex g_scratch_mu;
 float* g_scratch_addr[128];
 
-cudaError_t scratch_address(float** out) {
+cudaError_t scratch_address(cudaStream_t s, float** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  const bool capturing = cudaStreamIsCapturing(s, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  if (!capturing || !g_scratch_addr[dev]) {
+    if (capturing) return cudaErrorStreamCaptureUnsupported;  // first call on this device inside a capture
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_loss_scratch);
     if (e != cudaSuccess) return e;
@@ -126,13 +153,16 @@ extern "C" maglev_status maglev_consistency_loss_noalloc(const void* m, const vo
     return fail_msg(MAGLEV_ERR_UNSUPPORTED,
                     "maglev_consistency_loss_noalloc handles at most 67108864 elements (rows * d); "
                     "use maglev_consistency_loss with a workspace for larger inputs");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   float* partials = nullptr;
-  cudaError_t e = scratch_address(&partials);
+  cudaError_t e = scratch_address(s, &partials);
+  if (e == cudaErrorStreamCaptureUnsupported)
+    return fail_msg(MAGLEV_ERR_CUDA,
+                    "maglev_consistency_loss_noalloc: the first call on a device must come before any stream capture");
   if (e != cudaSuccess) return fail_msg(MAGLEV_ERR_CUDA, cudaGetErrorString(e));
   const double ic = inv_count == 0.0f ? 1.0 / (double)rows : (double)inv_count;
   const double sl = (double)lambda * ic / std::sqrt((double)d);
   const int nblk = (int)((n + NOALLOC_CHUNK - 1) / NOALLOC_CHUNK);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dtype == MAGLEV_BF16)
     noalloc_partial_kernel<bf16><<<nblk, NOALLOC_THREADS, 0, s>>>(
         (const bf16*)m, (const bf16*)m_target, n, (float)(2.0 * sl), (bf16*)dm, (bf16*)dm_target,

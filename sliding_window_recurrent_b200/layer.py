@@ -7,7 +7,7 @@ from __future__ import annotations
 
 import torch
 
-from . import (DecodeDesc, MAGLEV_BF16, MAGLEV_F32, SwaDesc, maglev_consistency_loss,
+from . import (DecodeDesc, MAGLEV_BF16, MAGLEV_DR_WRITE, MAGLEV_F32, SwaDesc, maglev_consistency_loss,
                maglev_consistency_workspace_bytes, maglev_decode_mem_project, maglev_decode_step,
                maglev_inject_swa_bwd, maglev_inject_swa_fwd, maglev_swa_bwd_workspace_bytes,
                maglev_swa_saved_bytes)
@@ -62,10 +62,13 @@ class InjectedSWALayer:
         return self.loss
 
     def backward(self, k, v, dout, gates=None, m_shift=None, w_mk=None, w_mv=None,
-                 accumulate_dR=False, stream=None):
+                 dR_mode=MAGLEV_DR_WRITE, dR_acc=(None, None), stream=None):
+        """dR_mode / dR_acc: how dL/dR is stored (maglev_dr_mode) and the fp32
+        running sums it reads or writes when several layers share W^rec."""
         maglev_inject_swa_bwd(self.desc, k, v, self.R_k, self.R_v, gates, self.out, self.lse,
                               self.saved, dout, self.dq, self.dk, self.dv, self.dR_k, self.dR_v,
-                              accumulate_dR, self.dgate, m_shift if self.inject else None, w_mk, w_mv,
+                              dR_acc[0], dR_acc[1], dR_mode, self.dgate,
+                              m_shift if self.inject else None, w_mk, w_mv,
                               self.dm_shift, self.dw_mk, self.dw_mv, self.workspace, stream)
 
 

@@ -13,7 +13,8 @@ One training step:
             P layers (injected, reading R_k, R_v) -> memory_state(O_P last) = m
             consistency_loss(m, m') -> loss, dm, dm'
   backward  memory_state_bwd(dm) + dout -> P's last layer; P layers in reverse,
-            summing dR_k, dR_v; mem_project_bwd -> dm_shift, dW_mk, dW_mv;
+            summing dR_k, dR_v in fp32 (rounded once, by layer 0);
+            mem_project_bwd -> dm_shift, dW_mk, dW_mv;
             memory_state_bwd(dm' + shifted dm_shift) + dout -> Q's last layer;
             Q layers in reverse.
 Every layer's own upstream gradient `dout` comes from the caller. This module
@@ -23,7 +24,7 @@ from __future__ import annotations
 
 import torch
 
-from . import (SwaDesc, maglev_consistency_loss, maglev_consistency_workspace_bytes, maglev_inject_swa_bwd,
+from . import (MAGLEV_DR_ADD, MAGLEV_DR_FIRST, MAGLEV_DR_LAST, MAGLEV_DR_WRITE, SwaDesc, maglev_consistency_loss, maglev_consistency_workspace_bytes, maglev_inject_swa_bwd,
                maglev_inject_swa_fwd, maglev_mem_project, maglev_mem_project_bwd, maglev_memory_state,
                maglev_memory_state_bwd, maglev_swa_bwd_workspace_bytes, maglev_swa_saved_bytes)
 from .layer import CODE, TORCH_DTYPE, _bytes
@@ -70,6 +71,10 @@ class PrefillerDecoderStack:
         self.rstd_q, self.rstd_p = e(B * T, t=torch.float32), e(B * T, t=torch.float32)
         self.R_k, self.R_v = e(B, T, d), e(B, T, d)
         self.dR_k, self.dR_v = e(B, T, d), e(B, T, d)
+        # fp32 running sums of dL/dR over P's layers (rounded once into dR_k, dR_v)
+        n_acc = 1 if len(self.p) > 1 else 0
+        self.dR_acc_k = e(n_acc * B, T, d, t=torch.float32) if n_acc else None
+        self.dR_acc_v = e(n_acc * B, T, d, t=torch.float32) if n_acc else None
         self.dm, self.dm_prime, self.dm_shift = e(B, T, d), e(B, T, d), e(B, T, d)
         self.dw_mk, self.dw_mv = e(d, d), e(d, d)
         self.dout_p_last, self.dout_q_last = e(B, T, H, hd), e(B, T, H, hd)
@@ -104,8 +109,9 @@ class PrefillerDecoderStack:
             _, k, v, g = p_inputs[i]
             dout = self.dout_p_last if i == n - 1 else p_douts[i]
             maglev_inject_swa_bwd(L.desc, k, v, self.R_k, self.R_v, g, L.out, L.lse, L.saved, dout, L.dq, L.dk,
-                                  L.dv, self.dR_k, self.dR_v, i != n - 1, L.dgate, None, None, None, None, None,
-                                  None, self.workspace, stream)
+                                  L.dv, self.dR_k, self.dR_v, self.dR_acc_k, self.dR_acc_v,
+                                  self._dr_mode(i, n), L.dgate, None, None, None, None, None, None,
+                                  self.workspace, stream)
         maglev_mem_project_bwd(self.p[0].desc, self.m_shift, w_mk, w_mv, self.dR_k, self.dR_v, self.dm_shift,
                                self.dw_mk, self.dw_mv, stream)
         maglev_memory_state_bwd(B, T, d, code, self.q[-1].out, self.rstd_q, self.dm_prime, self.dm_shift,
@@ -116,8 +122,18 @@ class PrefillerDecoderStack:
             _, k, v = q_inputs[i]
             dout = self.dout_q_last if i == n - 1 else q_douts[i]
             maglev_inject_swa_bwd(L.desc, k, v, None, None, None, L.out, L.lse, L.saved, dout, L.dq, L.dk, L.dv,
-                                  None, None, False, None, None, None, None, None, None, None, self.workspace,
-                                  stream)
+                                  None, None, None, None, MAGLEV_DR_WRITE, None, None, None, None, None, None,
+                                  None, self.workspace, stream)
+
+    @staticmethod
+    def _dr_mode(i, n):
+        """P's backward runs from layer n-1 down to 0: the first call starts the
+        fp32 sum, the last one adds its share and rounds the total into dR."""
+        if n == 1:
+            return MAGLEV_DR_WRITE
+        if i == n - 1:
+            return MAGLEV_DR_FIRST
+        return MAGLEV_DR_LAST if i == 0 else MAGLEV_DR_ADD
 
     def step(self, q_inputs, p_inputs, q_douts, p_douts, w_mk, w_mv, stream=None):
         self.forward(q_inputs, p_inputs, w_mk, w_mv, stream)

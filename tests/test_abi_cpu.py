@@ -81,17 +81,25 @@ def test_empty_problems_enqueue_nothing():
         mg.maglev_inject_swa_fwd(d, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
                                  FAKE, FAKE, stream=0)
         mg.maglev_inject_swa_bwd(d, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
-                                 FAKE, FAKE, FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
-                                 FAKE, FAKE, stream=0)
+                                 FAKE, FAKE, FAKE, FAKE, None, None, mg.MAGLEV_DR_WRITE, FAKE, FAKE,
+                                 FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, stream=0)
     mg.maglev_consistency_loss(FAKE, FAKE, 0, 16, mg.MAGLEV_F32, 1.0, 0.0, FAKE, None, None, 0,
                                FAKE, stream=0)
 
 
 def test_bwd_and_loss_and_decode_validation():
-    with pytest.raises(mg.MaglevError):
+    with pytest.raises(mg.MaglevError):  # dR_k is needed in mode WRITE
         mg.maglev_inject_swa_bwd(desc(), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
-                                 FAKE, FAKE, FAKE, None, FAKE, 0, FAKE, None, None, None, None,
-                                 None, None, FAKE, stream=0)
+                                 FAKE, FAKE, FAKE, None, FAKE, None, None, mg.MAGLEV_DR_WRITE, FAKE,
+                                 None, None, None, None, None, None, FAKE, stream=0)
+    for mode, acc, m_shift, what in [(mg.MAGLEV_DR_ADD, None, None, "dR_acc_k"),
+                                     (7, FAKE, None, "dR_mode"),
+                                     (mg.MAGLEV_DR_FIRST, FAKE, FAKE, "m_shift")]:
+        with pytest.raises(mg.MaglevError) as e:
+            mg.maglev_inject_swa_bwd(desc(), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                     FAKE, FAKE, FAKE, None, None, acc, acc, mode, FAKE,
+                                     m_shift, FAKE, FAKE, None, None, None, FAKE, stream=0)
+        assert e.value.status == mg.MAGLEV_ERR_INVALID_ARG and what in str(e.value), str(e.value)
     with pytest.raises(mg.MaglevError):
         mg.maglev_consistency_loss(FAKE, FAKE, 10, 0, mg.MAGLEV_F32, 1.0, 0.0, FAKE, None, None,
                                    0, FAKE, stream=0)

@@ -1,8 +1,11 @@
 """GPU parity of libmaglev against the CPU fp64 oracle, through the C ABI.
 
-Tolerance (normwise, max|gpu - ref| / max|ref| per tensor): 1e-4 for fp32
-storage, 2e-2 for bf16 storage with fp32 accumulation. Index work (window
-membership, ring slots, untouched ring entries) is compared bit-exactly.
+Tolerance: 1e-4 for fp32 storage, 2e-2 for bf16 storage with fp32
+accumulation, on the normwise error max|gpu - ref| / max|ref| of each tensor
+(of each row for LSE and the gate gradients). The full-size layer test also
+bounds the element-wise relative error max|gpu - ref| / max(|ref|, rms(ref)).
+Index work (window membership, ring slots, untouched ring entries) is compared
+bit-exactly.
 """
 import numpy as np
 import pytest
@@ -86,10 +89,17 @@ def run_oracle(wl, x, inject=True, lam=None, bwd=True, pos0=0):
     return res
 
 
-def compare(gpu, ref, dtype, names):
+# LSE [B,H,T] and the gate gradients [4,H] are judged row by row (their rows
+# differ in scale); every other tensor normwise over the whole tensor.
+ROW_METRIC = {"lse", "dgate"}
+
+
+def compare(gpu, ref, dtype, names, elementwise_too=False):
     errs = {}
     for n in names:
-        errs[n] = assert_close(gpu[n], ref[n], dtype, n)
+        errs[n] = assert_close(gpu[n], ref[n], dtype, n, "rows" if n in ROW_METRIC else "normwise")
+        if elementwise_too and n not in ROW_METRIC:
+            errs[n + ":elementwise"] = assert_close(gpu[n], ref[n], dtype, n, "elementwise")
     return errs
 
 
@@ -135,7 +145,8 @@ def test_layer_bf16_full_size():
     x = synth.layer_inputs(wl, 1234)
     g = run_gpu(wl, x, lam=wl["lam"])
     r = run_oracle(wl, x, lam=wl["lam"])
-    compare(g, r, "bf16", FWD + BWD)
+    errs = compare(g, r, "bf16", FWD + BWD, elementwise_too=True)
+    print("full-size layer errors:", {k: f"{v:.2e}" for k, v in errs.items()})
     assert abs(g["loss"] - r["loss"]) <= 2e-2 * abs(r["loss"])
 
 
@@ -186,30 +197,38 @@ def test_window_perturbation_bitwise():
     assert np.abs(pert[0, i - 40] - base[0, i - 40]).max() > 0
 
 
-def test_accumulated_memory_gradient_over_layers():
-    """accumulate_dR sums dL/dR over layers that share W^rec."""
-    wl = wl_of("layer_bf16", B=1, T=256, H=2, hd=64, d=64, W=32, dtype="f32")
-    xs = [synth.layer_inputs(wl, 40, layer=l) for l in range(2)]
-    B, T, H, hd, d, W = 1, 256, 2, 64, 64, 32
+@pytest.mark.parametrize("dtype,hd,n_layers", [("f32", 64, 3), ("bf16", 128, 4)])
+def test_accumulated_memory_gradient_over_layers(dtype, hd, n_layers):
+    """dR_mode FIRST / ADD / LAST sums dL/dR over layers that share W^rec in
+    fp32 and rounds the total once; mode FIRST and ADD leave dR_k/dR_v alone."""
+    wl = wl_of("layer_bf16", B=1, T=256, H=2, hd=hd, d=64, W=32, dtype=dtype)
+    xs = [synth.layer_inputs(wl, 40, layer=l) for l in range(n_layers)]
+    B, T, H, d, W = 1, 256, 2, 64, 32
+    td = torch.bfloat16 if dtype == "bf16" else torch.float32
     m, wk, wv = dev(xs[0]["m_shift"]), dev(xs[0]["w_mk"]), dev(xs[0]["w_mv"])
-    dRk = torch.zeros(B, T, H * hd, device="cuda")
-    dRv = torch.zeros(B, T, H * hd, device="cuda")
+    dRk = torch.full((B, T, H * hd), 7.0, dtype=td, device="cuda")
+    dRv = torch.full((B, T, H * hd), 7.0, dtype=td, device="cuda")
+    acc = (torch.empty(B, T, H * hd, device="cuda"), torch.empty(B, T, H * hd, device="cuda"))
     want_k = 0
     want_v = 0
     Rk, Rv = oracle.mem_project(xs[0]["m_shift"].f64, xs[0]["w_mk"].f64, xs[0]["w_mv"].f64)
-    for l, x in enumerate(xs):
-        L = InjectedSWALayer(B, T, H, hd, d, W, dtype="f32")
+    modes = [mg.MAGLEV_DR_FIRST] + [mg.MAGLEV_DR_ADD] * (n_layers - 2) + [mg.MAGLEV_DR_LAST]
+    for l, (x, mode) in enumerate(zip(xs, modes)):
+        L = InjectedSWALayer(B, T, H, hd, d, W, dtype=dtype)
         q, k, v, gt = dev(x["q"]), dev(x["k"]), dev(x["v"]), dev(x["gates"])
         L.forward(q, k, v, gt, m, wk, wv)
         L.dR_k, L.dR_v = dRk, dRv
-        L.backward(k, v, dev(x["dout"]), gt, accumulate_dR=(l > 0))
+        L.backward(k, v, dev(x["dout"]), gt, dR_mode=mode, dR_acc=acc)
+        if mode != mg.MAGLEV_DR_LAST:
+            torch.cuda.synchronize()
+            assert torch.all(dRk == 7.0) and torch.all(dRv == 7.0), "running sums stay in dR_acc"
         g = oracle.inject_swa_backward(x["q"].f64, x["k"].f64, x["v"].f64, Rk, Rv,
                                        x["gates"].astype(np.float64), x["dout"].f64, W)
         want_k = want_k + g["dR_k"]
         want_v = want_v + g["dR_v"]
     torch.cuda.synchronize()
-    assert_close(host(dRk), want_k, "f32", "dR_k sum")
-    assert_close(host(dRv), want_v, "f32", "dR_v sum")
+    assert_close(host(dRk), want_k, dtype, "dR_k sum")
+    assert_close(host(dRv), want_v, dtype, "dR_v sum")
 
 
 # --------------------------------------------------------------------------- consistency loss
@@ -315,26 +334,32 @@ def test_decode_full_shape_mixed_positions():
         assert normwise(vr[b][:, s_], vr2[i][:, s_]) <= TOL["bf16"], (b, pos[b])
 
 
-def test_decode_matches_training_row():
-    """Ring filled with the forward's mixed entries: decode at p equals forward row p."""
-    wl = wl_of("layer_bf16", B=1, T=700, H=2, hd=128, d=128, W=512, dtype="f32")
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_decode_matches_training_row(dtype):
+    """Ring filled with the forward's mixed entries (in the ring's storage
+    type): decode at p equals forward row p -- recurrence equals teacher
+    forcing when the ring holds what the training pass mixed."""
+    wl = wl_of("layer_bf16", B=1, T=700, H=2, hd=128, d=128, W=512, dtype=dtype)
     x = synth.layer_inputs(wl, 8)
     B, T, H, hd, W = 1, 700, 2, 128, 512
     Rk, Rv = oracle.mem_project(x["m_shift"].f64, x["w_mk"].f64, x["w_mv"].f64)
     f = oracle.inject_swa_forward(x["q"].f64, x["k"].f64, x["v"].f64, Rk, Rv,
                                   x["gates"].astype(np.float64), W)
-    for p in (300, 511, 699):
+    for p in (0, 300, 511, 699):
         kr = np.zeros((1, H, W, hd), np.float32)
         vr = np.zeros((1, H, W, hd), np.float32)
         for j in range(max(0, p - W + 1), p):
             kr[0, :, j % W] = f["k_bar"][0, j]
             vr[0, :, j % W] = f["v_bar"][0, j]
-        S = DecodeLayerState(1, H, hd, 128, W, dtype="f32")
+        kr_t = synth.Tensor.from_float(kr, dtype)
+        vr_t = synth.Tensor.from_float(vr, dtype)
+        S = DecodeLayerState(1, H, hd, 128, W, dtype=dtype)
         pos_t = torch.tensor([p], dtype=torch.int64, device="cuda")
-        S.mem_project(pos_t, dev(x["m_shift"].bits[:, p]), dev(x["w_mk"]), dev(x["w_mv"]))
-        o = S.step(pos_t, dev(x["q"].bits[:, p]), dev(x["k"].bits[:, p]), dev(x["v"].bits[:, p]),
-                   dev(x["gates"]), dev(kr), dev(vr))
-        assert_close(host(o)[0], f["out"][0, p], "f32", f"decode row {p}")
+        row = lambda t: synth.Tensor(np.ascontiguousarray(t.bits[:, p]), t.dtype)
+        S.mem_project(pos_t, dev(row(x["m_shift"])), dev(x["w_mk"]), dev(x["w_mv"]))
+        o = S.step(pos_t, dev(row(x["q"])), dev(row(x["k"])), dev(row(x["v"])),
+                   dev(x["gates"]), dev(kr_t), dev(vr_t))
+        assert_close(host(o)[0], f["out"][0, p], dtype, f"decode row {p}")
 
 
 def test_device_status_clean():

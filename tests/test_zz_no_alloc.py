@@ -5,9 +5,10 @@ that passes only its input and output tensors, or a latency-critical loop in
 which cudaMalloc (which may synchronise the device) is not allowed. For them
 the library keeps the loss's partial sums in a file-scope device array. This
 test calls that entry point through the C ABI and checks it against the
-workspace-taking maglev_consistency_loss on the same inputs, for two calls in
-a row (a large problem, then a smaller one, so stale partials from the first
-call would show), and checks that oversize inputs are refused.
+workspace-taking maglev_consistency_loss and against the CPU oracle on the
+same inputs, for two calls in a row (a large problem, then a smaller one, so
+stale partials from the first call would show), and checks that oversize
+inputs are refused.
 
 It lives in its own file, collected last, and passes both alone in a fresh
 process and after the rest of the suite.
@@ -15,6 +16,7 @@ process and after the rest of the suite.
 import numpy as np
 import pytest
 
+import oracle
 import synth
 from helpers import TOL, assert_close, dev, host
 
@@ -60,6 +62,13 @@ def test_noalloc_matches_workspace_entry_point_twice(dtype):
         assert abs(g_loss - r_loss) <= 1e-5 * abs(r_loss), (call, g_loss, r_loss)
         assert_close(host(got[1]), host(ref[1]), dtype, f"dm call {call}")
         assert_close(host(got[2]), host(ref[2]), dtype, f"dm_target call {call}")
+        # and directly against the CPU oracle of the loss
+        o_loss, o_dm, o_dmt = oracle.consistency_loss(host(m), host(t), lam)
+        if accumulate:
+            o_dm = o_dm + host(dm0)
+        assert abs(g_loss - o_loss) <= 1e-5 * abs(o_loss), (call, g_loss, o_loss)
+        assert_close(host(got[1]), o_dm, dtype, f"dm vs oracle, call {call}")
+        assert_close(host(got[2]), o_dmt, dtype, f"dm_target vs oracle, call {call}")
     assert TOL[dtype] > 0
 
 
