@@ -65,6 +65,21 @@ def gate_slope(a):
     return 2.0 * s * (1.0 - s)
 
 
+def gate_rows(gate_logits):
+    """The four per-head gate logits (k_loc, k_rec, v_loc, v_rec) as a [4, H]
+    array. rainbus, 方法步骤详情, gives the key's gates and says the value is
+    mixed "likewise"; a [2, H] argument is the reading in which the value reuses
+    the key's two gates (shared K/V gates: rows loc, rec)."""
+    a = np.asarray(gate_logits, dtype=np.float64)
+    return np.concatenate([a, a]) if a.shape[0] == 2 else a
+
+
+def fold_gate_grads(dgate4, gate_logits):
+    """Gradient of the logits as given: [4, H] as is, or for shared K/V gates
+    [2, H] the sum of the key's and the value's share of each gate."""
+    return dgate4[:2] + dgate4[2:] if np.asarray(gate_logits).shape[0] == 2 else dgate4
+
+
 def rope_angles(pos, hd: int, base: float):
     """angle[..., c] = pos * base^(-2c/hd), c = 0..hd/2-1 (rainbus, 前置知识: RoPE)."""
     c = np.arange(hd // 2, dtype=np.float64)
@@ -138,7 +153,8 @@ def inject_swa_forward(q, k, v, R_k, R_v, gate_logits, window: int, pos0: int = 
 
     q, k, v: [B, T, H, hd] pre-RoPE local projections.
     R_k, R_v: [B, T, H*hd] projected shifted memory (row t uses m'_{t-1}).
-    gate_logits: [4, H] = (k_loc, k_rec, v_loc, v_rec).
+    gate_logits: [4, H] = (k_loc, k_rec, v_loc, v_rec), or [2, H] = (loc, rec)
+    shared by the key and the value (see gate_rows).
     Returns a dict with out [B,T,H,hd], lse [B,H,T] and the intermediates.
     """
     B, T, H, hd = q.shape
@@ -148,7 +164,7 @@ def inject_swa_forward(q, k, v, R_k, R_v, gate_logits, window: int, pos0: int = 
     k_loc = rope(k, posb, rope_base)
     res = {"q_rot": q_rot, "k_loc": k_loc}
     if inject:
-        g = gate(gate_logits)                                 # [4, H]
+        g = gate(gate_rows(gate_logits))                      # [4, H]
         Rk = R_k.reshape(B, T, H, hd)
         Rv = R_v.reshape(B, T, H, hd)
         n = rmsnorm(Rk, eps)                                  # per head, hd channels
@@ -220,7 +236,7 @@ def inject_swa_backward(q, k, v, R_k, R_v, gate_logits, dout, window: int, pos0:
             np.sum(dv_bar * v, axis=(0, 1, 3)),
             np.sum(dv_bar * R_v.reshape(B, T, H, hd), axis=(0, 1, 3)),
         ])
-        out["dgate"] = dg * gate_slope(gate_logits)
+        out["dgate"] = fold_gate_grads(dg * gate_slope(gate_rows(gate_logits)), gate_logits)
     else:
         out["dk"] = rope(dk_bar, posb, rope_base, inverse=True)
         out["dv"] = dv_bar
@@ -281,18 +297,27 @@ def stack_forward_backward(q_layers, p_layers, w_mk, w_mv, lam: float, rope_base
     `inv_count` is the loss's 1/|I| (default 1/(B*T)); batch rows are
     independent apart from |I| and the sums over rows (loss, dW, gate grads),
     so a slice of rows with the full batch's |I| reproduces those rows.
+    Per-layer memory projection (rainbus, 未来方向: 逐层记忆投影): when every P
+    layer dict carries its own w_mk, w_mv, layer l reads R^l = m_shift W^l^T,
+    the shifted memory's gradient is the sum of every layer's dR^l W^l, and
+    each layer's dW^l is returned in its p_grads entry (w_mk, w_mv unused).
     """
     store = store if store is not None else (lambda x: x)
     B, T, H, hd = q_layers[-1]["q"].shape
     D = H * hd
+    per_layer = all("w_mk" in L for L in p_layers)
     qf = [inject_swa_forward(L["q"], L["k"], L["v"], None, None, None, L["window"], 0, rope_base, eps,
                              inject=False) for L in q_layers]
     oq = qf[-1]["out"].reshape(B, T, D)
     m_prime = memory_state(oq, eps)
     m_shift = shift_memory(m_prime)
-    R_k, R_v = mem_project(m_shift, w_mk, w_mv)
-    pf = [inject_swa_forward(L["q"], L["k"], L["v"], R_k, R_v, L["gates"], L["window"], 0, rope_base, eps)
-          for L in p_layers]
+    if per_layer:
+        Rs = [mem_project(m_shift, L["w_mk"], L["w_mv"]) for L in p_layers]
+    else:
+        Rs = [mem_project(m_shift, w_mk, w_mv)] * len(p_layers)
+    R_k, R_v = Rs[0]
+    pf = [inject_swa_forward(L["q"], L["k"], L["v"], Rs[i][0], Rs[i][1], L["gates"], L["window"], 0, rope_base,
+                             eps) for i, L in enumerate(p_layers)]
     op = pf[-1]["out"].reshape(B, T, D)
     m = memory_state(op, eps)
     loss, dm, dm_prime = consistency_loss(m.reshape(B * T, D), m_prime.reshape(B * T, D), lam, inv_count)
@@ -303,16 +328,26 @@ def stack_forward_backward(q_layers, p_layers, w_mk, w_mv, lam: float, rope_base
     p_grads = []
     dR_k = np.zeros_like(R_k)
     dR_v = np.zeros_like(R_v)
+    dm_shift = np.zeros_like(m_shift)
     for i, L in enumerate(p_layers):
         dout = L["dout"]
         if i == len(p_layers) - 1:
             dout = store(dout + rmsnorm_backward(op, dm, eps).reshape(B, T, H, hd))
-        g = inject_swa_backward(L["q"], L["k"], L["v"], R_k, R_v, L["gates"], dout, L["window"], 0,
+        g = inject_swa_backward(L["q"], L["k"], L["v"], Rs[i][0], Rs[i][1], L["gates"], dout, L["window"], 0,
                                 rope_base, eps)
-        dR_k += g["dR_k"]
-        dR_v += g["dR_v"]
-        p_grads.append({"dq": g["dq"], "dk": g["dk"], "dv": g["dv"], "dgate": g["dgate"], "dout": dout})
-    dm_shift, dw_mk, dw_mv = mem_project_backward(m_shift, w_mk, w_mv, dR_k, dR_v)
+        grads = {"dq": g["dq"], "dk": g["dk"], "dv": g["dv"], "dgate": g["dgate"], "dout": dout}
+        if per_layer:
+            dms, dwk, dwv = mem_project_backward(m_shift, L["w_mk"], L["w_mv"], g["dR_k"], g["dR_v"])
+            dm_shift += dms
+            grads.update(dR_k=g["dR_k"], dR_v=g["dR_v"], dw_mk=dwk, dw_mv=dwv)
+        else:
+            dR_k += g["dR_k"]
+            dR_v += g["dR_v"]
+        p_grads.append(grads)
+    if per_layer:
+        dw_mk = dw_mv = None
+    else:
+        dm_shift, dw_mk, dw_mv = mem_project_backward(m_shift, w_mk, w_mv, dR_k, dR_v)
     # m_shift[t] = m'[t-1]: its gradient lands one row earlier
     dm_prime = dm_prime.copy()
     dm_prime[:, :-1] += dm_shift[:, 1:]
@@ -361,7 +396,7 @@ def decode_step(pos, q, k, v, krec_rot, vrec, gate_logits, k_ring, v_ring,
     q_rot = rope(q, posb, rope_base)
     k_loc = rope(k, posb, rope_base)
     if inject:
-        g = gate(gate_logits)
+        g = gate(gate_rows(gate_logits))
         k_new = g[0][None, :, None] * k_loc + g[1][None, :, None] * krec_rot
         v_new = g[2][None, :, None] * v + g[3][None, :, None] * vrec
     else:

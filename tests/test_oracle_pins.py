@@ -357,12 +357,19 @@ def test_mem_project_backward_matches_autograd():
 
 
 # ---------------------------------------------------------------- stack (Q -> memory -> P -> loss)
-def _stack(B=1, T=7, H=1, hd=4, nq=2, np_=2):
+def _stack(B=1, T=7, H=1, hd=4, nq=2, np_=2, variant="shared"):
+    """variant: "shared" (one W^rec, four gates), "per_layer" (each P layer its
+    own W^rec), "kv_gates" (one W^rec, [2, H] gates shared by K and V)."""
     D = H * hd
+    ng = 2 if variant == "kv_gates" else 4
     ql = [dict(q=rand(B, T, H, hd), k=rand(B, T, H, hd), v=rand(B, T, H, hd), dout=rand(B, T, H, hd),
                window=3 if i % 2 == 0 else T) for i in range(nq)]
     pl = [dict(q=rand(B, T, H, hd), k=rand(B, T, H, hd), v=rand(B, T, H, hd), dout=rand(B, T, H, hd),
-               gates=RNG.uniform(-2, 2, (4, H)), window=3) for _ in range(np_)]
+               gates=RNG.uniform(-2, 2, (ng, H)), window=3) for _ in range(np_)]
+    if variant == "per_layer":
+        for L in pl:
+            L["w_mk"], L["w_mv"] = rand(D, D) / np.sqrt(D), rand(D, D) / np.sqrt(D)
+        return ql, pl, None, None
     return ql, pl, rand(D, D) / np.sqrt(D), rand(D, D) / np.sqrt(D)
 
 
@@ -385,10 +392,12 @@ def test_shift_memory_and_state():
     np.testing.assert_allclose(oracle.memory_state(o), ref, rtol=1e-13)
 
 
-def test_stack_central_differences():
+@pytest.mark.parametrize("variant", ["shared", "per_layer", "kv_gates"])
+def test_stack_central_differences(variant):
     """Every gradient of the stack objective, including the path from P's loss
-    and injection back through the shift into Q's last layer."""
-    ql, pl, wk, wv = _stack()
+    and injection back through the shift into Q's last layer; for one shared
+    W^rec, a W^rec per decoder layer, and gates shared by K and V."""
+    ql, pl, wk, wv = _stack(np_=3 if variant == "per_layer" else 2, variant=variant)
     lam = 0.7
     r = oracle.stack_forward_backward(ql, pl, wk, wv, lam)
     cases = []
@@ -399,14 +408,18 @@ def test_stack_central_differences():
         for key in ("q", "k", "v"):
             cases.append((("p", li, key), r["p_grads"][li]["d" + key]))
         cases.append((("p", li, "gates"), r["p_grads"][li]["dgate"]))
-    cases += [(("w", 0, "wk"), r["dw_mk"]), (("w", 0, "wv"), r["dw_mv"])]
+        if variant == "per_layer":
+            cases += [(("p", li, "w_mk"), r["p_grads"][li]["dw_mk"]), (("p", li, "w_mv"), r["p_grads"][li]["dw_mv"])]
+    if variant != "per_layer":
+        cases += [(("w", 0, "wk"), r["dw_mk"]), (("w", 0, "wv"), r["dw_mv"])]
     h = 1e-6
     for (side, li, key), grad in cases:
         for idx in [tuple(RNG.integers(0, s) for s in grad.shape) for _ in range(3)]:
             def j_at(delta):
                 ql2 = [{k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in L.items()} for L in ql]
                 pl2 = [{k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in L.items()} for L in pl]
-                wk2, wv2 = wk.copy(), wv.copy()
+                wk2 = wk.copy() if wk is not None else None
+                wv2 = wv.copy() if wv is not None else None
                 if side == "q":
                     ql2[li][key][idx] += delta
                 elif side == "p":
@@ -416,6 +429,35 @@ def test_stack_central_differences():
                 return _stack_objective(ql2, pl2, wk2, wv2, lam)
             fd = (j_at(h) - j_at(-h)) / (2 * h)
             assert abs(fd - grad[idx]) <= 1e-6 * max(1.0, abs(fd)), (side, li, key, idx, fd, grad[idx])
+
+
+def test_shared_kv_gates_equal_four_equal_gates():
+    """The shared K/V form is the four-gate form with the value's logits set
+    equal to the key's; its gradient is the sum of the two shares."""
+    B, T, H, hd, W = 1, 9, 2, 4, 3
+    q, k, v, dout = (rand(B, T, H, hd) for _ in range(4))
+    Rk, Rv = rand(B, T, H * hd), rand(B, T, H * hd)
+    g2 = RNG.uniform(-2, 2, (2, H))
+    g4 = np.concatenate([g2, g2])
+    f2 = oracle.inject_swa_forward(q, k, v, Rk, Rv, g2, W)
+    f4 = oracle.inject_swa_forward(q, k, v, Rk, Rv, g4, W)
+    assert np.array_equal(f2["out"], f4["out"])
+    d2 = oracle.inject_swa_backward(q, k, v, Rk, Rv, g2, dout, W)["dgate"]
+    d4 = oracle.inject_swa_backward(q, k, v, Rk, Rv, g4, dout, W)["dgate"]
+    assert d2.shape == (2, H)
+    np.testing.assert_allclose(d2, d4[:2] + d4[2:], rtol=1e-14)
+
+
+def test_per_layer_projection_with_equal_weights_equals_shared():
+    """Giving every decoder layer the same W^rec reproduces the shared form:
+    the per-layer dW^l sum to the shared dW."""
+    ql, pl, wk, wv = _stack(np_=3)
+    r = oracle.stack_forward_backward(ql, pl, wk, wv, 0.3)
+    pl2 = [dict(L, w_mk=wk, w_mv=wv) for L in pl]
+    r2 = oracle.stack_forward_backward(ql, pl2, None, None, 0.3)
+    np.testing.assert_allclose(r2["loss"], r["loss"], rtol=1e-14)
+    np.testing.assert_allclose(sum(g["dw_mk"] for g in r2["p_grads"]), r["dw_mk"], rtol=1e-10, atol=1e-13)
+    np.testing.assert_allclose(r2["dm_shift"], r["dm_shift"], rtol=1e-10, atol=1e-13)
 
 
 def test_stack_gates_off_decouples_memory():
