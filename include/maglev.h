@@ -55,7 +55,11 @@ typedef enum { MAGLEV_F32 = 0, MAGLEV_BF16 = 1 } maglev_dtype;
  * width, window W >= 1 (keys j in [i-W+1, i]; W >= T is full causal attention),
  * rope_base (10000 in the d20 model), rms_eps (1e-6), inject (0: plain SWA --
  * memory arguments may be NULL), pos0 (absolute position of row 0), dtype,
- * spin_limit (bound on each in-kernel wait in microseconds, 0 = 1 s). */
+ * spin_limit (bound on each in-kernel wait in microseconds, 0 = 1 s),
+ * shared_kv_gates: 0 -- gate_logits is [4,H] (k_loc, k_rec, v_loc, v_rec);
+ * 1 -- gate_logits is [2,H] (loc, rec), the value reusing the key's gates
+ * ([rainbus] 方法步骤详情 gives the key's gates and mixes the value "likewise");
+ * the gate gradient then has the same [2,H] shape. */
 typedef struct {
   int B, T, H, hd, d_mem, window;
   float rope_base, rms_eps;
@@ -63,16 +67,18 @@ typedef struct {
   int pos0;
   int dtype;
   int64_t spin_limit;
+  int shared_kv_gates;
 } maglev_swa_desc;
 
 /* Shapes of one recurrent decode layer: B sequences, H heads, hd, d_mem,
- * window W = ring length. */
+ * window W = ring length; shared_kv_gates as in maglev_swa_desc. */
 typedef struct {
   int B, H, hd, d_mem, window;
   float rope_base, rms_eps;
   int inject;
   int dtype;
   int64_t spin_limit;
+  int shared_kv_gates;
 } maglev_decode_desc;
 
 /* Library version string (static storage). */
@@ -125,7 +131,7 @@ maglev_status maglev_mem_project(const maglev_swa_desc* desc, const void* m_shif
  *     inputs computed earlier (shared across layers). Unused when inject == 0.
  *   R_k, R_v [B,T,D]: raw projected memory (see a1), written or read as above.
  *   gate_logits [4,H] fp32: (k_loc, k_rec, v_loc, v_rec); g = 2*sigmoid(a),
- *     a = -inf allowed (g = 0).
+ *     a = -inf allowed (g = 0); [2,H] (loc, rec) with shared_kv_gates.
  *   out [B,T,H,hd] (out): o_i = sum_j softmax_j(q~_i . k_bar_j / sqrt(hd)) v_bar_j
  *     over j in [i-W+1, i], with q~ = RoPE(q), k_bar = g_kl RoPE(k) +
  *     g_kr RoPE(RMSNorm_head(R_k)), v_bar = g_vl v + g_vr R_v.
@@ -162,7 +168,8 @@ typedef enum {
  *   dR_acc_k, dR_acc_v [B,T,D] fp32: the running sums, written (FIRST), updated
  *     (ADD) or read (LAST); unused (may be NULL) in mode WRITE.
  *   dR_mode: a maglev_dr_mode value.
- *   dgate_logits [4,H] fp32 (out, overwritten); NULL when inject == 0.
+ *   dgate_logits [4,H] fp32 ([2,H] with shared_kv_gates; out, overwritten);
+ *     NULL when inject == 0.
  *   m_shift, w_mk, w_mv, dm_shift, dw_mk, dw_mv: if m_shift != NULL the call
  *     finishes with maglev_mem_project_bwd on dR_k, dR_v (modes WRITE and LAST).
  *   workspace: maglev_swa_bwd_workspace_bytes(desc) bytes of scratch.
@@ -184,6 +191,23 @@ maglev_status maglev_mem_project_bwd(const maglev_swa_desc* desc, const void* m_
                                      const void* w_mk, const void* w_mv, const void* dR_k,
                                      const void* dR_v, void* dm_shift, void* dw_mk, void* dw_mv,
                                      void* stream);
+
+/* Backward of per-layer memory projections: one W^rec per decoder layer, the
+ * variant [rainbus] 未来方向 lists (逐层记忆投影) beside the shared projection.
+ * Layer l's forward is maglev_mem_project with that layer's weights into its
+ * own R^l; its maglev_inject_swa_bwd writes dL/dR^l in mode MAGLEV_DR_WRITE.
+ *   n_layers L >= 1.
+ *   w_mk, w_mv [L, D, d_mem]: the layers' projections, layer-strided.
+ *   dR_k, dR_v [L, B, T, D]: each layer's dL/dR^l, layer-strided.
+ *   dm_shift [B,T,d_mem] (out, nullable) = sum over l of dR_k^l W_mk^l +
+ *     dR_v^l W_mv^l, accumulated in fp32 over all layers and rounded once.
+ *   dw_mk, dw_mv [L, D, d_mem] (out, nullable as a pair): dW^l = dR^l^T m_shift.
+ * Errors: INVALID_ARG for n_layers < 1 or bad pointers; UNSUPPORTED for bf16
+ * unless d_mem % 8 == 0 and H*hd % 128 == 0. */
+maglev_status maglev_mem_project_bwd_layers(const maglev_swa_desc* desc, int n_layers,
+                                            const void* m_shift, const void* w_mk, const void* w_mv,
+                                            const void* dR_k, const void* dR_v, void* dm_shift,
+                                            void* dw_mk, void* dw_mv, void* stream);
 
 /* Memory state of a decoder stack ([rainbus] 方法步骤详情: m_t is the stack's
  * final state after RMSNorm; the injection reads the shifted memory m_{t-1},
@@ -258,6 +282,23 @@ maglev_status maglev_decode_mem_project(const maglev_decode_desc* desc, const in
                                         const void* m_prev, const void* w_mk, const void* w_mv,
                                         void* krec_rot, void* vrec, void* stream);
 
+/* Ring prefill from a prompt: the bridge from the training form to recurrent
+ * decoding ([rainbus] 研究动机: at inference m_t = P(x_{t-W+1:t}, M_{t-1}) over a
+ * fixed window; 前置知识: the cache is that of plain SWA; [gist]
+ * Inferentiemechanisme: the memory rides in the existing K/V entries).
+ * After maglev_inject_swa_fwd over a prompt of T tokens at positions
+ * pos0..pos0+T-1 (same desc), copies the mixed entries k_bar, v_bar of its
+ * last min(T, W) positions from the forward's `saved` buffer into the rings:
+ * the entry of absolute position j goes to slot j mod W of ring [b, h], with
+ * W = desc->window (the ring length). No other slot changes. The rings then
+ * hold the window that maglev_decode_step continues from at position pos0 + T,
+ * fed with m_{pos0+T-1}.
+ *   saved: the forward's saved buffer (maglev_swa_saved_bytes(desc) bytes).
+ *   k_ring, v_ring [B,H,W,hd] of desc->dtype (in/out).
+ * Errors: INVALID_ARG for a bad desc or a NULL / misaligned pointer. */
+maglev_status maglev_decode_prefill(const maglev_swa_desc* desc, const void* saved, void* k_ring,
+                                    void* v_ring, void* stream);
+
 /* a8 -- one recurrent decode step of one layer over its rolling W-entry K/V
  * ring ([rainbus] 研究动机: m_t = P(x_{t-W+1:t}, M_{t-1}); 前置知识: the cache is
  * that of plain SWA; [gist] Inferentiemechanisme).
@@ -265,7 +306,7 @@ maglev_status maglev_decode_mem_project(const maglev_decode_desc* desc, const in
  *     entry leaves that sequence's ring untouched and writes zeros to its out.
  *   q, k, v [B,H,hd]: local projections of the new token, before RoPE.
  *   krec_rot, vrec [B,H,hd]: from maglev_decode_mem_project (unused if inject == 0).
- *   gate_logits [4,H] fp32: this layer's gates.
+ *   gate_logits [4,H] fp32 ([2,H] with shared_kv_gates): this layer's gates.
  *   k_ring, v_ring [B,H,W,hd] (in/out): post-RoPE, post-mix entries; the entry
  *     of position j lives in slot j mod W. The call writes the new entry to slot
  *     p mod W (no other slot changes), then attends over the live slots

@@ -32,13 +32,14 @@ class SwaDesc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("hd", ctypes.c_int),
                 ("d_mem", ctypes.c_int), ("window", ctypes.c_int), ("rope_base", ctypes.c_float),
                 ("rms_eps", ctypes.c_float), ("inject", ctypes.c_int), ("pos0", ctypes.c_int),
-                ("dtype", ctypes.c_int), ("spin_limit", ctypes.c_int64)]
+                ("dtype", ctypes.c_int), ("spin_limit", ctypes.c_int64), ("shared_kv_gates", ctypes.c_int)]
 
 
 class DecodeDesc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("hd", ctypes.c_int), ("d_mem", ctypes.c_int),
                 ("window", ctypes.c_int), ("rope_base", ctypes.c_float), ("rms_eps", ctypes.c_float),
-                ("inject", ctypes.c_int), ("dtype", ctypes.c_int), ("spin_limit", ctypes.c_int64)]
+                ("inject", ctypes.c_int), ("dtype", ctypes.c_int), ("spin_limit", ctypes.c_int64),
+                ("shared_kv_gates", ctypes.c_int)]
 
 
 def _load():
@@ -67,12 +68,14 @@ _SIGS = {
     "maglev_inject_swa_fwd": ([ctypes.POINTER(SwaDesc)] + [_P] * 13, _I),
     "maglev_inject_swa_bwd": ([ctypes.POINTER(SwaDesc)] + [_P] * 16 + [_I] + [_P] * 9, _I),
     "maglev_mem_project_bwd": ([ctypes.POINTER(SwaDesc)] + [_P] * 9, _I),
+    "maglev_mem_project_bwd_layers": ([ctypes.POINTER(SwaDesc), _I] + [_P] * 9, _I),
     "maglev_consistency_loss": ([_P, _P, _I64, _I, _I, _F, _F, _P, _P, _P, _I, _P, _P], _I),
     "maglev_consistency_loss_noalloc": ([_P, _P, _I64, _I, _I, _F, _F, _P, _P, _P, _I, _P], _I),
     "maglev_memory_state": ([_I, _I, _I, _F, _I] + [_P] * 5, _I),
     "maglev_memory_state_bwd": ([_I, _I, _I, _I] + [_P] * 7, _I),
     "maglev_decode_mem_project": ([ctypes.POINTER(DecodeDesc)] + [_P] * 7, _I),
     "maglev_decode_step": ([ctypes.POINTER(DecodeDesc)] + [_P] * 11, _I),
+    "maglev_decode_prefill": ([ctypes.POINTER(SwaDesc)] + [_P] * 4, _I),
 }
 
 
@@ -200,6 +203,13 @@ def maglev_mem_project_bwd(desc, m_shift, w_mk, w_mv, dR_k, dR_v, dm_shift, dw_m
                                        _ptr(dw_mv), _stream(stream)))
 
 
+def maglev_mem_project_bwd_layers(desc, n_layers, m_shift, w_mk, w_mv, dR_k, dR_v, dm_shift, dw_mk, dw_mv,
+                                  stream=None):
+    _check(_lib.maglev_mem_project_bwd_layers(ctypes.byref(desc), int(n_layers), _ptr(m_shift), _ptr(w_mk),
+                                              _ptr(w_mv), _ptr(dR_k), _ptr(dR_v), _ptr(dm_shift), _ptr(dw_mk),
+                                              _ptr(dw_mv), _stream(stream)))
+
+
 def maglev_consistency_loss(m, m_target, rows, d, dtype, lam, inv_count, loss, dm, dm_target,
                             accumulate_dm, workspace, stream=None):
     _check(_lib.maglev_consistency_loss(_ptr(m), _ptr(m_target), int(rows), int(d), int(dtype),
@@ -237,3 +247,8 @@ def maglev_decode_step(desc, pos, q, k, v, krec_rot, vrec, gate_logits, k_ring, 
     _check(_lib.maglev_decode_step(ctypes.byref(desc), _ptr(pos), _ptr(q), _ptr(k), _ptr(v),
                                    _ptr(krec_rot), _ptr(vrec), _ptr(gate_logits), _ptr(k_ring),
                                    _ptr(v_ring), _ptr(out), _stream(stream)))
+
+
+def maglev_decode_prefill(desc, saved, k_ring, v_ring, stream=None):
+    _check(_lib.maglev_decode_prefill(ctypes.byref(desc), _ptr(saved), _ptr(k_ring), _ptr(v_ring),
+                                      _stream(stream)))

@@ -130,6 +130,7 @@ SwaShape shape_of(const maglev_swa_desc* d) {
   s.pos0 = d->pos0;
   s.inject = d->inject ? 1 : 0;
   s.dtype = d->dtype;
+  s.vg = d->shared_kv_gates ? 0 : 2;
   s.log2_base = std::log2((double)d->rope_base);
   s.eps = d->rms_eps;
   return s;
@@ -522,7 +523,8 @@ maglev_status maglev_inject_swa_bwd(const maglev_swa_desc* d, const void* k, con
                                    dR_acc_k, dR_acc_v, dR_mode, gpart, dq_acc, dq, s),
                 "unmix");
   if (d->inject) {
-    MAGLEV_LAUNCH(1, s, launch_gate_reduce((int64_t)d->B * d->T, d->H, gpart, gate_logits, dgate_logits, s),
+    MAGLEV_LAUNCH(1, s, launch_gate_reduce((int64_t)d->B * d->T, d->H, d->shared_kv_gates ? 1 : 0, gpart,
+                                           gate_logits, dgate_logits, s),
                   "gate_reduce");
     if (m_shift) {
       st = run_mem_project_bwd(d, m_shift, w_mk, w_mv, dR_k, dR_v, dm_shift, dw_mk, dw_mv, s);
@@ -550,6 +552,79 @@ maglev_status maglev_mem_project_bwd(const maglev_swa_desc* d, const void* m_shi
   if (d->B == 0 || d->T == 0) return MAGLEV_OK;
   return run_mem_project_bwd(d, m_shift, w_mk, w_mv, dR_k, dR_v, dm_shift, dw_mk, dw_mv,
                              static_cast<cudaStream_t>(stream));
+}
+
+maglev_status maglev_mem_project_bwd_layers(const maglev_swa_desc* d, int n_layers, const void* m_shift,
+                                            const void* w_mk, const void* w_mv, const void* dR_k,
+                                            const void* dR_v, void* dm_shift, void* dw_mk, void* dw_mv,
+                                            void* stream) {
+  maglev_status st = check_swa(d);
+  if (st != MAGLEV_OK) return st;
+  if (d->d_mem < 1) return fail(MAGLEV_ERR_INVALID_ARG, "d_mem must be >= 1");
+  if (n_layers < 1) return fail(MAGLEV_ERR_INVALID_ARG, "n_layers must be >= 1");
+  NEED_PTR(m_shift);
+  NEED_PTR(w_mk);
+  NEED_PTR(w_mv);
+  NEED_PTR(dR_k);
+  NEED_PTR(dR_v);
+  OPT_PTR(dm_shift);
+  OPT_PTR(dw_mk);
+  OPT_PTR(dw_mv);
+  if ((dw_mk == nullptr) != (dw_mv == nullptr))
+    return fail(MAGLEV_ERR_INVALID_ARG, "dw_mk and dw_mv must both be given or both be NULL");
+  const int64_t M = (int64_t)d->B * d->T, D = (int64_t)d->H * d->hd, K = d->d_mem;
+  const bool tc = d->dtype == MAGLEV_BF16;
+  if (tc && (K % 8 != 0 || D % 128 != 0))
+    return fail(MAGLEV_ERR_UNSUPPORTED, "bf16 per-layer projection needs d_mem %% 8 == 0 and H*hd %% 128 == 0");
+  if (M == 0) return MAGLEV_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t e = elt(d->dtype);
+  const size_t w_layer = (size_t)D * K * e, r_layer = (size_t)M * D * e;
+  int* err = nullptr;
+  st = status_word(&err, s);
+  if (st != MAGLEV_OK) return st;
+  if (dm_shift) {
+    if (tc) {
+      MAGLEV_LAUNCH(1, s, launch_proj_bwd_dm_layers_tc(M, (int)D, (int)K, n_layers, dR_k, dR_v, w_mk, w_mv,
+                                                       dm_shift, spin_limit_of(d->spin_limit), err, s),
+                    "mem_project_bwd_dm_layers_tc");
+    } else {  // fp32: accumulate the layers' products in the fp32 output
+      for (int l = 0; l < n_layers; ++l) {
+        GemmArgs g{};
+        g.M = M;
+        g.N = K;
+        g.K1 = D;
+        g.K2 = D;
+        g.A1 = at<char>(dR_k, l * r_layer);
+        g.sa1m = D;
+        g.sa1k = 1;
+        g.B1 = at<char>(w_mk, l * w_layer);
+        g.sb1k = K;
+        g.sb1n = 1;
+        g.A2 = at<char>(dR_v, l * r_layer);
+        g.sa2m = D;
+        g.sa2k = 1;
+        g.B2 = at<char>(w_mv, l * w_layer);
+        g.sb2k = K;
+        g.sb2n = 1;
+        g.C = dm_shift;
+        g.scm = K;
+        g.scn = 1;
+        g.accumulate = l > 0;
+        g.dtype = d->dtype;
+        MAGLEV_LAUNCH(1, s, launch_gemm_simt(g, s), "mem_project_bwd_dm_gemm");
+      }
+    }
+  }
+  if (dw_mk) {
+    for (int l = 0; l < n_layers; ++l) {
+      st = run_mem_project_bwd(d, m_shift, at<char>(w_mk, l * w_layer), at<char>(w_mv, l * w_layer),
+                               at<char>(dR_k, l * r_layer), at<char>(dR_v, l * r_layer), nullptr,
+                               at<char>(dw_mk, l * w_layer), at<char>(dw_mv, l * w_layer), s);
+      if (st != MAGLEV_OK) return st;
+    }
+  }
+  return MAGLEV_OK;
 }
 
 maglev_status maglev_consistency_loss(const void* m, const void* m_target, int64_t rows, int d,
@@ -641,6 +716,7 @@ static DecShape dec_shape(const maglev_decode_desc* d) {
   s.W = d->window;
   s.inject = d->inject ? 1 : 0;
   s.dtype = d->dtype;
+  s.vg = d->shared_kv_gates ? 0 : 2;
   s.log2_base = std::log2((double)d->rope_base);
   s.eps = d->rms_eps;
   return s;
@@ -689,6 +765,22 @@ maglev_status maglev_decode_mem_project(const maglev_decode_desc* d, const int64
     MAGLEV_LAUNCH(1, s, launch_gemm_simt(g, s), "decode_mem_project_gemm");
   }
   MAGLEV_LAUNCH(1, s, launch_rmsnorm_rope_rows(dec_shape(d), pos, krec_rot, s), "decode_krec_norm_rope");
+  return MAGLEV_OK;
+}
+
+maglev_status maglev_decode_prefill(const maglev_swa_desc* d, const void* saved, void* k_ring, void* v_ring,
+                                    void* stream) {
+  maglev_status st = check_swa(d);
+  if (st != MAGLEV_OK) return st;
+  NEED_PTR(saved);
+  NEED_PTR(k_ring);
+  NEED_PTR(v_ring);
+  if (d->B == 0 || d->T == 0) return MAGLEV_OK;
+  const SavedLayout L = saved_layout(d);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MAGLEV_LAUNCH(1, s, launch_ring_prefill(d->B, d->T, d->H, d->hd, (int)elt(d->dtype), d->window, d->pos0,
+                                          at<char>(saved, L.k), at<char>(saved, L.v), k_ring, v_ring, s),
+                "decode_prefill");
   return MAGLEV_OK;
 }
 

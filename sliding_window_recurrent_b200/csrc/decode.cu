@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(256) decode_step_kernel(
     float v1 = to_f(v[tok + c]), v2 = to_f(v[tok + c + HALF]);
     if (s.inject) {
       const float gkl = gate_value(gates[0 * s.H + h]), gkr = gate_value(gates[1 * s.H + h]);
-      const float gvl = gate_value(gates[2 * s.H + h]), gvr = gate_value(gates[3 * s.H + h]);
+      const float gvl = gate_value(gates[(s.vg + 0) * s.H + h]), gvr = gate_value(gates[(s.vg + 1) * s.H + h]);
       a1 = gkl * a1 + gkr * to_f(krec[tok + c]);
       a2 = gkl * a2 + gkr * to_f(krec[tok + c + HALF]);
       v1 = gvl * v1 + gvr * to_f(vrec[tok + c]);
@@ -316,8 +316,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
         load_pairs<NPL>(vrec + tok, c0, HALF, wa, wb);
         ga = gates[0 * s.H + h];
         gb = gates[1 * s.H + h];
-        gc = gates[2 * s.H + h];
-        gd = gates[3 * s.H + h];
+        gc = gates[(s.vg + 0) * s.H + h];
+        gd = gates[(s.vg + 1) * s.H + h];
       }
       const int64_t p = pos[bh / s.H];
       if (p >= 0) {

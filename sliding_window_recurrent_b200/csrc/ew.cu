@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(256) prep_vec_kernel(SwaShape s, RopeTable rt,
   if (!live) return;
   const float rinv = rsqrtf(ss / HD + s.eps);
   const float gkl = gate_value(gates[0 * s.H + h]), gkr = gate_value(gates[1 * s.H + h]);
-  const float gvl = gate_value(gates[2 * s.H + h]), gvr = gate_value(gates[3 * s.H + h]);
+  const float gvl = gate_value(gates[(s.vg + 0) * s.H + h]), gvr = gate_value(gates[(s.vg + 1) * s.H + h]);
   V8 o1, o2;
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
@@ -278,7 +278,7 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 2 : 1) unmix_vec_kernel(
     return;
   }
   const float gkl = gate_value(gates[0 * s.H + h]), gkr = gate_value(gates[1 * s.H + h]);
-  const float gvl = gate_value(gates[2 * s.H + h]), gvr = gate_value(gates[3 * s.H + h]);
+  const float gvl = gate_value(gates[(s.vg + 0) * s.H + h]), gvr = gate_value(gates[(s.vg + 1) * s.H + h]);
   const V8 r1 = cvt8(r1r), r2 = cvt8(r2r), k1 = cvt8(k1r), k2 = cvt8(k2r);
   float ss = 0.f;
 #pragma unroll
@@ -401,14 +401,17 @@ __global__ void __launch_bounds__(256) delta_vec_kernel(SwaShape s, const T* __r
 }
 
 // dgate[col] = sum_r gpart[col * rows + r] * dg/da, fixed reduction order.
-__global__ void __launch_bounds__(512) gate_reduce_vec_kernel(int64_t rows, const float* __restrict__ gpart,
+// With gates shared by K and V (fold = 2H) the value's partials of the same
+// gate, column col + 2H, are added to the key's: dgate is [2, H].
+__global__ void __launch_bounds__(512) gate_reduce_vec_kernel(int64_t rows, int fold, const float* __restrict__ gpart,
                                                               const float* __restrict__ gates,
                                                               float* __restrict__ dgate) {
   __shared__ float red[16];
   const int col = blockIdx.x;
   const float* g = gpart + (int64_t)col * rows;
+  const float* g2 = fold ? gpart + (int64_t)(col + fold) * rows : nullptr;
   float acc = 0.f;
-  for (int64_t r = threadIdx.x; r < rows; r += 512) acc += g[r];
+  for (int64_t r = threadIdx.x; r < rows; r += 512) acc += g2 ? g[r] + g2[r] : g[r];
   acc = warp_sum(acc);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x / 32] = acc;
   __syncthreads();
@@ -473,9 +476,10 @@ cudaError_t launch_attn_delta(const SwaShape& s, const void* out, const void* do
   return cudaGetLastError();
 }
 
-cudaError_t launch_gate_reduce(int64_t rows, int H, const float* gpart, const float* gates, float* dgate,
-                               cudaStream_t st) {
-  gate_reduce_vec_kernel<<<4 * H, 512, 0, st>>>(rows, gpart, gates, dgate);
+cudaError_t launch_gate_reduce(int64_t rows, int H, int shared_kv, const float* gpart, const float* gates,
+                               float* dgate, cudaStream_t st) {
+  const int cols = shared_kv ? 2 * H : 4 * H;
+  gate_reduce_vec_kernel<<<cols, 512, 0, st>>>(rows, shared_kv ? 2 * H : 0, gpart, gates, dgate);
   return cudaGetLastError();
 }
 

@@ -23,6 +23,7 @@ cudaError_t launch_gemm_simt(const GemmArgs& g, cudaStream_t s);
 
 struct SwaShape {
   int B, T, H, hd, W, pos0, inject, dtype;
+  int vg;  // row of the value's first gate logit: 2 ([4, H] logits) or 0 (shared K/V gates, [2, H])
   double log2_base;
   float eps;
 };
@@ -56,7 +57,8 @@ cudaError_t launch_unmix(const SwaShape& s, const void* dk_bar, const void* dv_b
                          const float* gates, void* dk, void* dv, void* dRk, void* dRv,
                          float* accRk, float* accRv, int dr_mode, float* gpart,
                          const float* dq_acc, void* dq, cudaStream_t st);
-cudaError_t launch_gate_reduce(int64_t rows, int H, const float* gpart, const float* gates,
+// dgate [4, H] (or [2, H] when shared_kv) from the per-row partials.
+cudaError_t launch_gate_reduce(int64_t rows, int H, int shared_kv, const float* gpart, const float* gates,
                                float* dgate, cudaStream_t st);
 
 int loss_partial_blocks(int64_t n);
@@ -75,6 +77,7 @@ cudaError_t launch_consistency_loss(const void* m, const void* mt, int64_t rows,
 
 struct DecShape {
   int B, H, hd, W, inject, dtype;
+  int vg;  // as in SwaShape
   double log2_base;
   float eps;
 };
@@ -94,6 +97,11 @@ cudaError_t launch_proj_fwd_tc(int64_t M, int D, int d, const void* m_shift, con
 cudaError_t launch_proj_bwd_dm_tc(int64_t M, int D, int d, const void* dRk, const void* dRv,
                                   const void* w_mk, const void* w_mv, void* dm, int64_t spin_limit,
                                   int* err, cudaStream_t s);
+// dm [M, d] = sum over L layer-strided slabs of dR_k^l W_mk^l + dR_v^l W_mv^l
+// (dR [L][M][D], W [L][D][d]). Needs d % 8 == 0, D % 64 == 0.
+cudaError_t launch_proj_bwd_dm_layers_tc(int64_t M, int D, int d, int L, const void* dRk, const void* dRv,
+                                         const void* w_mk, const void* w_mv, void* dm, int64_t spin_limit,
+                                         int* err, cudaStream_t s);
 // dW_mk | dW_mv [D, d] = dR^T m_shift. Needs d % 8 == 0, D % 128 == 0.
 cudaError_t launch_proj_bwd_dw_tc(int64_t M, int D, int d, const void* dRk, const void* dRv,
                                   const void* m_shift, void* dwk, void* dwv, int64_t spin_limit,
@@ -110,6 +118,12 @@ cudaError_t launch_attn_bwd_tc(const SwaShape& s, const void* q_rot, const void*
 // tcgen05 banded attention forward on the saved bf16 q_rot / k_bar / v_bar.
 cudaError_t launch_attn_fwd_tc(const SwaShape& s, const void* q_rot, const void* k_bar, const void* v_bar,
                                void* out, float* lse, int64_t spin_limit, int* err, cudaStream_t st);
+
+// Copies k_bar, v_bar [B,T,H,hd] of the last min(T, W) positions into the
+// rings [B,H,W,hd], position pos0 + t to slot (pos0 + t) mod W.
+cudaError_t launch_ring_prefill(int B, int T, int H, int hd, int elt_bytes, int64_t W, int64_t pos0,
+                                const void* k_bar, const void* v_bar, void* k_ring, void* v_ring,
+                                cudaStream_t st);
 
 // Default bound of one in-kernel wait, in microseconds of GPU time (1 s).
 constexpr int64_t DEFAULT_SPIN_LIMIT = 1000000;

@@ -374,16 +374,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // ranked by decreasing cost and dealt in a snake order. A unit visits the
 // 64-query half-tiles that see its keys (at most 10 for W = 512); g counts
 // half-tiles over all of the CTA's units.
-//   S^T_g  = K Q_g^T, dP^T_g = V dO_g^T   128 keys x 64 queries, TMEM S[g&1], DP[g&1]
+//   S^T_g  = K Q_g^T, dP^T_g = V dO_g^T   128 keys x 64 queries, TMEM S, DP (one each)
 //   P^T_g, dS^T_g                          bf16, shared memory buffer g&1
 //   dV += P^T_g dO_g, dK += dS^T_g Q_g     TMEM accumulators (whole unit)
-//   dQ^T_g = K^T dS^T_g                    128 channels x 64 queries, into S[g&1]
-// The MMA warp issues S/dP of half-tile g+1 before dV/dK/dQ of g, so the
-// tensor core works on g+1 while the softmax warps work on g. The softmax
-// warps drain dQ^T_{g-1} right after producing P/dS of g: TMEM -> registers
-// (S[(g-1)&1] released at once) -> 4 KiB slices of the free P^T/dS^T buffer
-// (g-1)&1 -> one 32 x 32 fp32 TMA reduce-add per warp. Q/dO arrive through
-// a 3-deep ring; K/V once per unit.
+//   dQ^T_g = K^T dS^T_g                    128 channels x 64 queries, TMEM DQ[g&1]
+// The softmax warps release S / dP as soon as their tcgen05.ld of half-tile g
+// has completed, so the MMA warp issues S/dP of g+1 at once and the tensor
+// core computes it (and then dV/dK/dQ of g) while the softmax warps turn g's
+// scores into P and dS. After storing P/dS of g the softmax warps drain
+// dQ^T_{g-1} from its own TMEM columns: TMEM -> registers (DQ[(g-1)&1]
+// released at once) -> 4 KiB slices of the free P^T/dS^T buffer (g-1)&1 ->
+// one 32 x 32 fp32 TMA reduce-add per warp. Q/dO arrive through a 3-deep
+// ring; K/V once per unit.
 __device__ __forceinline__ void store_half_row(uint8_t* tile, int r, const float* x, int half) {
   // 32 values (columns 32*half .. +31) of row r of a [rows x 64] bf16 tile in
   // 128B-swizzled K-major layout (one 64-column chunk, 128 B per row).
@@ -418,7 +420,8 @@ struct PipeCfg {
   static constexpr int OFF_LD = OFF_DS + 2 * PH;  // [2][128] floats: LSE*log2e (64), Delta (64)
   static constexpr int OFF_BAR = OFF_LD + 2 * 128 * 4;
   static constexpr size_t SMEM = OFF_BAR + 256;   // base is 1024-aligned (checked in the kernel)
-  static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 384;  // S/dP: 64 columns x 2
+  // TMEM columns: S 64, dP 64, dQ 2 x 64, dV 128, dK 128
+  static constexpr uint32_t T_S = 0, T_DP = 64, T_DQ = 128, T_DV = 256, T_DK = 384;
 };
 
 struct PipeParams {
@@ -466,7 +469,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* kv_empty = bars + 1;
   uint64_t* q_full = bars + 2;     // [3]
   uint64_t* q_empty = bars + 5;    // [3]
-  uint64_t* s_full = bars + 8;     // [2]
+  uint64_t* s_full = bars + 8;     // S / dP of the current half-tile computed
+  uint64_t* s_free = bars + 9;     // ... and loaded by every softmax thread
   uint64_t* p_full = bars + 10;    // [2]
   uint64_t* dq_full = bars + 12;   // [2]
   uint64_t* dq_empty = bars + 14;  // [2]
@@ -486,8 +490,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
     }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, SOFT_THREADS);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], SOFT_THREADS);
       mbar_init(&dq_full[s], 1);
       mbar_init(&dq_empty[s], SOFT_THREADS);
@@ -561,79 +566,82 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       constexpr uint32_t ID_DQ = idesc_bf16(HD, 64, true, true);    // dQ^T: hd x 64 queries
       const uint32_t k_addr = smem_u32(smem + C::OFF_K);
       const uint32_t v_addr = smem_u32(smem + C::OFF_V);
-      // S^T_gs, dP^T_gs into buffer gs&1, once that buffer's dQ^T_{gs-2} is drained
+      // S^T_gs, dP^T_gs, once Q/dO have arrived and the softmax warps have
+      // loaded S/dP of half-tile gs-1
       auto issue_sdp = [&](int gs) -> bool {
-        const int s = gs % 3, buf = gs & 1;
+        const int s = gs % 3;
         if (!mbar_wait(&q_full[s], (uint32_t)(gs / 3) & 1u, ab)) return false;
-        if (gs >= 2 && !mbar_wait(&dq_empty[buf], (uint32_t)((gs - 2) >> 1) & 1u, ab)) return false;
+        if (gs >= 1 && !mbar_wait(s_free, (uint32_t)(gs - 1) & 1u, ab)) return false;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(smem + C::OFF_Q + s * C::QH);
         const uint32_t do_addr = smem_u32(smem + C::OFF_DO + s * C::QH);
 #pragma unroll
         for (int k16 = 0; k16 < HD / 16; ++k16) {
           const uint32_t ka = (uint32_t)(k16 >> 2) * C::KCHUNK, qa = (uint32_t)(k16 >> 2) * C::QCHUNK;
-          mma_ss(tmem + C::T_S + 64u * buf, kmajor_desc(k_addr + ka, k16 & 3), kmajor_desc(q_addr + qa, k16 & 3),
-                 ID_S, k16 > 0 ? 1u : 0u);
+          mma_ss(tmem + C::T_S, kmajor_desc(k_addr + ka, k16 & 3), kmajor_desc(q_addr + qa, k16 & 3), ID_S,
+                 k16 > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int k16 = 0; k16 < HD / 16; ++k16) {
           const uint32_t ka = (uint32_t)(k16 >> 2) * C::KCHUNK, qa = (uint32_t)(k16 >> 2) * C::QCHUNK;
-          mma_ss(tmem + C::T_DP + 64u * buf, kmajor_desc(v_addr + ka, k16 & 3), kmajor_desc(do_addr + qa, k16 & 3),
-                 ID_S, k16 > 0 ? 1u : 0u);
+          mma_ss(tmem + C::T_DP, kmajor_desc(v_addr + ka, k16 & 3), kmajor_desc(do_addr + qa, k16 & 3), ID_S,
+                 k16 > 0 ? 1u : 0u);
         }
-        mma_commit(&s_full[buf]);
+        mma_commit(s_full);
+        return true;
+      };
+      // dV, dK and dQ^T of half-tile gr (local index jr of unit nr), once the
+      // softmax warps have stored its P / dS
+      auto issue_rest = [&](int gr, int jr, int nr) -> bool {
+        const int s = gr % 3, buf = gr & 1;
+        if (!mbar_wait(&p_full[buf], (uint32_t)(gr >> 1) & 1u, ab)) return false;
+        // the first dV/dK of a unit overwrites the accumulators: the previous
+        // unit's epilogue must have read them
+        if (jr == 0 && !mbar_wait(acc_empty, ((uint32_t)nr & 1u) ^ 1u, ab)) return false;
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(smem + C::OFF_Q + s * C::QH);
+        const uint32_t do_addr = smem_u32(smem + C::OFF_DO + s * C::QH);
+        const uint32_t p_addr = smem_u32(smem + C::OFF_P + buf * C::PH);
+        const uint32_t ds_addr = smem_u32(smem + C::OFF_DS + buf * C::PH);
+#pragma unroll
+        for (int k16 = 0; k16 < 4; ++k16) {  // K = 64 queries
+          mma_ss(tmem + C::T_DV, kmajor_desc(p_addr, k16),
+                 sw128_desc(do_addr + (uint32_t)k16 * 2048u, (uint32_t)C::QCHUNK, 1024u), ID_KV,
+                 (jr > 0 || k16 > 0) ? 1u : 0u);
+        }
+#pragma unroll
+        for (int k16 = 0; k16 < 4; ++k16) {
+          mma_ss(tmem + C::T_DK, kmajor_desc(ds_addr, k16),
+                 sw128_desc(q_addr + (uint32_t)k16 * 2048u, (uint32_t)C::QCHUNK, 1024u), ID_KV,
+                 (jr > 0 || k16 > 0) ? 1u : 0u);
+        }
+        mma_commit(&q_empty[s]);
+        // DQ[buf] held dQ^T of half-tile gr-2: drained by now in practice
+        if (gr >= 2 && !mbar_wait(&dq_empty[buf], (uint32_t)((gr - 2) >> 1) & 1u, ab)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int k16 = 0; k16 < 8; ++k16) {  // K = 128 keys
+          mma_ss(tmem + C::T_DQ + 64u * buf, sw128_desc(k_addr + (uint32_t)k16 * 2048u, (uint32_t)C::KCHUNK, 1024u),
+                 sw128_desc(ds_addr + (uint32_t)k16 * 2048u, (uint32_t)C::PH, 1024u), ID_DQ, k16 > 0 ? 1u : 0u);
+        }
+        mma_commit(&dq_full[buf]);
         return true;
       };
       int g = 0, n = 0;
       bool ok = true;
       for (int u = kunit_rank(pp, 0); u >= 0 && ok; u = kunit_rank(pp, ++n)) {
         const KUnit x = kunit_of(pp, u);
-        if (!mbar_wait(kv_full, (uint32_t)n & 1u, ab) || !issue_sdp(g)) break;
+        if (!mbar_wait(kv_full, (uint32_t)n & 1u, ab)) break;
+        // S/dP of g+1 go to the tensor core ahead of dV/dK/dQ of g
         for (int j = 0; j < x.nh; ++j, ++g) {
-          if (j + 1 < x.nh && !issue_sdp(g + 1)) {
+          if (!issue_sdp(g) || (j > 0 && !issue_rest(g - 1, j - 1, n))) {
             ok = false;
             break;
-          }
-          const int s = g % 3, buf = g & 1;
-          if (!mbar_wait(&p_full[buf], (uint32_t)(g >> 1) & 1u, ab)) {
-            ok = false;
-            break;
-          }
-          // the first dV/dK of a unit overwrites the accumulators: the previous
-          // unit's epilogue must have read them
-          if (j == 0 && !mbar_wait(acc_empty, ((uint32_t)n & 1u) ^ 1u, ab)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t q_addr = smem_u32(smem + C::OFF_Q + s * C::QH);
-          const uint32_t do_addr = smem_u32(smem + C::OFF_DO + s * C::QH);
-          const uint32_t p_addr = smem_u32(smem + C::OFF_P + buf * C::PH);
-          const uint32_t ds_addr = smem_u32(smem + C::OFF_DS + buf * C::PH);
-#pragma unroll
-          for (int k16 = 0; k16 < 4; ++k16) {  // K = 64 queries
-            mma_ss(tmem + C::T_DV, kmajor_desc(p_addr, k16),
-                   sw128_desc(do_addr + (uint32_t)k16 * 2048u, (uint32_t)C::QCHUNK, 1024u), ID_KV,
-                   (j > 0 || k16 > 0) ? 1u : 0u);
-          }
-#pragma unroll
-          for (int k16 = 0; k16 < 4; ++k16) {
-            mma_ss(tmem + C::T_DK, kmajor_desc(ds_addr, k16),
-                   sw128_desc(q_addr + (uint32_t)k16 * 2048u, (uint32_t)C::QCHUNK, 1024u), ID_KV,
-                   (j > 0 || k16 > 0) ? 1u : 0u);
-          }
-          mma_commit(&q_empty[s]);
-#pragma unroll
-          for (int k16 = 0; k16 < 8; ++k16) {  // K = 128 keys
-            mma_ss(tmem + C::T_S + 64u * buf, sw128_desc(k_addr + (uint32_t)k16 * 2048u, (uint32_t)C::KCHUNK, 1024u),
-                   sw128_desc(ds_addr + (uint32_t)k16 * 2048u, (uint32_t)C::PH, 1024u), ID_DQ, k16 > 0 ? 1u : 0u);
-          }
-          mma_commit(&dq_full[buf]);
-          if (j + 1 == x.nh) {
-            mma_commit(acc_full);
-            mma_commit(kv_empty);
           }
         }
+        if (!ok || !issue_rest(g - 1, x.nh - 1, n)) break;
+        mma_commit(acc_full);
+        mma_commit(kv_empty);  // the next unit's K/V may overwrite this one's
       }
       mma_commit(drain);
       mbar_drain(drain, 0, DRAIN_LIMIT_NS);
@@ -664,10 +672,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) return;
       tc_fence_after();
       uint32_t v[32];
-      tmem_ld32(tmem + lane_off + C::T_S + 64u * (uint32_t)buf + 32u * (uint32_t)half, v);
+      tmem_ld32(tmem + lane_off + C::T_DQ + 64u * (uint32_t)buf + 32u * (uint32_t)half, v);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(&dq_empty[buf]);  // S[buf] may take S^T of half-tile gd + 2
+      mbar_arrive(&dq_empty[buf]);  // DQ[buf] may take dQ^T of half-tile gd + 2
       // box of 32 query rows x 32 channels (128 B rows, 16-byte chunks swizzled by row)
       const int w8 = q4 + 4 * half;
       uint8_t* slice = smem + (w8 < 4 ? C::OFF_P : C::OFF_DS) + buf * C::PH + (w8 & 3) * 4096;
@@ -708,13 +716,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int un = kunit_rank(pp, n + 1);
           if (un >= 0) fetch(kunit_of(pp, un), 0);
         }
-        ok = ok && warp_wait(&s_full[buf], (uint32_t)(g >> 1) & 1u, ab);
+        ok = ok && warp_wait(s_full, (uint32_t)g & 1u, ab);
         if (ok) {
           tc_fence_after();
           uint32_t sv[32], dv[32];
-          tmem_ld32(tmem + lane_off + C::T_S + 64u * buf + 32u * half, sv);
-          tmem_ld32(tmem + lane_off + C::T_DP + 64u * buf + 32u * half, dv);
+          tmem_ld32(tmem + lane_off + C::T_S + 32u * half, sv);
+          tmem_ld32(tmem + lane_off + C::T_DP + 32u * half, dv);
           tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(s_free);  // S / dP may take half-tile g + 1
           const int q0 = qt + 32 * half;  // first query column of this warp
           const int lo = kj - q0;         // query >= key
           const int hi = min(kj + p.W - 1, p.T - 1) - q0;

@@ -5,6 +5,10 @@
 //   forward  R = m_shift [B*T, d] x [W_mk; W_mv]^T           -> R_k | R_v
 //   backward dm = [dR_k | dR_v] x [W_mk; W_mv]                (K = 2D)
 //            dW = [dR_k | dR_v]^T x m_shift                   (M = 2D)
+//   per-layer projection (one W^rec per decoder layer, paper.rainbus.top,
+//   未来方向: 逐层记忆投影): dm = sum over layers l of [dR_k^l | dR_v^l] x
+//   [W_mk^l; W_mv^l], one GEMM with K = 2 L D over layer-strided operands
+//   (3-D tensor maps), so the sum over layers accumulates in fp32 in TMEM.
 //
 // One CTA per SM, 6 warps: warp 0 issues TMA loads of 64-wide K blocks into a
 // ring of 128B-swizzled shared-memory stages, warp 1 issues tcgen05.mma
@@ -33,6 +37,7 @@ struct TcGemmParams {
   int a_switch_m, a_switch_k;  // rows / K index where operand A moves to map 1
   int b_switch_n, b_switch_k;
   int out_switch_m, out_switch_n;
+  int k_layers;  // > 0: A is [k_layers][M][a_switch_k], B [k_layers][a_switch_k][N] (3-D maps), K = 2 L a_switch_k
   void* out0;
   void* out1;
   int64_t ldo;
@@ -121,6 +126,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           const int k0 = kb * BK;
+          if constexpr (!A_MN && B_MN) {
+            if (p.k_layers > 0) {  // layer-strided K: (k or v, layer l, k within the layer)
+              const int LD = p.k_layers * p.a_switch_k;
+              const int which = k0 >= LD ? 1 : 0;
+              const int kr = k0 - which * LD;
+              const int l = kr / p.a_switch_k, kk = kr - l * p.a_switch_k;
+              tma_load_3d(sA + stage * C::A_BYTES, which ? &tmA1 : &tmA0, &full[stage], kk, m0, l);
+              uint8_t* dstb = sB + stage * C::B_BYTES;
+#pragma unroll
+              for (int j = 0; j < BN / 64; ++j)
+                tma_load_3d(dstb + j * 8192, which ? &tmB1 : &tmB0, &full[stage], n0 + 64 * j, kk, l);
+              if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1;
+              }
+              continue;
+            }
+          }
           // operand A
           {
             const bool second = (p.a_switch_m > 0 && m0 >= p.a_switch_m) || (p.a_switch_k > 0 && k0 >= p.a_switch_k);
@@ -300,6 +323,27 @@ cudaError_t make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, 
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// bf16 [outer][mid][inner] tensor, 128B swizzle, box {box_inner, box_mid, 1}.
+cudaError_t make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+                              uint32_t box_inner, uint32_t box_mid) {
+  std::call_once(g_encode_once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  if (!g_encode) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {inner, mid, outer};
+  const cuuint64_t strides[2] = {inner * 2, inner * mid * 2};
+  const cuuint32_t box[3] = {box_inner, box_mid, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t make_tmap_tokens(CUtensorMap* m, const void* base, int B, int T, int H, int hd, uint32_t box_rows) {
   std::call_once(g_encode_once, [] {
     cudaDriverEntryPointQueryResult q;
@@ -435,6 +479,35 @@ cudaError_t launch_proj_bwd_dm_tc(int64_t M, int D, int d, const void* dRk, cons
   p.tiles_n = (d + BN - 1) / BN;
   p.a_switch_k = D;
   p.b_switch_k = D;
+  p.out0 = dm;
+  p.out1 = dm;
+  p.ldo = d;
+  p.spin_limit = spin_limit;
+  p.err = err;
+  return run_gemm<BN, false, true>(a0, a1, b0, b1, p, s);
+}
+
+// dm [M, d] = sum over L layers of dR_k^l [M, D] W_mk^l [D, d] + dR_v^l W_mv^l, with
+// dR [L][M][D] and W [L][D][d] layer-strided (K = 2 L D, one fp32 accumulation).
+cudaError_t launch_proj_bwd_dm_layers_tc(int64_t M, int D, int d, int L, const void* dRk, const void* dRv,
+                                         const void* w_mk, const void* w_mv, void* dm, int64_t spin_limit,
+                                         int* err, cudaStream_t s) {
+  constexpr int BN = 256;
+  CUtensorMap a0, a1, b0, b1;
+  cudaError_t e;
+  if ((e = make_tmap_bf16_3d(&a0, dRk, D, M, L, 64, BM)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_3d(&a1, dRv, D, M, L, 64, BM)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_3d(&b0, w_mk, d, D, L, 64, 64)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_3d(&b1, w_mv, d, D, L, 64, 64)) != cudaSuccess) return e;
+  TcGemmParams p{};
+  p.M = (int)M;
+  p.N = d;
+  p.K = 2 * L * D;
+  p.tiles_m = (int)((M + BM - 1) / BM);
+  p.tiles_n = (d + BN - 1) / BN;
+  p.a_switch_k = D;
+  p.b_switch_k = D;
+  p.k_layers = L;
   p.out0 = dm;
   p.out1 = dm;
   p.ldo = d;

@@ -22,13 +22,13 @@ def _bytes(n: int, device) -> torch.Tensor:
 
 class InjectedSWALayer:
     def __init__(self, B, T, H, hd, d_mem, window, dtype="bf16", inject=True, pos0=0,
-                 rope_base=10000.0, eps=1e-6, device="cuda", spin_limit=0):
+                 rope_base=10000.0, eps=1e-6, device="cuda", spin_limit=0, shared_kv_gates=False):
         self.shape = (B, T, H, hd)
         self.d_mem, self.dtype, self.device = d_mem, dtype, device
         self.inject = bool(inject)
         self.desc = SwaDesc(B=B, T=T, H=H, hd=hd, d_mem=d_mem, window=window, rope_base=rope_base,
                             rms_eps=eps, inject=int(inject), pos0=pos0, dtype=CODE[dtype],
-                            spin_limit=spin_limit)
+                            spin_limit=spin_limit, shared_kv_gates=int(shared_kv_gates))
         td = TORCH_DTYPE[dtype]
         D = H * hd
         self.out = torch.empty(B, T, H, hd, dtype=td, device=device)
@@ -42,7 +42,8 @@ class InjectedSWALayer:
         self.dv = torch.empty_like(self.dq)
         self.dR_k = torch.empty(B, T, D, dtype=td, device=device) if inject else None
         self.dR_v = torch.empty(B, T, D, dtype=td, device=device) if inject else None
-        self.dgate = torch.empty(4, H, dtype=torch.float32, device=device) if inject else None
+        self.dgate = torch.empty(2 if shared_kv_gates else 4, H, dtype=torch.float32,
+                                 device=device) if inject else None
         self.dm_shift = torch.empty(B, T, d_mem, dtype=td, device=device) if inject else None
         self.dw_mk = torch.empty(D, d_mem, dtype=td, device=device) if inject else None
         self.dw_mv = torch.empty(D, d_mem, dtype=td, device=device) if inject else None
@@ -76,9 +77,10 @@ class DecodeLayerState:
     """Buffers of one decode step of one layer (rings are caller tensors)."""
 
     def __init__(self, B, H, hd, d_mem, window, dtype="bf16", inject=True, rope_base=10000.0,
-                 eps=1e-6, device="cuda"):
+                 eps=1e-6, device="cuda", shared_kv_gates=False):
         self.desc = DecodeDesc(B=B, H=H, hd=hd, d_mem=d_mem, window=window, rope_base=rope_base,
-                               rms_eps=eps, inject=int(inject), dtype=CODE[dtype], spin_limit=0)
+                               rms_eps=eps, inject=int(inject), dtype=CODE[dtype], spin_limit=0,
+                               shared_kv_gates=int(shared_kv_gates))
         td = TORCH_DTYPE[dtype]
         self.krec = torch.empty(B, H, hd, dtype=td, device=device)
         self.vrec = torch.empty(B, H, hd, dtype=td, device=device)

@@ -138,11 +138,13 @@ def layer_inputs(wl: dict, seed: int, layer: int = 0, inject: bool = True) -> di
     return out
 
 
-def stack_inputs(wl: dict, seed: int, q_windows, p_windows) -> dict:
+def stack_inputs(wl: dict, seed: int, q_windows, p_windows, per_layer_wrec: bool = False,
+                 shared_kv_gates: bool = False) -> dict:
     """Seeded inputs of a prefiller Q (no injection) and a decoder P sharing a
     memory: per layer q, k, v, dout ~ N(0,1) [B,T,H,hd]; P's gate logits
-    ~ U[-2,2]; W_mk, W_mv [D,D] ~ N(0,1/D). P's layer l draws with layer index
-    l, Q's layer l with index 32 + l."""
+    ~ U[-2,2] ([4,H], or [2,H] with shared_kv_gates); W_mk, W_mv [D,D]
+    ~ N(0,1/D), and with per_layer_wrec one more pair per P layer (in its layer
+    dict). P's layer l draws with layer index l, Q's layer l with index 32 + l."""
     B, T, H, hd, dt = wl["B"], wl["T"], wl["H"], wl["hd"], wl["dtype"]
     D = H * hd
 
@@ -150,7 +152,10 @@ def stack_inputs(wl: dict, seed: int, q_windows, p_windows) -> dict:
         off = 64 * layer
         x = {k: normal(seed, TID[k] + off, (B, T, H, hd), dtype=dt) for k in ("q", "k", "v", "dout")}
         if gates:
-            x["gates"] = uniform(seed, TID["gates"] + off, (4, H), -2.0, 2.0)
+            x["gates"] = uniform(seed, TID["gates"] + off, (2 if shared_kv_gates else 4, H), -2.0, 2.0)
+            if per_layer_wrec:
+                x["w_mk"] = normal(seed, TID["w_mk"] + off, (D, D), std=1.0 / np.sqrt(D), dtype=dt, sub=1)
+                x["w_mv"] = normal(seed, TID["w_mv"] + off, (D, D), std=1.0 / np.sqrt(D), dtype=dt, sub=1)
         return x
 
     q_layers = [dict(one(32 + l, False), window=w) for l, w in enumerate(q_windows)]

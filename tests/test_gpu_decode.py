@@ -154,3 +154,45 @@ def test_decode_teacher_forced_checkpoints():
                 np.testing.assert_array_equal(got[:, :, keep], before[l][r][:, :, keep])
                 assert_close(got[:, :, slot], after[l][r][:, :, slot], "bf16", f"step {s} layer {l} slot")
         del before, after
+
+
+@pytest.mark.parametrize("T", [700, 300])
+def test_prefill_from_prompt_then_decode(T):
+    """Training-form forward over a T-token prompt, maglev_decode_prefill into
+    fresh rings, then one decode step at position T: its output must equal row
+    T of the oracle's (T+1)-row forward (recurrence = teacher forcing). T = 700
+    fills the whole ring (positions 188..699, slot 188 then takes position 700);
+    T = 300 fills slots 0..299 and must leave the others untouched."""
+    from sliding_window_recurrent_b200.layer import DecodeLayerState, InjectedSWALayer
+
+    Bq, Hq = 2, 10
+    wl = dict(synth.WORKLOADS["layer_bf16"])
+    wl.update(B=Bq, T=T + 1, H=Hq)
+    x = synth.layer_inputs(wl, 51)
+    rows = lambda t, a, b: synth.Tensor(np.ascontiguousarray(t.bits[:, a:b]), t.dtype)
+    Lyr = InjectedSWALayer(Bq, T, Hq, HD, D, W, dtype="bf16")
+    Lyr.forward(dev(rows(x["q"], 0, T)), dev(rows(x["k"], 0, T)), dev(rows(x["v"], 0, T)), dev(x["gates"]),
+                dev(rows(x["m_shift"], 0, T)), dev(x["w_mk"]), dev(x["w_mv"]))
+    fill = 9.0
+    kr = torch.full((Bq, Hq, W, HD), fill, dtype=torch.bfloat16, device="cuda")
+    vr = torch.full_like(kr, fill)
+    mg.maglev_decode_prefill(Lyr.desc, Lyr.saved, kr, vr)
+    torch.cuda.synchronize()
+
+    Rk, Rv = oracle.mem_project(x["m_shift"].f64, x["w_mk"].f64, x["w_mv"].f64)
+    f = oracle.inject_swa_forward(x["q"].f64, x["k"].f64, x["v"].f64, Rk, Rv, x["gates"].astype(np.float64), W)
+    live = list(range(max(0, T - W), T))
+    slots = [j % W for j in live]
+    got_k, got_v = host(kr), host(vr)
+    assert_close(got_k[:, :, slots], f["k_bar"][:, live].transpose(0, 2, 1, 3), "bf16", "prefilled k")
+    assert_close(got_v[:, :, slots], f["v_bar"][:, live].transpose(0, 2, 1, 3), "bf16", "prefilled v")
+    dead = sorted(set(range(W)) - set(slots))
+    assert np.all(got_k[:, :, dead] == fill) and np.all(got_v[:, :, dead] == fill)
+
+    S = DecodeLayerState(Bq, Hq, HD, D, W, dtype="bf16")
+    pos_t = torch.full((Bq,), T, dtype=torch.int64, device="cuda")
+    S.mem_project(pos_t, dev(rows(x["m_shift"], T, T + 1)).view(Bq, D), dev(x["w_mk"]), dev(x["w_mv"]))
+    o = S.step(pos_t, *(dev(rows(x[n], T, T + 1)).view(Bq, Hq, HD) for n in ("q", "k", "v")), dev(x["gates"]),
+               kr, vr)
+    torch.cuda.synchronize()
+    assert_close(host(o), f["out"][:, T], "bf16", f"decode at {T} after prefill")

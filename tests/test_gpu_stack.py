@@ -28,29 +28,35 @@ def _zero_last_dout(x):
         L["dout"] = synth.Tensor(np.zeros_like(L["dout"].bits), L["dout"].dtype)
 
 
-def _run(wl, seed, q_windows, p_windows, zero_last_dout=False):
+def _run(wl, seed, q_windows, p_windows, zero_last_dout=False, per_layer_wrec=False, shared_kv_gates=False):
     import torch
     from sliding_window_recurrent_b200.stack import PrefillerDecoderStack
 
-    x = synth.stack_inputs(wl, seed, q_windows, p_windows)
+    x = synth.stack_inputs(wl, seed, q_windows, p_windows, per_layer_wrec, shared_kv_gates)
     if zero_last_dout:
         _zero_last_dout(x)
     B, T, H, hd = wl["B"], wl["T"], wl["H"], wl["hd"]
-    S = PrefillerDecoderStack(B, T, H, hd, q_windows, p_windows, lam=wl["lam"], dtype=wl["dtype"])
+    S = PrefillerDecoderStack(B, T, H, hd, q_windows, p_windows, lam=wl["lam"], dtype=wl["dtype"],
+                              per_layer_wrec=per_layer_wrec, shared_kv_gates=shared_kv_gates)
     qi = [(dev(L["q"]), dev(L["k"]), dev(L["v"])) for L in x["q_layers"]]
     pi = [(dev(L["q"]), dev(L["k"]), dev(L["v"]), dev(L["gates"])) for L in x["p_layers"]]
     qd = [dev(L["dout"]) for L in x["q_layers"]]
     pd = [dev(L["dout"]) for L in x["p_layers"]]
-    wk, wv = dev(x["w_mk"]), dev(x["w_mv"])
+    if per_layer_wrec:
+        wk = torch.stack([dev(L["w_mk"]) for L in x["p_layers"]])
+        wv = torch.stack([dev(L["w_mv"]) for L in x["p_layers"]])
+    else:
+        wk, wv = dev(x["w_mk"]), dev(x["w_mv"])
     S.step(qi, pi, qd, pd, wk, wv)
     torch.cuda.synchronize()
 
     f64 = lambda L, keys: {k: (L[k].f64 if isinstance(L[k], synth.Tensor) else L[k]) for k in keys}
     ql = [dict(f64(L, ("q", "k", "v", "dout")), window=L["window"]) for L in x["q_layers"]]
-    pl = [dict(f64(L, ("q", "k", "v", "dout")), gates=L["gates"].astype(np.float64), window=L["window"])
-          for L in x["p_layers"]]
+    pkeys = ("q", "k", "v", "dout") + (("w_mk", "w_mv") if per_layer_wrec else ())
+    pl = [dict(f64(L, pkeys), gates=L["gates"].astype(np.float64), window=L["window"]) for L in x["p_layers"]]
     store = _bf16 if wl["dtype"] == "bf16" else None
-    ref = oracle.stack_forward_backward(ql, pl, x["w_mk"].f64, x["w_mv"].f64, wl["lam"], store=store)
+    w = (None, None) if per_layer_wrec else (x["w_mk"].f64, x["w_mv"].f64)
+    ref = oracle.stack_forward_backward(ql, pl, w[0], w[1], wl["lam"], store=store)
     return S, ref
 
 
@@ -70,11 +76,18 @@ def _check_all(S, ref, dt):
     assert np.all(host(S.m_shift)[:, 0] == 0), "row 0 of the shifted memory is m'_0 = 0"
     assert_close(host(S.m), ref["m"], dt, "m")
     assert abs(float(S.loss.item()) - ref["loss"]) <= TOL[dt] * abs(ref["loss"]), (float(S.loss.item()), ref["loss"])
-    assert_close(host(S.dR_k), ref["dR_k"], dt, "dR_k")
-    assert_close(host(S.dR_v), ref["dR_v"], dt, "dR_v")
     assert_close(host(S.dm_shift), ref["dm_shift"], dt, "dm_shift")
-    assert_close(host(S.dw_mk), ref["dw_mk"], dt, "dW_mk")
-    assert_close(host(S.dw_mv), ref["dw_mv"], dt, "dW_mv")
+    if S.per_layer_wrec:
+        for i, g in enumerate(ref["p_grads"]):
+            for n in ("dR_k", "dR_v"):
+                assert_close(host(getattr(S, n)[i]), g[n].reshape(B, T, -1), dt, f"P{i} {n}")
+            for n in ("dw_mk", "dw_mv"):
+                assert_close(host(getattr(S, n)[i]), g[n], dt, f"P{i} {n}")
+    else:
+        assert_close(host(S.dR_k), ref["dR_k"], dt, "dR_k")
+        assert_close(host(S.dR_v), ref["dR_v"], dt, "dR_v")
+        assert_close(host(S.dw_mk), ref["dw_mk"], dt, "dW_mk")
+        assert_close(host(S.dw_mv), ref["dw_mv"], dt, "dW_mv")
 
 
 @pytest.mark.parametrize("T", [200, 129])
@@ -100,6 +113,18 @@ def test_stack_loss_gradient_drives_last_layers(dtype):
     S, ref = _run(wl, 1237, [48, 150], [48, 48, 48], zero_last_dout=True)
     g = ref["p_grads"][-1]
     assert 0 < np.abs(g["dq"]).max() < 0.1, "P's last layer sees only the small loss gradient"
+    _check_all(S, ref, dtype)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("per_layer_wrec,shared_kv_gates", [(True, False), (False, True), (True, True)])
+def test_stack_variants(dtype, per_layer_wrec, shared_kv_gates):
+    """The decoder with one W^rec per layer (dm_shift summed over the layers'
+    projections in one fp32 accumulation) and/or gates shared by K and V."""
+    hd = 128 if dtype == "bf16" else 64
+    wl = dict(B=2, T=170, H=2, hd=hd, dtype=dtype, lam=0.5)
+    S, ref = _run(wl, 1239, [64, 170], [64, 64, 64], per_layer_wrec=per_layer_wrec,
+                  shared_kv_gates=shared_kv_gates)
     _check_all(S, ref, dtype)
 
 
