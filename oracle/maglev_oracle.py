@@ -262,6 +262,38 @@ def consistency_loss(m, m_target, lam: float, inv_count: float | None = None):
 
 
 # --------------------------------------------------------------------------
+# LM head with softcapped logits and cross-entropy
+# --------------------------------------------------------------------------
+def lm_head_ce(m, U, targets, softcap: float = 15.0, inv_count: float | None = None):
+    """Per-token next-token loss of the memory state (rainbus, 方法步骤详情):
+    p(x_{t+1} | x_<=t) = softmax(c_t), c_t = softcap * tanh(U m_t / softcap)
+    with softcap = 15, and the loss (1/|I|) sum_t CE_t with
+    CE_t = -log p(targets_t) = logsumexp(c_t) - c_t[targets_t].
+
+    m [N, d], U [V, d], targets [N] int. inv_count = 1/|I| (default 1/N).
+    Returns (loss, lse [N], dm [N, d], dU [V, d]): by the chain rule,
+    dL/dc_t = inv_count (softmax(c_t) - onehot(targets_t)) and
+    dc/dz = 1 - tanh(z / softcap)^2 for the raw logits z = U m_t.
+    """
+    N = m.shape[0]
+    if inv_count is None:
+        inv_count = 1.0 / N
+    z = m @ U.T                                        # [N, V] raw logits
+    t = np.tanh(z / softcap)
+    c = softcap * t
+    mx = c.max(axis=1, keepdims=True)
+    lse = (mx + np.log(np.sum(np.exp(c - mx), axis=1, keepdims=True)))[:, 0]
+    rows = np.arange(N)
+    ce = lse - c[rows, targets]
+    loss = inv_count * np.sum(ce)
+    dc = np.exp(c - lse[:, None])                      # softmax(c_t)
+    dc[rows, targets] -= 1.0
+    dc *= inv_count
+    dz = dc * (1.0 - t * t)
+    return loss, lse, dz @ U, dz.T @ m
+
+
+# --------------------------------------------------------------------------
 # stack: prefiller Q and decoder P around one shared memory
 # --------------------------------------------------------------------------
 def memory_state(o, eps: float = 1e-6):

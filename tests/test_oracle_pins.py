@@ -560,3 +560,76 @@ def test_synth_inputs_are_seeded_and_sliceable():
     x = np.array([1.0, 1.00390625, 1.005859375, -3.14159], dtype=np.float32)
     bits = synth.round_to_bf16_bits(x)
     np.testing.assert_array_equal(synth.bf16_bits_to_f64(bits), [1.0, 1.0, 1.0078125, -3.140625])
+
+
+# ---------------------------------------------------------------- LM head, softcapped CE
+def test_lm_head_zero_weights_give_log_vocab():
+    """U = 0: every logit is 0, the softmax is uniform and each token's CE is
+    log V exactly; dm is 0 and dU = -(1/N) sum_t (onehot - 1/V) m_t^T."""
+    N, d, V = 5, 8, 11
+    m = rand(N, d)
+    y = RNG.integers(0, V, N)
+    loss, lse, dm, dU = oracle.lm_head_ce(m, np.zeros((V, d)), y)
+    np.testing.assert_allclose(loss, np.log(V), rtol=1e-15)
+    np.testing.assert_allclose(lse, np.log(V), rtol=1e-15)
+    assert np.all(dm == 0)
+    oh = np.zeros((N, V))
+    oh[np.arange(N), y] = 1.0
+    np.testing.assert_allclose(dU, ((1.0 / V - oh) / N).T @ m, rtol=1e-13, atol=1e-15)
+
+
+def test_lm_head_softcap_limits():
+    """The cap bounds every logit: a huge raw logit saturates at +15 (its
+    probability then e^15 / (e^15 + (V-1) e^c_other)), and the cap's slope is
+    1 at 0 and vanishes in saturation."""
+    d, V = 4, 3
+    m = np.array([[1.0, 0, 0, 0]])
+    U = np.zeros((V, d))
+    U[0, 0] = 1e6                                     # z = (1e6, 0, 0)
+    loss, lse, _, dU = oracle.lm_head_ce(m, U, np.array([1]))
+    np.testing.assert_allclose(lse[0], np.log(np.exp(15.0) + 2.0), rtol=1e-14)
+    np.testing.assert_allclose(loss, lse[0] - 0.0, rtol=1e-14)
+    assert abs(dU[0, 0]) < 1e-300                     # tanh' = 0 in saturation
+    # small logits: softcap(z) = z to third order, so the CE matches the plain one
+    U2 = rand(V, d) * 1e-3
+    l_cap = oracle.lm_head_ce(m, U2, np.array([2]))[0]
+    z = (m @ U2.T)[0]
+    l_plain = np.log(np.sum(np.exp(z))) - z[2]
+    assert abs(l_cap - l_plain) < 1e-9
+
+
+def test_lm_head_matches_torch_cross_entropy_and_autograd():
+    """Loss against torch's cross_entropy of the softcapped logits, gradients
+    against autograd through matmul, tanh and cross_entropy (fp64)."""
+    N, d, V = 6, 10, 17
+    m, U = rand(N, d), rand(V, d)
+    y = RNG.integers(0, V, N)
+    loss, lse, dm, dU = oracle.lm_head_ce(m, U, y, inv_count=1.0 / 4)
+    tm = torch.from_numpy(m).requires_grad_(True)
+    tU = torch.from_numpy(U).requires_grad_(True)
+    c = 15.0 * torch.tanh((tm @ tU.T) / 15.0)
+    tl = F.cross_entropy(c, torch.from_numpy(y), reduction="sum") / 4
+    tl.backward()
+    np.testing.assert_allclose(loss, tl.item(), rtol=1e-13)
+    np.testing.assert_allclose(lse, torch.logsumexp(c, 1).detach().numpy(), rtol=1e-13)
+    np.testing.assert_allclose(dm, tm.grad.numpy(), rtol=1e-11, atol=1e-14)
+    np.testing.assert_allclose(dU, tU.grad.numpy(), rtol=1e-11, atol=1e-14)
+
+
+def test_lm_head_central_differences():
+    N, d, V = 4, 6, 9
+    m, U = rand(N, d) * 3, rand(V, d) * 3               # large enough for the cap to bend
+    y = RNG.integers(0, V, N)
+    _, _, dm, dU = oracle.lm_head_ce(m, U, y)
+    h = 1e-6
+    for arr, grad in ((m, dm), (U, dU)):
+        for _ in range(6):
+            idx = tuple(RNG.integers(0, s) for s in arr.shape)
+            a0 = arr[idx]
+            arr[idx] = a0 + h
+            lp = oracle.lm_head_ce(m, U, y)[0]
+            arr[idx] = a0 - h
+            lm = oracle.lm_head_ce(m, U, y)[0]
+            arr[idx] = a0
+            fd = (lp - lm) / (2 * h)
+            assert abs(fd - grad[idx]) <= 1e-7 * max(1.0, abs(fd)), (idx, fd, grad[idx])
