@@ -36,6 +36,9 @@ METRIC = "Injected-SWA attn fwd+bwd TFLOP/s & % bf16 peak; decode tokens/s"
 LAYER = dict(B=4, T=2048, H=10, hd=128, d=1280, W=512, lam=0.1)
 DECODE = dict(B=64, L=20, H=10, hd=128, d=1280, W=512, first_pos=512)
 STACK = dict(B=8, T=2048, H=10, hd=128, L=20, W=512, lam=0.1)
+# LM head over the memory states of the d20 layer's tokens; the pages give no
+# vocabulary size, 65,536 stands in
+LMHEAD = dict(N=8192, d=1280, V=65536, softcap=15.0)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # Datasheet dense peaks of one B200 (context beside the measured peaks).
@@ -527,6 +530,52 @@ def run_decode_bench(torch, dev, steps, warmup, peaks):
                         f"{c['first_pos']} (after {warmup + 3} warm-up steps), CUDA graph"}
 
 
+def run_lm_head_bench(torch, dev, steps, warmup, peaks):
+    """Softcapped LM head + CE, fwd+bwd: logits GEMM with the CE statistics in
+    its epilogue, the loss and dz, then dm = dz U and dU = dz^T m."""
+    import sliding_window_recurrent_b200 as mg
+    c = LMHEAD
+    N, d, V = c["N"], c["d"], c["V"]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(97)
+    bf = torch.bfloat16
+    m = torch.randn(N, d, generator=gen, device=dev).to(bf)
+    U = (torch.randn(V, d, generator=gen, device=dev) * (4.0 / d ** 0.5)).to(bf)
+    y = torch.randint(0, V, (N,), generator=gen, device=dev)
+    loss = torch.zeros((), device=dev)
+    lse = torch.empty(N, device=dev)
+    dm = torch.empty(N, d, dtype=bf, device=dev)
+    dU = torch.empty(V, d, dtype=bf, device=dev)
+    ws = torch.empty(mg.maglev_lm_head_workspace_bytes(N, d, V), dtype=torch.uint8, device=dev)
+    step = lambda: mg.maglev_lm_head_ce(N, d, V, mg.MAGLEV_BF16, c["softcap"], 0.0, m, U, y, loss, lse, dm, dU, ws)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    mg.maglev_profile_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    mg.maglev_profile_enable(False)
+    prof = aggregate_profile(mg.maglev_profile_report())
+    ms = e0.elapsed_time(e1) / steps
+    flops = 3 * 2.0 * N * d * V  # logits, dm, dU
+    kern = {n: {"calls": v[0], "ms_total": round(v[1], 4)} for n, v in prof.items()}
+    roof = None
+    if "lm_logits_ce_tc" in prof:
+        calls, tot, _ = prof["lm_logits_ce_tc"]
+        tf = 2.0 * N * d * V / (tot / calls * 1e-3) / 1e12
+        roof = {"kernel": "lm_logits_ce_tc", "bound": "tensor", "achieved": round(tf, 2),
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4)}
+    del ws
+    torch.cuda.empty_cache()
+    return {"value": round(flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
+            "gflop_per_step": round(flops / 1e9, 1), "roofline": roof, "kernels": kern,
+            "workload": f"softcapped LM head + CE fwd+bwd: N={N} tokens, d={d}, V={V}, softcap 15, bf16"}
+
+
 # --------------------------------------------------------------------------- oracle arm
 def oracle_sample_step(x, c):
     """The oracle's fwd + loss + bwd on a bounded sample of the layer workload:
@@ -630,6 +679,7 @@ def main():
     ap.add_argument("--stack-steps", type=int, default=5)
     ap.add_argument("--no-stack", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-lm-head", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -686,6 +736,10 @@ def main():
         dec = run_decode_bench(torch, dev, args.decode_steps, args.warmup, peaks)
         dec["tokens_per_s"] = job_rate(DECODE["B"], world, max_over_ranks(dist, dec["ms_per_step"], dev))
 
+    lmh = None
+    if not args.no_lm_head:
+        lmh = run_lm_head_bench(torch, dev, max(3, args.steps // 4), args.warmup, peaks)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline()
@@ -711,6 +765,7 @@ def main():
         "clocks": r["clocks"],
         "forward": fwd,
         "stack": stack,
+        "lm_head": lmh,
         "decode": None if dec is None else {
             "value": round(dec["tokens_per_s"], 1), "unit": "tokens/s", "ms_per_step": round(dec["ms_per_step"], 4),
             "workload": dec["workload"], "roofline": dec["roofline"], "kernels": dec["kernels"]},

@@ -272,6 +272,29 @@ maglev_status maglev_consistency_loss_noalloc(const void* m, const void* m_targe
                                               float* loss, void* dm, void* dm_target,
                                               int accumulate_dm, void* stream);
 
+/* Bytes of scratch memory maglev_lm_head_ce needs: the capped logits (fp32)
+ * and their gradient (bf16), N x V each, plus per-row statistics. */
+size_t maglev_lm_head_workspace_bytes(int64_t N, int d, int V);
+
+/* LM head with softcapped logits and cross-entropy ([rainbus] 方法步骤详情: the
+ * memory state m_t feeds p(x_{t+1} | x_<=t) = softmax(15 tanh(U m_t / 15)); the
+ * loss averages the per-token CE over the positions in I).
+ *   m [N, d] bf16: the memory states (rows = tokens); U [V, d] bf16.
+ *   targets [N] int64 (device): the next token of each row, in [0, V); a row
+ *     with a target outside that range gets a NaN CE (and so a NaN loss).
+ *   softcap: 15 in the pages' model. inv_count = 1/|I| (0 means 1/N).
+ *   loss: device fp32 scalar (out) = inv_count * sum_t (LSE_t - c_t[y_t]),
+ *     c = softcap * tanh(U m / softcap), reduced in a fixed order.
+ *   lse [N] fp32 (out): LSE_t of each row's capped logits.
+ *   dm [N, d], dU [V, d] bf16 (out, nullable): gradients of the loss.
+ *   workspace: maglev_lm_head_workspace_bytes(N, d, V) bytes.
+ *   spin_limit: bound on each in-kernel wait in microseconds (0 = 1 s).
+ * Errors: UNSUPPORTED unless dtype is MAGLEV_BF16 and d, V are multiples of 8. */
+maglev_status maglev_lm_head_ce(int64_t N, int d, int V, int dtype, float softcap, float inv_count,
+                                const void* m, const void* U, const int64_t* targets, float* loss,
+                                float* lse, void* dm, void* dU, void* workspace, int64_t spin_limit,
+                                void* stream);
+
 /* a8 -- decode-side memory projection, once per token step (W^rec is shared by
  * all layers and m_{p-1} is the same for all of them):
  *   pos [B] int64 (device): absolute position p of each sequence's new token.

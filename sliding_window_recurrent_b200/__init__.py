@@ -76,6 +76,8 @@ _SIGS = {
     "maglev_decode_mem_project": ([ctypes.POINTER(DecodeDesc)] + [_P] * 7, _I),
     "maglev_decode_step": ([ctypes.POINTER(DecodeDesc)] + [_P] * 11, _I),
     "maglev_decode_prefill": ([ctypes.POINTER(SwaDesc)] + [_P] * 4, _I),
+    "maglev_lm_head_workspace_bytes": ([_I64, _I, _I], _SZ),
+    "maglev_lm_head_ce": ([_I64, _I, _I, _I, _F, _F] + [_P] * 8 + [_I64, _P], _I),
 }
 
 
@@ -252,3 +254,14 @@ def maglev_decode_step(desc, pos, q, k, v, krec_rot, vrec, gate_logits, k_ring, 
 def maglev_decode_prefill(desc, saved, k_ring, v_ring, stream=None):
     _check(_lib.maglev_decode_prefill(ctypes.byref(desc), _ptr(saved), _ptr(k_ring), _ptr(v_ring),
                                       _stream(stream)))
+
+
+def maglev_lm_head_workspace_bytes(N: int, d: int, V: int) -> int:
+    return _lib.maglev_lm_head_workspace_bytes(int(N), int(d), int(V))
+
+
+def maglev_lm_head_ce(N, d, V, dtype, softcap, inv_count, m, U, targets, loss, lse, dm, dU, workspace,
+                      spin_limit=0, stream=None):
+    _check(_lib.maglev_lm_head_ce(int(N), int(d), int(V), int(dtype), float(softcap), float(inv_count), _ptr(m),
+                                  _ptr(U), _ptr(targets), _ptr(loss), _ptr(lse), _ptr(dm), _ptr(dU),
+                                  _ptr(workspace), int(spin_limit), _stream(stream)))

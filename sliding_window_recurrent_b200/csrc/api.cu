@@ -654,6 +654,67 @@ maglev_status maglev_consistency_loss(const void* m, const void* m_target, int64
   return MAGLEV_OK;
 }
 
+// Offsets inside the LM head's workspace.
+struct LmLayout {
+  size_t c, dz, part, tgt, ce, total;
+};
+LmLayout lm_layout(int64_t N, int V) {
+  LmLayout L;
+  L.c = 0;
+  L.dz = align256((size_t)N * V * 4);
+  L.part = L.dz + align256((size_t)N * V * 2);
+  L.tgt = L.part + align256((size_t)N * lm_ce_tiles(V) * 8);
+  L.ce = L.tgt + align256((size_t)N * 4);
+  L.total = L.ce + align256((size_t)N * 4);
+  return L;
+}
+
+size_t maglev_lm_head_workspace_bytes(int64_t N, int d, int V) {
+  if (N < 0 || d < 1 || V < 1) return 0;
+  return lm_layout(N, V).total;
+}
+
+maglev_status maglev_lm_head_ce(int64_t N, int d, int V, int dtype, float softcap, float inv_count,
+                                const void* m, const void* U, const int64_t* targets, float* loss, float* lse,
+                                void* dm, void* dU, void* workspace, int64_t spin_limit, void* stream) {
+  if (N < 0 || d < 1 || V < 1) return fail(MAGLEV_ERR_INVALID_ARG, "need N >= 0, d >= 1, V >= 1");
+  if (dtype != MAGLEV_BF16) return fail(MAGLEV_ERR_UNSUPPORTED, "the LM head runs in bf16 only");
+  if (d % 8 != 0 || V % 8 != 0) return fail(MAGLEV_ERR_UNSUPPORTED, "d and V must be multiples of 8");
+  if ((int64_t)V * N > ((int64_t)1 << 40)) return fail(MAGLEV_ERR_UNSUPPORTED, "N * V too large");
+  if (!(softcap > 0.0f) || !std::isfinite(softcap)) return fail(MAGLEV_ERR_INVALID_ARG, "softcap must be > 0");
+  if (!std::isfinite(inv_count) || inv_count < 0)
+    return fail(MAGLEV_ERR_INVALID_ARG, "inv_count must be finite and >= 0");
+  NEED_PTR(loss);
+  OPT_PTR(dm);
+  OPT_PTR(dU);
+  if (N == 0) return MAGLEV_OK;
+  NEED_PTR(m);
+  NEED_PTR(U);
+  NEED_PTR(targets);
+  NEED_PTR(lse);
+  NEED_PTR(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* err = nullptr;
+  maglev_status st = status_word(&err, s);
+  if (st != MAGLEV_OK) return st;
+  const LmLayout L = lm_layout(N, V);
+  const float ic = inv_count == 0.0f ? (float)(1.0 / (double)N) : inv_count;
+  const int64_t lim = spin_limit_of(spin_limit);
+  float* c = at<float>(workspace, L.c);
+  void* dz = (dm || dU) ? at<char>(workspace, L.dz) : nullptr;
+  float2* part = at<float2>(workspace, L.part);
+  float* tgt = at<float>(workspace, L.tgt);
+  float* ce = at<float>(workspace, L.ce);
+  MAGLEV_LAUNCH(1, s, launch_lm_logits_ce_tc(N, d, V, softcap, m, U, targets, c, part, tgt, lim, err, s),
+                "lm_logits_ce_tc");
+  MAGLEV_LAUNCH(dz ? 3 : 2, s, launch_lm_ce_finish(N, V, lm_ce_tiles(V), ic, softcap, part, tgt, targets, c, lse,
+                                                    ce, loss, dz, s),
+                "lm_ce_finish");
+  if (dm) MAGLEV_LAUNCH(1, s, launch_lm_dm_tc(N, d, V, dz, U, dm, lim, err, s), "lm_dm_tc");
+  if (dU) MAGLEV_LAUNCH(1, s, launch_lm_dU_tc(N, d, V, dz, m, dU, lim, err, s), "lm_dU_tc");
+  return MAGLEV_OK;
+}
+
 maglev_status maglev_memory_state(int B, int T, int d, float eps, int dtype, const void* o, void* m,
                                   void* m_shift, float* rstd, void* stream) {
   if (B < 0 || T < 0) return fail(MAGLEV_ERR_INVALID_ARG, "B and T must be >= 0");

@@ -125,6 +125,23 @@ cudaError_t launch_ring_prefill(int B, int T, int H, int hd, int elt_bytes, int6
                                 const void* k_bar, const void* v_bar, void* k_ring, void* v_ring,
                                 cudaStream_t st);
 
+// LM head with softcapped logits and cross-entropy (bf16 m [N,d], U [V,d]).
+// Capped logits c [N,V] fp32 with per-row, per-256-column (max, sum exp) in
+// part [N, lm_ce_tiles(V)] and the target's capped logit in tgt [N].
+cudaError_t launch_lm_logits_ce_tc(int64_t N, int d, int V, float softcap, const void* m, const void* U,
+                                   const int64_t* targets, float* c, float2* part, float* tgt,
+                                   int64_t spin_limit, int* err, cudaStream_t s);
+int lm_ce_tiles(int V);
+// lse [N], ce [N] per row, loss = inv_count * sum ce; dz [N,V] bf16 when non-null.
+cudaError_t launch_lm_ce_finish(int64_t N, int V, int tiles, float inv_count, float softcap, const float2* part,
+                                const float* tgt, const int64_t* targets, const float* c, float* lse, float* ce,
+                                float* loss, void* dz, cudaStream_t st);
+// dm [N,d] = dz U; dU [V,d] = dz^T m (bf16, fp32 accumulation).
+cudaError_t launch_lm_dm_tc(int64_t N, int d, int V, const void* dz, const void* U, void* dm, int64_t spin_limit,
+                            int* err, cudaStream_t s);
+cudaError_t launch_lm_dU_tc(int64_t N, int d, int V, const void* dz, const void* m, void* dU, int64_t spin_limit,
+                            int* err, cudaStream_t s);
+
 // Default bound of one in-kernel wait, in microseconds of GPU time (1 s).
 constexpr int64_t DEFAULT_SPIN_LIMIT = 1000000;
 

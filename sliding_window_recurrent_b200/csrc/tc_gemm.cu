@@ -38,6 +38,14 @@ struct TcGemmParams {
   int b_switch_n, b_switch_k;
   int out_switch_m, out_switch_n;
   int k_layers;  // > 0: A is [k_layers][M][a_switch_k], B [k_layers][a_switch_k][N] (3-D maps), K = 2 L a_switch_k
+  // softcapped cross-entropy epilogue (EPI_CE): out0 receives the capped
+  // logits c = softcap * tanh(z / softcap) in fp32; per row and N tile the
+  // (max, sum of exp(c - max)) pair goes to ce_part[row * tiles_n + tile], and
+  // the capped logit of the row's target to ce_tgt[row]
+  const int64_t* targets;
+  float softcap;
+  float2* ce_part;
+  float* ce_tgt;
   void* out0;
   void* out1;
   int64_t ldo;
@@ -58,7 +66,18 @@ struct Cfg {
   static constexpr size_t SMEM = 1024 + (size_t)OFF_EPI + 4 * 4096;
 };
 
-template <int BN, bool A_MN, bool B_MN>
+// Epilogues: bf16 store of the accumulator, or the softcapped cross-entropy
+// statistics with an fp32 store of the capped logits.
+constexpr int EPI_BF16 = 0, EPI_CE = 1;
+
+// softcap * tanh(z / softcap), with tanh(x) = 1 - 2 / (1 + e^{2x}) (exact at
+// +-inf: e^{2x} = inf gives 1, 0 gives -1; absolute error ~1e-7 near 0).
+__device__ __forceinline__ float softcap_of(float z, float cap, float two_log2e_over_cap) {
+  const float e = ex2_fast(z * two_log2e_over_cap);
+  return cap * (1.0f - 2.0f * __frcp_rn(1.0f + e));
+}
+
+template <int BN, bool A_MN, bool B_MN, int EPI = EPI_BF16>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                    const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
@@ -224,6 +243,72 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // all issued MMAs must finish before TMEM is released
       mma_commit(drain);
       mbar_drain(drain, 0, DRAIN_LIMIT_NS);
+    }
+  } else if constexpr (EPI == EPI_CE) {
+    // -------------------------------------------------------------- CE epilogue
+    // Thread = one row of the tile. 32 columns at a time: TMEM -> capped logits
+    // (running max / sum of exponentials of the row over the tile, target
+    // logit) -> the warp's 4 KiB of fp32 staging -> 128-byte row pieces.
+    constexpr float LOG2E_F = 1.4426950408889634f;
+    const float k2 = 2.0f * LOG2E_F / p.softcap;
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    uint8_t* stg = smem + C::OFF_EPI + q * 4096;
+    float* outc = static_cast<float*>(p.out0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      const int tm = t % p.tiles_m, tn = t / p.tiles_m;
+      const int m0 = tm * BM, n0 = tn * BN;
+      if (!warp_wait(&tfull[acc], acc_phase, ab)) break;
+      tc_fence_after();
+      const int gm = m0 + row;
+      const int64_t y = gm < p.M ? p.targets[gm] : -1;
+      float mx = -INFINITY, sm = 0.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::ACC_STRIDE + c0), r);
+        tmem_wait_ld();
+        float cmx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int col = n0 + c0 + e;
+          const float c = softcap_of(__uint_as_float(r[e]), p.softcap, k2);
+          if (col == y) p.ce_tgt[gm] = c;
+          const float cv = col < p.N ? c : -INFINITY;
+          cmx = fmaxf(cmx, cv);
+          r[e] = __float_as_uint(cv);
+        }
+        const float nmx = fmaxf(mx, cmx);  // finite: column n0 < N is in the first chunk
+        float se = 0.f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) se += ex2_fast((__uint_as_float(r[e]) - nmx) * LOG2E_F);
+        sm = sm * ex2_fast((mx - nmx) * LOG2E_F) + se;
+        mx = nmx;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+              make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 4 * i + (lane >> 3), j = lane & 7;  // row of the warp's 32, 16-byte chunk
+          const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 128 + ((j ^ (rr & 7)) << 4));
+          const int col = n0 + c0 + 4 * j;
+          const int grow = m0 + q * 32 + rr;
+          if (grow < p.M && col + 4 <= p.N)
+            *reinterpret_cast<uint4*>(outc + (int64_t)grow * p.ldo + col) = v;
+        }
+        __syncwarp();
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      if (gm < p.M) p.ce_part[(int64_t)gm * p.tiles_n + tn] = make_float2(mx, sm);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
     }
   } else {
     // -------------------------------------------------------------- epilogue
@@ -419,11 +504,11 @@ int num_sms() {
 
 namespace {
 
-template <int BN, bool A_MN, bool B_MN>
+template <int BN, bool A_MN, bool B_MN, int EPI = EPI_BF16>
 cudaError_t run_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0, const CUtensorMap& b1,
                      TcGemmParams p, cudaStream_t s) {
   using C = Cfg<BN, A_MN, B_MN>;
-  auto kern = tc_gemm_kernel<BN, A_MN, B_MN>;
+  auto kern = tc_gemm_kernel<BN, A_MN, B_MN, EPI>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   if (e != cudaSuccess) return e;
   const int tiles = p.tiles_m * p.tiles_n;
@@ -544,6 +629,82 @@ cudaError_t launch_proj_bwd_dw_tc(int64_t M, int D, int d, const void* dRk, cons
   p.spin_limit = spin_limit;
   p.err = err;
   return run_gemm<BN, true, true>(a0, a1, b, b, p, s);
+}
+
+// ---------------------------------------------------------------- LM head
+// c [N, V] fp32 = softcap * tanh(m [N, d] U [V, d]^T / softcap), with per-row,
+// per-256-column (max, sum exp) pairs in part [N, ceil(V / 256)] and the
+// target's capped logit in tgt [N]. Needs d % 8 == 0, V % 8 == 0.
+cudaError_t launch_lm_logits_ce_tc(int64_t N, int d, int V, float softcap, const void* m, const void* U,
+                                   const int64_t* targets, float* c, float2* part, float* tgt,
+                                   int64_t spin_limit, int* err, cudaStream_t s) {
+  constexpr int BN = 256;
+  CUtensorMap a, b;
+  cudaError_t e;
+  if ((e = make_tmap_bf16_2d(&a, m, d, N, (uint64_t)d * 2, 64, BM)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&b, U, d, V, (uint64_t)d * 2, 64, BN)) != cudaSuccess) return e;
+  TcGemmParams p{};
+  p.M = (int)N;
+  p.N = V;
+  p.K = d;
+  p.tiles_m = (int)((N + BM - 1) / BM);
+  p.tiles_n = (V + BN - 1) / BN;
+  p.targets = targets;
+  p.softcap = softcap;
+  p.ce_part = part;
+  p.ce_tgt = tgt;
+  p.out0 = c;
+  p.out1 = c;
+  p.ldo = V;
+  p.spin_limit = spin_limit;
+  p.err = err;
+  return run_gemm<BN, false, false, EPI_CE>(a, a, b, b, p, s);
+}
+
+int lm_ce_tiles(int V) { return (V + 255) / 256; }
+
+// dm [N, d] = dz [N, V] U [V, d] (K = V).
+cudaError_t launch_lm_dm_tc(int64_t N, int d, int V, const void* dz, const void* U, void* dm, int64_t spin_limit,
+                            int* err, cudaStream_t s) {
+  constexpr int BN = 256;
+  CUtensorMap a, b;
+  cudaError_t e;
+  if ((e = make_tmap_bf16_2d(&a, dz, V, N, (uint64_t)V * 2, 64, BM)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&b, U, d, V, (uint64_t)d * 2, 64, 64)) != cudaSuccess) return e;
+  TcGemmParams p{};
+  p.M = (int)N;
+  p.N = d;
+  p.K = V;
+  p.tiles_m = (int)((N + BM - 1) / BM);
+  p.tiles_n = (d + BN - 1) / BN;
+  p.out0 = dm;
+  p.out1 = dm;
+  p.ldo = d;
+  p.spin_limit = spin_limit;
+  p.err = err;
+  return run_gemm<BN, false, true>(a, a, b, b, p, s);
+}
+
+// dU [V, d] = dz^T [V, N] m [N, d] (K = N).
+cudaError_t launch_lm_dU_tc(int64_t N, int d, int V, const void* dz, const void* m, void* dU, int64_t spin_limit,
+                            int* err, cudaStream_t s) {
+  constexpr int BN = 256;
+  CUtensorMap a, b;
+  cudaError_t e;
+  if ((e = make_tmap_bf16_2d(&a, dz, V, N, (uint64_t)V * 2, 64, 64)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&b, m, d, N, (uint64_t)d * 2, 64, 64)) != cudaSuccess) return e;
+  TcGemmParams p{};
+  p.M = V;
+  p.N = d;
+  p.K = (int)N;
+  p.tiles_m = (V + BM - 1) / BM;
+  p.tiles_n = (d + BN - 1) / BN;
+  p.out0 = dU;
+  p.out1 = dU;
+  p.ldo = d;
+  p.spin_limit = spin_limit;
+  p.err = err;
+  return run_gemm<BN, true, true>(a, a, b, b, p, s);
 }
 
 }  // namespace maglev
