@@ -105,6 +105,18 @@ size_t maglev_last_error(char* buf, size_t n);
  * *code receives MAGLEV_OK or the first MAGLEV_ERR_TIMEOUT recorded. */
 maglev_status maglev_device_status(void* stream, int* code);
 
+/* Self-test of the bounded waits that every tensor-core kernel of this library
+ * uses (no counterpart in the pages: part of this library's failure handling).
+ * One CTA starts a bulk copy of `bytes` bytes from `src` into shared memory,
+ * allocates tensor memory, then waits on an mbarrier that nothing completes;
+ * after spin_limit microseconds of GPU time the wait gives up, raises the
+ * CTA's abort flag and records MAGLEV_ERR_TIMEOUT in the device status word,
+ * the copy is drained, the tensor memory freed, and the kernel returns. After
+ * the work on `stream` completes, maglev_device_status reports the timeout.
+ *   src: device buffer, 16-byte aligned; bytes: a multiple of 16 in [16, 4096].
+ *   spin_limit: in [1, 1e7] microseconds. */
+maglev_status maglev_wait_selftest(const void* src, int bytes, int64_t spin_limit, void* stream);
+
 /* Bytes of the activations the forward saves for the backward ("saved"):
  * the rotated queries and the mixed keys/values, 3 x [B,T,H,hd] of dtype. */
 size_t maglev_swa_saved_bytes(const maglev_swa_desc* desc);

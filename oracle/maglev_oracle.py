@@ -230,13 +230,16 @@ def inject_swa_backward(q, k, v, R_k, R_v, gate_logits, dout, window: int, pos0:
         Rk = R_k.reshape(B, T, H, hd)
         out["dR_k"] = rmsnorm_backward(Rk, dn, eps).reshape(B, T, H * hd)
         out["dR_v"] = (gv_r * dv_bar).reshape(B, T, H * hd)
-        dg = np.stack([
-            np.sum(dk_bar * f["k_loc"], axis=(0, 1, 3)),
-            np.sum(dk_bar * f["k_rec"], axis=(0, 1, 3)),
-            np.sum(dv_bar * v, axis=(0, 1, 3)),
-            np.sum(dv_bar * R_v.reshape(B, T, H, hd), axis=(0, 1, 3)),
-        ])
-        out["dgate"] = fold_gate_grads(dg * gate_slope(gate_rows(gate_logits)), gate_logits)
+        terms = [dk_bar * f["k_loc"], dk_bar * f["k_rec"], dv_bar * v, dv_bar * R_v.reshape(B, T, H, hd)]
+        dg = np.stack([np.sum(t, axis=(0, 1, 3)) for t in terms])
+        slope = gate_slope(gate_rows(gate_logits))
+        out["dgate"] = fold_gate_grads(dg * slope, gate_logits)
+        # Scale of each gate gradient's rounding error: each is a sum of B*T*hd
+        # products, whose rounding error grows with the RMS size of the summands
+        # (sqrt of the sum of their squares), not with the sum itself, which can
+        # cancel. Test infrastructure: not a quantity of the method.
+        sc2 = np.stack([np.sum(t * t, axis=(0, 1, 3)) for t in terms]) * slope ** 2
+        out["dgate_scale"] = np.sqrt(fold_gate_grads(sc2, gate_logits))
     else:
         out["dk"] = rope(dk_bar, posb, rope_base, inverse=True)
         out["dv"] = dv_bar
@@ -367,7 +370,8 @@ def stack_forward_backward(q_layers, p_layers, w_mk, w_mv, lam: float, rope_base
             dout = store(dout + rmsnorm_backward(op, dm, eps).reshape(B, T, H, hd))
         g = inject_swa_backward(L["q"], L["k"], L["v"], Rs[i][0], Rs[i][1], L["gates"], dout, L["window"], 0,
                                 rope_base, eps)
-        grads = {"dq": g["dq"], "dk": g["dk"], "dv": g["dv"], "dgate": g["dgate"], "dout": dout}
+        grads = {"dq": g["dq"], "dk": g["dk"], "dv": g["dv"], "dgate": g["dgate"], "dgate_scale": g["dgate_scale"],
+                 "dout": dout}
         if per_layer:
             dms, dwk, dwv = mem_project_backward(m_shift, L["w_mk"], L["w_mv"], g["dR_k"], g["dR_v"])
             dm_shift += dms

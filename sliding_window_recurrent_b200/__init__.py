@@ -76,6 +76,7 @@ _SIGS = {
     "maglev_decode_mem_project": ([ctypes.POINTER(DecodeDesc)] + [_P] * 7, _I),
     "maglev_decode_step": ([ctypes.POINTER(DecodeDesc)] + [_P] * 11, _I),
     "maglev_decode_prefill": ([ctypes.POINTER(SwaDesc)] + [_P] * 4, _I),
+    "maglev_wait_selftest": ([_P, _I, _I64, _P], _I),
     "maglev_lm_head_workspace_bytes": ([_I64, _I, _I], _SZ),
     "maglev_lm_head_ce": ([_I64, _I, _I, _I, _F, _F] + [_P] * 8 + [_I64, _P], _I),
 }
@@ -265,3 +266,7 @@ def maglev_lm_head_ce(N, d, V, dtype, softcap, inv_count, m, U, targets, loss, l
     _check(_lib.maglev_lm_head_ce(int(N), int(d), int(V), int(dtype), float(softcap), float(inv_count), _ptr(m),
                                   _ptr(U), _ptr(targets), _ptr(loss), _ptr(lse), _ptr(dm), _ptr(dU),
                                   _ptr(workspace), int(spin_limit), _stream(stream)))
+
+
+def maglev_wait_selftest(src, nbytes, spin_limit, stream=None):
+    _check(_lib.maglev_wait_selftest(_ptr(src), int(nbytes), int(spin_limit), _stream(stream)))

@@ -829,6 +829,20 @@ maglev_status maglev_decode_mem_project(const maglev_decode_desc* d, const int64
   return MAGLEV_OK;
 }
 
+maglev_status maglev_wait_selftest(const void* src, int bytes, int64_t spin_limit, void* stream) {
+  NEED_PTR(src);
+  if (bytes < 16 || bytes > 4096 || bytes % 16 != 0)
+    return fail(MAGLEV_ERR_INVALID_ARG, "bytes must be a multiple of 16 in [16, 4096]");
+  if (spin_limit < 1 || spin_limit > 10000000)
+    return fail(MAGLEV_ERR_INVALID_ARG, "spin_limit must be in [1, 1e7] microseconds");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* err = nullptr;
+  maglev_status st = status_word(&err, s);
+  if (st != MAGLEV_OK) return st;
+  MAGLEV_LAUNCH(1, s, launch_wait_selftest(src, bytes, spin_limit, err, s), "wait_selftest");
+  return MAGLEV_OK;
+}
+
 maglev_status maglev_decode_prefill(const maglev_swa_desc* d, const void* saved, void* k_ring, void* v_ring,
                                     void* stream) {
   maglev_status st = check_swa(d);

@@ -142,6 +142,11 @@ cudaError_t launch_lm_dm_tc(int64_t N, int d, int V, const void* dz, const void*
 cudaError_t launch_lm_dU_tc(int64_t N, int d, int V, const void* dz, const void* m, void* dU, int64_t spin_limit,
                             int* err, cudaStream_t s);
 
+// One CTA: bulk copy of `bytes` from src into shared memory, tensor memory
+// held, then a bounded wait on an mbarrier nothing completes (expires after
+// limit_us, records DEV_TIMEOUT), drain, free, return.
+cudaError_t launch_wait_selftest(const void* src, int bytes, int64_t limit_us, int* err, cudaStream_t st);
+
 // Default bound of one in-kernel wait, in microseconds of GPU time (1 s).
 constexpr int64_t DEFAULT_SPIN_LIMIT = 1000000;
 

@@ -31,9 +31,10 @@ from __future__ import annotations
 
 import torch
 
-from . import (MAGLEV_DR_ADD, MAGLEV_DR_FIRST, MAGLEV_DR_LAST, MAGLEV_DR_WRITE, SwaDesc, maglev_consistency_loss, maglev_consistency_workspace_bytes, maglev_inject_swa_bwd,
-               maglev_inject_swa_fwd, maglev_mem_project, maglev_mem_project_bwd, maglev_memory_state,
-               maglev_memory_state_bwd, maglev_swa_bwd_workspace_bytes, maglev_swa_saved_bytes)
+from . import (MAGLEV_DR_ADD, MAGLEV_DR_FIRST, MAGLEV_DR_LAST, MAGLEV_DR_WRITE, SwaDesc, maglev_consistency_loss,
+               maglev_consistency_workspace_bytes, maglev_inject_swa_bwd, maglev_inject_swa_fwd, maglev_mem_project,
+               maglev_mem_project_bwd, maglev_mem_project_bwd_layers, maglev_memory_state, maglev_memory_state_bwd,
+               maglev_swa_bwd_workspace_bytes, maglev_swa_saved_bytes)
 from .layer import CODE, TORCH_DTYPE, _bytes
 
 

@@ -62,11 +62,40 @@ def elementwise(gpu, ref):
     return float(np.max(np.abs(gpu - ref) / np.maximum(np.abs(ref), rms)))
 
 
-def assert_close(gpu, ref, dtype, name="", metric="normwise"):
-    """metric: "normwise" (whole tensor), "rows" (each row of the last axis) or
-    "elementwise" (per entry, RMS floor)."""
-    fn = {"normwise": normwise, "rows": rowwise, "elementwise": elementwise}[metric]
-    err = fn(gpu, ref)
+def logwise(gpu, ref):
+    """Error of a log-domain quantity (LSE) row by row, each row's normwise error
+    with a floor of 1 below the row's largest magnitude: an absolute error d in
+    a log-sum-exp is a relative error e^d - 1 ~ d of the partition function, so
+    near zero the error is judged in absolute terms."""
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
+    n = ref.shape[-1]
+    g2, r2 = gpu.reshape(-1, n), ref.reshape(-1, n)
+    den = np.maximum(np.max(np.abs(r2), axis=1), 1.0)
+    return float(np.max(np.max(np.abs(g2 - r2), axis=1) / den))
+
+
+def scaled(gpu, ref, scale):
+    """max_i |gpu_i - ref_i| / scale_i: the error of each entry of a reduced
+    quantity against the RMS size of the summands it adds up (the scale of its
+    rounding error; see the oracle's dgate_scale)."""
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    scale = np.asarray(scale, dtype=np.float64)
+    assert gpu.shape == ref.shape == scale.shape, (gpu.shape, ref.shape, scale.shape)
+    return float(np.max(np.abs(gpu - ref) / np.where(scale > 0, scale, 1.0)))
+
+
+def assert_close(gpu, ref, dtype, name="", metric="normwise", scale=None):
+    """metric: "normwise" (whole tensor), "rows" (each row of the last axis),
+    "log" (LSE rows, floor 1), "elementwise" (per entry, RMS floor) or
+    "scaled" (per entry against `scale`)."""
+    if metric == "scaled":
+        err = scaled(gpu, ref, scale)
+    else:
+        fn = {"normwise": normwise, "rows": rowwise, "log": logwise, "elementwise": elementwise}[metric]
+        err = fn(gpu, ref)
     assert np.all(np.isfinite(np.asarray(gpu))), f"{name}: non-finite values"
     assert err <= TOL[dtype], f"{name}: {metric} error {err:.3e} > {TOL[dtype]:.0e}"
     return err

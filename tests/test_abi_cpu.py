@@ -118,3 +118,17 @@ def test_bwd_and_loss_and_decode_validation():
     dd.hd = 64
     dd.B = 0
     mg.maglev_decode_step(dd, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, stream=0)
+
+
+def test_driver_modules_only_call_bound_entry_points():
+    """Every maglev_* name the Python drivers (layer.py, stack.py) call is
+    imported there and bound by the package (a missing import only shows at
+    call time, on the GPU)."""
+    import re
+    import sliding_window_recurrent_b200.layer as layer
+    import sliding_window_recurrent_b200.stack as stack
+    for mod in (layer, stack):
+        src = open(mod.__file__).read()
+        for name in set(re.findall(r"\b(maglev_[a-z0-9_]+)\(", src)):
+            assert hasattr(mod, name), (mod.__name__, name)
+            assert hasattr(mg, name), name

@@ -70,7 +70,8 @@ def _check_all(S, ref, dt):
         assert_close(host(L.out), ref["p_out"][i], dt, f"P{i} out")
         for g in ("dq", "dk", "dv"):
             assert_close(host(getattr(L, g)), ref["p_grads"][i][g], dt, f"P{i} {g}")
-        assert_close(host(L.dgate), ref["p_grads"][i]["dgate"], dt, f"P{i} dgate", "rows")
+        assert_close(host(L.dgate), ref["p_grads"][i]["dgate"], dt, f"P{i} dgate", "scaled",
+                     ref["p_grads"][i]["dgate_scale"])
     assert_close(host(S.m_prime), ref["m_prime"], dt, "m'")
     assert_close(host(S.m_shift), ref["m_shift"], dt, "m_shift")
     assert np.all(host(S.m_shift)[:, 0] == 0), "row 0 of the shifted memory is m'_0 = 0"

@@ -633,3 +633,21 @@ def test_lm_head_central_differences():
             arr[idx] = a0
             fd = (lp - lm) / (2 * h)
             assert abs(fd - grad[idx]) <= 1e-7 * max(1.0, abs(fd)), (idx, fd, grad[idx])
+
+
+def test_gate_gradient_scale_bounds_the_sum():
+    """dgate_scale is the RMS size sqrt(sum t^2) of the B*T*hd products t each
+    gate gradient sums (times the gate's slope): by Cauchy-Schwarz
+    |dgate| <= sqrt(B*T*hd) * dgate_scale, with equality when all products are
+    equal; with the shared K/V form the two shares' scales add in quadrature."""
+    B, T, H, hd, W = 1, 9, 2, 4, 3
+    q, k, v, dout = (rand(B, T, H, hd) for _ in range(4))
+    Rk, Rv = rand(B, T, H * hd), rand(B, T, H * hd)
+    g4 = RNG.uniform(-2, 2, (4, H))
+    r = oracle.inject_swa_backward(q, k, v, Rk, Rv, g4, dout, W)
+    assert np.all(np.abs(r["dgate"]) <= np.sqrt(B * T * hd) * r["dgate_scale"] * (1 + 1e-12))
+    assert np.all(r["dgate_scale"] > 0)
+    r2 = oracle.inject_swa_backward(q, k, v, Rk, Rv, g4[:2], dout, W)
+    r4 = oracle.inject_swa_backward(q, k, v, Rk, Rv, np.concatenate([g4[:2], g4[:2]]), dout, W)
+    np.testing.assert_allclose(r2["dgate_scale"], np.sqrt(r4["dgate_scale"][:2] ** 2 + r4["dgate_scale"][2:] ** 2),
+                               rtol=1e-13)
