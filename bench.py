@@ -272,7 +272,28 @@ def aggregate_profile(rows):
     return agg
 
 
+def capture_graph(torch, fn):
+    """fn's launches captured once into a CUDA graph (after a side-stream run,
+    as torch's graph capture wants)."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
 def run_layer_bench(torch, dist, rank, world, dev, steps, warmup, peaks, peaks_src, gpu_uuid):
+    """The step's launches are captured in a CUDA graph and replayed for the
+    timed steps (no host gaps between the kernels). The library's per-launch
+    tracing is on while the graph is captured, so the CUDA events around every
+    kernel are nodes of the graph: after the timed replays they hold the
+    per-kernel durations of the last timed step."""
     import sliding_window_recurrent_b200 as mg
     c = LAYER
     x = make_layer_inputs(torch, dev, 1234 + rank)
@@ -281,6 +302,24 @@ def run_layer_bench(torch, dist, rank, world, dev, steps, warmup, peaks, peaks_s
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
+    s = torch.cuda.Stream()  # side-stream run before capture, as torch's graph capture wants
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    mg.maglev_profile_report()  # drop any earlier records
+    graph = torch.cuda.CUDAGraph()
+    mg.maglev_profile_enable(True)
+    n0 = mg.maglev_launch_count()
+    with torch.cuda.graph(graph):
+        step()
+    per_step = mg.maglev_launch_count() - n0
+    mg.maglev_profile_enable(False)
+    torch.cuda.synchronize()
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     sampler = ClockSampler(gpu_uuid)
@@ -288,18 +327,16 @@ def run_layer_bench(torch, dist, rank, world, dev, steps, warmup, peaks, peaks_s
     time.sleep(0.3)
     stream = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    mg.maglev_profile_enable(True)
-    n0 = mg.maglev_launch_count()
     torch.cuda.synchronize()
     e0.record(stream)
     for _ in range(steps):
-        step()
+        graph.replay()
     e1.record(stream)
     torch.cuda.synchronize()
-    launches = mg.maglev_launch_count() - n0
-    mg.maglev_profile_enable(False)
-    prof = aggregate_profile(mg.maglev_profile_report())
+    launches = per_step * steps
     clocks = sampler.stop()
+    prof = aggregate_profile(mg.maglev_profile_report())  # the last timed replay's kernels
+    del graph
     ms = e0.elapsed_time(e1) / steps
     ms_max = max_over_ranks(dist, ms, dev)
     if dist is not None:
@@ -328,6 +365,7 @@ def run_layer_bench(torch, dist, rank, world, dev, steps, warmup, peaks, peaks_s
         roof["spec_peak"] = SPEC_PEAKS[key]
         roof["frac_of_spec"] = round(roof["achieved"] / SPEC_PEAKS[key], 5)
         roof["avg_launch_ms"] = round(avg_ms, 5)
+        roof["duration_source"] = "CUDA events recorded by nodes of the replayed graph, last timed step"
         roof["work_per_launch"] = work
     kernels = {n: {"calls": v[0], "ms_total": round(v[1], 4), "share": round(v[1] / sum(w[1] for w in prof.values()), 4)}
                for n, v in sorted(prof.items(), key=lambda kv: -kv[1][1])}
@@ -368,7 +406,8 @@ def run_layer_e2e(torch, dev, steps, warmup, step):
 
 
 def run_layer_fwd_bench(torch, dev, steps, warmup, step):
-    """Forward only (projection, injection, attention) of the same layer."""
+    """Forward only (projection, injection, attention) of the same layer, as a
+    replayed CUDA graph."""
     x, L = step.x, step.L
 
     def fwd():
@@ -377,12 +416,17 @@ def run_layer_fwd_bench(torch, dev, steps, warmup, step):
     for _ in range(warmup):
         fwd()
     torch.cuda.synchronize()
+    graph = capture_graph(torch, fwd)
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(steps):
-        fwd()
+        graph.replay()
     e1.record()
     torch.cuda.synchronize()
+    del graph
     c = LAYER
     f = layer_flops(c["B"], c["T"], c["H"], c["hd"], c["d"], c["W"])
     ms = e0.elapsed_time(e1) / steps

@@ -565,7 +565,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       constexpr uint32_t ID_KV = idesc_bf16(128, HD, false, true);  // dV, dK: 128 keys x hd
       constexpr uint32_t ID_DQ = idesc_bf16(HD, 64, true, true);    // dQ^T: hd x 64 queries
       const uint32_t k_addr = smem_u32(smem + C::OFF_K);
-      const uint32_t v_addr = smem_u32(smem + C::OFF_V);
+      // base descriptors: each MMA's operand is a constant offset from these
+      const uint64_t kd0 = kmajor_desc(k_addr, 0), vd0 = kmajor_desc(smem_u32(smem + C::OFF_V), 0);
+      const uint64_t kmn = sw128_desc(k_addr, (uint32_t)C::KCHUNK, 1024u);  // K read MN-major (dQ^T)
       // S^T_gs, dP^T_gs, once Q/dO have arrived and the softmax warps have
       // loaded S/dP of half-tile gs-1
       auto issue_sdp = [&](int gs) -> bool {
@@ -573,19 +575,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(&q_full[s], (uint32_t)(gs / 3) & 1u, ab)) return false;
         if (gs >= 1 && !mbar_wait(s_free, (uint32_t)(gs - 1) & 1u, ab)) return false;
         tc_fence_after();
-        const uint32_t q_addr = smem_u32(smem + C::OFF_Q + s * C::QH);
-        const uint32_t do_addr = smem_u32(smem + C::OFF_DO + s * C::QH);
+        const uint64_t qd = kmajor_desc(smem_u32(smem + C::OFF_Q + s * C::QH), 0);
+        const uint64_t dod = kmajor_desc(smem_u32(smem + C::OFF_DO + s * C::QH), 0);
 #pragma unroll
         for (int k16 = 0; k16 < HD / 16; ++k16) {
-          const uint32_t ka = (uint32_t)(k16 >> 2) * C::KCHUNK, qa = (uint32_t)(k16 >> 2) * C::QCHUNK;
-          mma_ss(tmem + C::T_S, kmajor_desc(k_addr + ka, k16 & 3), kmajor_desc(q_addr + qa, k16 & 3), ID_S,
-                 k16 > 0 ? 1u : 0u);
+          const uint32_t ka = (uint32_t)(k16 >> 2) * C::KCHUNK + (k16 & 3) * 32u;
+          const uint32_t qa = (uint32_t)(k16 >> 2) * C::QCHUNK + (k16 & 3) * 32u;
+          mma_ss(tmem + C::T_S, desc_at(kd0, ka), desc_at(qd, qa), ID_S, k16 > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int k16 = 0; k16 < HD / 16; ++k16) {
-          const uint32_t ka = (uint32_t)(k16 >> 2) * C::KCHUNK, qa = (uint32_t)(k16 >> 2) * C::QCHUNK;
-          mma_ss(tmem + C::T_DP, kmajor_desc(v_addr + ka, k16 & 3), kmajor_desc(do_addr + qa, k16 & 3), ID_S,
-                 k16 > 0 ? 1u : 0u);
+          const uint32_t ka = (uint32_t)(k16 >> 2) * C::KCHUNK + (k16 & 3) * 32u;
+          const uint32_t qa = (uint32_t)(k16 >> 2) * C::QCHUNK + (k16 & 3) * 32u;
+          mma_ss(tmem + C::T_DP, desc_at(vd0, ka), desc_at(dod, qa), ID_S, k16 > 0 ? 1u : 0u);
         }
         mma_commit(s_full);
         return true;
@@ -599,31 +601,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // unit's epilogue must have read them
         if (jr == 0 && !mbar_wait(acc_empty, ((uint32_t)nr & 1u) ^ 1u, ab)) return false;
         tc_fence_after();
-        const uint32_t q_addr = smem_u32(smem + C::OFF_Q + s * C::QH);
-        const uint32_t do_addr = smem_u32(smem + C::OFF_DO + s * C::QH);
-        const uint32_t p_addr = smem_u32(smem + C::OFF_P + buf * C::PH);
         const uint32_t ds_addr = smem_u32(smem + C::OFF_DS + buf * C::PH);
+        const uint64_t pd = kmajor_desc(smem_u32(smem + C::OFF_P + buf * C::PH), 0);
+        const uint64_t dsd = kmajor_desc(ds_addr, 0);
+        const uint64_t domn = sw128_desc(smem_u32(smem + C::OFF_DO + s * C::QH), (uint32_t)C::QCHUNK, 1024u);
+        const uint64_t qmn = sw128_desc(smem_u32(smem + C::OFF_Q + s * C::QH), (uint32_t)C::QCHUNK, 1024u);
+        const uint64_t dsmn = sw128_desc(ds_addr, (uint32_t)C::PH, 1024u);
 #pragma unroll
-        for (int k16 = 0; k16 < 4; ++k16) {  // K = 64 queries
-          mma_ss(tmem + C::T_DV, kmajor_desc(p_addr, k16),
-                 sw128_desc(do_addr + (uint32_t)k16 * 2048u, (uint32_t)C::QCHUNK, 1024u), ID_KV,
+        for (int k16 = 0; k16 < 4; ++k16)  // K = 64 queries
+          mma_ss(tmem + C::T_DV, desc_at(pd, k16 * 32u), desc_at(domn, k16 * 2048u), ID_KV,
                  (jr > 0 || k16 > 0) ? 1u : 0u);
-        }
 #pragma unroll
-        for (int k16 = 0; k16 < 4; ++k16) {
-          mma_ss(tmem + C::T_DK, kmajor_desc(ds_addr, k16),
-                 sw128_desc(q_addr + (uint32_t)k16 * 2048u, (uint32_t)C::QCHUNK, 1024u), ID_KV,
+        for (int k16 = 0; k16 < 4; ++k16)
+          mma_ss(tmem + C::T_DK, desc_at(dsd, k16 * 32u), desc_at(qmn, k16 * 2048u), ID_KV,
                  (jr > 0 || k16 > 0) ? 1u : 0u);
-        }
         mma_commit(&q_empty[s]);
         // DQ[buf] held dQ^T of half-tile gr-2: drained by now in practice
         if (gr >= 2 && !mbar_wait(&dq_empty[buf], (uint32_t)((gr - 2) >> 1) & 1u, ab)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int k16 = 0; k16 < 8; ++k16) {  // K = 128 keys
-          mma_ss(tmem + C::T_DQ + 64u * buf, sw128_desc(k_addr + (uint32_t)k16 * 2048u, (uint32_t)C::KCHUNK, 1024u),
-                 sw128_desc(ds_addr + (uint32_t)k16 * 2048u, (uint32_t)C::PH, 1024u), ID_DQ, k16 > 0 ? 1u : 0u);
-        }
+        for (int k16 = 0; k16 < 8; ++k16)  // K = 128 keys
+          mma_ss(tmem + C::T_DQ + 64u * buf, desc_at(kmn, k16 * 2048u), desc_at(dsmn, k16 * 2048u), ID_DQ,
+                 k16 > 0 ? 1u : 0u);
         mma_commit(&dq_full[buf]);
         return true;
       };

@@ -210,18 +210,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
       // ------------------------------------------------------------ MMA issuer
       constexpr uint32_t ID_S = idesc_bf16(128, 64, false, false);  // 128 queries x 64 keys
       constexpr uint32_t ID_O = idesc_bf16(128, HD, false, true);   // 128 queries x hd
-      const uint32_t q_addr = smem_u32(smem + C::OFF_Q);
-      const uint32_t p_addr = smem_u32(smem + C::OFF_P);
+      // base descriptors: each MMA's operand is a constant offset from these
+      const uint64_t qd = kmajor_desc(smem_u32(smem + C::OFF_Q), 0);
+      const uint64_t pd = kmajor_desc(smem_u32(smem + C::OFF_P), 0);
       // S_gs = Q K_gs^T into S buffer gs&1; the K slot is released when it completes
       auto issue_s = [&](int gs) -> bool {
         const int s = gs & 1;
         if (!mbar_wait(&k_full[s], (uint32_t)(gs >> 1) & 1u, ab)) return false;
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(smem + C::OFF_K + s * C::KH);
+        const uint64_t kd = kmajor_desc(smem_u32(smem + C::OFF_K + s * C::KH), 0);
 #pragma unroll
         for (int k16 = 0; k16 < HD / 16; ++k16) {
-          mma_ss(tmem + C::T_S + 64u * (uint32_t)s, kmajor_desc(q_addr + (uint32_t)(k16 >> 2) * C::QCHUNK, k16 & 3),
-                 kmajor_desc(k_addr + (uint32_t)(k16 >> 2) * C::KCHUNK, k16 & 3), ID_S, k16 > 0 ? 1u : 0u);
+          mma_ss(tmem + C::T_S + 64u * (uint32_t)s, desc_at(qd, (uint32_t)(k16 >> 2) * C::QCHUNK + (k16 & 3) * 32u),
+                 desc_at(kd, (uint32_t)(k16 >> 2) * C::KCHUNK + (k16 & 3) * 32u), ID_S, k16 > 0 ? 1u : 0u);
         }
         mma_commit(&s_full[s]);
         mma_commit(&k_empty[s]);
@@ -257,13 +258,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
             break;
           }
           tc_fence_after();
-          const uint32_t v_addr = smem_u32(smem + C::OFF_V + (g & 1) * C::KH);
+          const uint64_t vmn = sw128_desc(smem_u32(smem + C::OFF_V + (g & 1) * C::KH), (uint32_t)C::KCHUNK, 1024u);
 #pragma unroll
-          for (int k16 = 0; k16 < 4; ++k16) {  // K = 64 keys
-            mma_ss(tmem + C::T_O, kmajor_desc(p_addr, k16),
-                   sw128_desc(v_addr + (uint32_t)k16 * 2048u, (uint32_t)C::KCHUNK, 1024u), ID_O,
+          for (int k16 = 0; k16 < 4; ++k16)  // K = 64 keys
+            mma_ss(tmem + C::T_O, desc_at(pd, k16 * 32u), desc_at(vmn, k16 * 2048u), ID_O,
                    (j > 0 || k16 > 0) ? 1u : 0u);
-          }
           mma_commit(&v_empty[g & 1]);
           mma_commit(pv_done);
         }

@@ -163,6 +163,10 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
   d |= (uint64_t)2 << 61;
   return d;
 }
+// The descriptor of the same layout `byte_off` bytes further on: only the
+// start-address field (bits 0-13, address >> 4) changes, and shared-memory
+// addresses (< 228 KiB) keep it below 2^14, so the sum never carries out.
+__device__ __forceinline__ uint64_t desc_at(uint64_t d, uint32_t byte_off) { return d + (byte_off >> 4); }
 // K-major operand tile: rows of 64 bf16 (128 B), 8-row atoms of 1024 B.
 // k16 selects the 16-element K slice inside the 64-wide swizzle span.
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_saddr, int k16) {

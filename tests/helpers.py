@@ -4,6 +4,14 @@ import numpy as np
 import synth
 
 TOL = {"f32": 1e-4, "bf16": 2e-2}
+# Gate gradients, per entry against the RMS size of the B*T*hd products each
+# sums (see `scaled`). Derived from the arithmetic: rounding the operands the
+# bf16 kernels round (q_rot, k_bar, v_bar, P, dS, dk_bar, dv_bar) in an fp64
+# emulation of the backward moves these sums by up to 2.0e-2 of that scale at
+# T = 2048 (each dk_bar sums ~512 dS q products with heavy cancellation, and the
+# rounding of dS does not cancel with it); 5e-2 leaves room for the spread
+# between rounding realisations. fp32 storage keeps the fp32 bound.
+GATE_TOL = {"f32": 1e-4, "bf16": 5e-2}
 
 
 def dev(t, device="cuda"):
@@ -96,6 +104,7 @@ def assert_close(gpu, ref, dtype, name="", metric="normwise", scale=None):
     else:
         fn = {"normwise": normwise, "rows": rowwise, "log": logwise, "elementwise": elementwise}[metric]
         err = fn(gpu, ref)
+    tol = GATE_TOL[dtype] if metric == "scaled" else TOL[dtype]
     assert np.all(np.isfinite(np.asarray(gpu))), f"{name}: non-finite values"
-    assert err <= TOL[dtype], f"{name}: {metric} error {err:.3e} > {TOL[dtype]:.0e}"
+    assert err <= tol, f"{name}: {metric} error {err:.3e} > {tol:.0e}"
     return err

@@ -4,7 +4,8 @@ Tolerance: 1e-4 for fp32 storage, 2e-2 for bf16 storage with fp32
 accumulation, on the normwise error max|gpu - ref| / max|ref| of each tensor;
 LSE row by row in the log domain (an absolute error below 1, a relative one
 above); each gate-gradient entry against the RMS size of the products it sums
-(a sum of B*T*hd terms can cancel far below its rounding-error scale). The
+(a sum of B*T*hd terms can cancel far below its rounding-error scale), within
+helpers.GATE_TOL (derived there from an emulation of the bf16 operands). The
 full-size layer test also reports the element-wise error max|gpu - ref| /
 max(|ref|, rms(ref)); it is not gated, because the bf16 operands of the
 attention (q_rot, k_bar and P rounded to bf16) move individual scores by ~1e-2
