@@ -32,7 +32,7 @@
 namespace maglev {
 
 cudaError_t make_tmap_tokens(CUtensorMap* m, const void* base, int B, int T, int H, int hd, uint32_t box_rows);
-cudaError_t make_tmap_f32_tokens(CUtensorMap* m, void* base, int B, int T, int H, int hd);
+cudaError_t make_tmap_f32_tokens(CUtensorMap* m, void* base, int B, int T, int H, int hd, uint32_t box_rows);
 int num_sms();
 
 namespace {
@@ -401,6 +401,10 @@ __device__ __forceinline__ void store_half_row(uint8_t* tile, int r, const float
   }
 }
 
+constexpr int PIPE_SOFT_WARPS = 16;                  // 4 per TMEM lane quarter
+constexpr int PIPE_SOFT_THREADS = 32 * PIPE_SOFT_WARPS;
+constexpr int PIPE_THREADS = 64 + PIPE_SOFT_THREADS;  // producer, MMA, softmax warps
+
 template <int HD>
 struct PipeCfg {
   static_assert(HD == 128, "pipelined backward is written for 128 channels");
@@ -453,7 +457,7 @@ __device__ __forceinline__ KUnit kunit_of(const PipeParams& p, int r) {
 }
 
 template <int HD>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(PIPE_THREADS, 1)
     attn_bwd_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                          const __grid_constant__ CUtensorMap tmDQ, PipeParams pp) {
@@ -491,14 +495,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&q_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_free, SOFT_THREADS);
+    mbar_init(s_free, PIPE_SOFT_THREADS);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&p_full[s], SOFT_THREADS);
+      mbar_init(&p_full[s], PIPE_SOFT_THREADS);
       mbar_init(&dq_full[s], 1);
-      mbar_init(&dq_empty[s], SOFT_THREADS);
+      mbar_init(&dq_empty[s], PIPE_SOFT_THREADS);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, SOFT_THREADS);
+    mbar_init(acc_empty, PIPE_SOFT_THREADS);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -647,10 +651,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // -------------------------------------------------------------- softmax-backward / drains
+    // 16 warps: warp w reads TMEM lane quarter q4 = w % 4 (key rows / dQ^T
+    // channels 32*q4 ..) and owns the 16 query columns [16*cs, 16*cs + 16) of
+    // each 64-query half-tile, cs = (w - 2) / 4.
     const int q4 = warp & 3;
-    const int half = (warp - 2) >> 2;  // 32 of the 64 query columns
+    const int cs = (warp - 2) >> 2;
     const int r = q4 * 32 + lane;      // TMEM lane: key row (S^T, dV, dK) / channel (dQ^T)
-    const int st = threadIdx.x - 64;   // 0..255 among the softmax threads
+    const int st = threadIdx.x - 64;   // 0..511 among the softmax threads
+    const int w16 = q4 + 4 * cs;       // this warp's 2 KiB staging slice
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     float* lds_all = reinterpret_cast<float*>(smem + C::OFF_LD);
     bool ok = true;
@@ -664,26 +672,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     };
     // dQ^T of half-tile gd (unit xd, its local index jd): lanes are channels,
-    // this warp's 32 columns are queries xd.kt + 64*jd + 32*half ...
+    // this warp's 16 columns are queries xd.kt + 64*jd + 16*cs ...
     auto drain_dq = [&](int gd, const KUnit& xd, int jd) {
       const int buf = gd & 1;
       ok = ok && warp_wait(&dq_full[buf], (uint32_t)(gd >> 1) & 1u, ab);
       if (!ok) return;
       tc_fence_after();
-      uint32_t v[32];
-      tmem_ld32(tmem + lane_off + C::T_DQ + 64u * (uint32_t)buf + 32u * (uint32_t)half, v);
+      uint32_t v[16];
+      tmem_ld16(tmem + lane_off + C::T_DQ + 64u * (uint32_t)buf + 16u * (uint32_t)cs, v);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&dq_empty[buf]);  // DQ[buf] may take dQ^T of half-tile gd + 2
-      // box of 32 query rows x 32 channels (128 B rows, 16-byte chunks swizzled by row)
-      const int w8 = q4 + 4 * half;
-      uint8_t* slice = smem + (w8 < 4 ? C::OFF_P : C::OFF_DS) + buf * C::PH + (w8 & 3) * 4096;
+      // box of 16 query rows x 32 channels (128 B rows, 16-byte chunks swizzled by row)
+      uint8_t* slice = smem + (w16 < 8 ? C::OFF_P : C::OFF_DS) + buf * C::PH + (w16 & 7) * 2048;
 #pragma unroll
-      for (int c = 0; c < 32; ++c)
+      for (int c = 0; c < 16; ++c)
         *reinterpret_cast<uint32_t*>(slice + c * 128 + ((((lane >> 2) ^ (c & 7))) << 4) + (lane & 3) * 4) = v[c];
       fence_proxy_async_smem();
       __syncwarp();
-      const int q0 = xd.kt + 64 * jd + 32 * half;
+      const int q0 = xd.kt + 64 * jd + 16 * cs;
       if (lane == 0 && q0 < p.T) {
         tma_reduce_add_4d(&tmDQ, slice, 32 * q4, xd.h, q0, xd.b);
         bulk_commit();
@@ -708,7 +715,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) bulk_wait_read_all();
         if (st < 128) lds[st] = pre;
         // every softmax thread reaches this barrier on every half-tile, aborted or not
-        asm volatile("bar.sync 1, %0;" ::"n"(SOFT_THREADS) : "memory");
+        asm volatile("bar.sync 1, %0;" ::"n"(PIPE_SOFT_THREADS) : "memory");
         if (j + 1 < x.nh) {
           fetch(x, j + 1);
         } else {
@@ -718,35 +725,64 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ok = ok && warp_wait(s_full, (uint32_t)g & 1u, ab);
         if (ok) {
           tc_fence_after();
-          uint32_t sv[32], dv[32];
-          tmem_ld32(tmem + lane_off + C::T_S + 32u * half, sv);
-          tmem_ld32(tmem + lane_off + C::T_DP + 32u * half, dv);
+          uint32_t sv[16], dv[16];
+          tmem_ld16(tmem + lane_off + C::T_S + 16u * cs, sv);
+          tmem_ld16(tmem + lane_off + C::T_DP + 16u * cs, dv);
           tmem_wait_ld();
           tc_fence_before();
           mbar_arrive(s_free);  // S / dP may take half-tile g + 1
-          const int q0 = qt + 32 * half;  // first query column of this warp
-          const int lo = kj - q0;         // query >= key
-          const int hi = min(kj + p.W - 1, p.T - 1) - q0;
-          const bool full = q0 >= kw + 31 && q0 + 31 <= kw + p.W - 1 && q0 + 31 <= p.T - 1 && kw + 31 < p.T;
-          float pt[32], ds[32];
+          const int q0 = qt + 16 * cs;  // first query column of this warp
+          // every (key, query) of this warp's 32 x 16 block inside the window
+          const bool full = q0 >= kw + 31 && q0 + 15 <= kw + p.W - 1 && q0 + 15 <= p.T - 1 && kw + 31 < p.T;
+          float pt[16], ds[16];
+          if (full) {
 #pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) {
-            const float4 L = *reinterpret_cast<const float4*>(lds + 32 * half + 4 * e4);
-            const float4 D = *reinterpret_cast<const float4*>(lds + 64 + 32 * half + 4 * e4);
-            const float Ls[4] = {L.x, L.y, L.z, L.w};
-            const float Ds[4] = {D.x, D.y, D.z, D.w};
+            for (int e4 = 0; e4 < 4; ++e4) {
+              const float4 L = *reinterpret_cast<const float4*>(lds + 16 * cs + 4 * e4);
+              const float4 D = *reinterpret_cast<const float4*>(lds + 64 + 16 * cs + 4 * e4);
+              const float Ls[4] = {L.x, L.y, L.z, L.w};
+              const float Ds[4] = {D.x, D.y, D.z, D.w};
 #pragma unroll
-            for (int uu = 0; uu < 4; ++uu) {
-              const int e = 4 * e4 + uu;
-              const float y = ex2_fast(fmaf(__uint_as_float(sv[e]), p.scale_log2, -Ls[uu]));
-              const float pe = (full || (e >= lo && e <= hi && kj < p.T)) ? y : 0.f;
-              pt[e] = pe;
-              ds[e] = pe * (__uint_as_float(dv[e]) - Ds[uu]) * p.scale;
+              for (int uu = 0; uu < 4; ++uu) {
+                const int e = 4 * e4 + uu;
+                const float pe = ex2_fast(fmaf(__uint_as_float(sv[e]), p.scale_log2, -Ls[uu]));
+                pt[e] = pe;
+                ds[e] = pe * (__uint_as_float(dv[e]) - Ds[uu]) * p.scale;
+              }
+            }
+          } else {
+            const int lo = kj - q0;  // query >= key
+            const int hi = min(kj + p.W - 1, p.T - 1) - q0;
+#pragma unroll
+            for (int e4 = 0; e4 < 4; ++e4) {
+              const float4 L = *reinterpret_cast<const float4*>(lds + 16 * cs + 4 * e4);
+              const float4 D = *reinterpret_cast<const float4*>(lds + 64 + 16 * cs + 4 * e4);
+              const float Ls[4] = {L.x, L.y, L.z, L.w};
+              const float Ds[4] = {D.x, D.y, D.z, D.w};
+#pragma unroll
+              for (int uu = 0; uu < 4; ++uu) {
+                const int e = 4 * e4 + uu;
+                const float y = ex2_fast(fmaf(__uint_as_float(sv[e]), p.scale_log2, -Ls[uu]));
+                const float pe = (e >= lo && e <= hi && kj < p.T) ? y : 0.f;
+                pt[e] = pe;
+                ds[e] = pe * (__uint_as_float(dv[e]) - Ds[uu]) * p.scale;
+              }
             }
           }
-          // buffer g&1: its MMAs (half-tile g-2) completed before dQ^T_{g-2} was drained
-          store_half_row(smem + C::OFF_P + buf * C::PH, r, pt, half);
-          store_half_row(smem + C::OFF_DS + buf * C::PH, r, ds, half);
+          // buffer g&1: its MMAs (half-tile g-2) completed before dQ^T_{g-2} was drained.
+          // Row r, columns 16*cs .. +15: 16-byte chunks 2*cs and 2*cs + 1 of the 128 B row.
+          uint8_t* prow = smem + C::OFF_P + buf * C::PH + r * 128;
+          uint8_t* drow = smem + C::OFF_DS + buf * C::PH + r * 128;
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int chunk = ((2 * cs + h2) ^ (r & 7)) << 4;
+            *reinterpret_cast<uint4*>(prow + chunk) =
+                make_uint4(pack_bf16(pt[8 * h2 + 0], pt[8 * h2 + 1]), pack_bf16(pt[8 * h2 + 2], pt[8 * h2 + 3]),
+                           pack_bf16(pt[8 * h2 + 4], pt[8 * h2 + 5]), pack_bf16(pt[8 * h2 + 6], pt[8 * h2 + 7]));
+            *reinterpret_cast<uint4*>(drow + chunk) =
+                make_uint4(pack_bf16(ds[8 * h2 + 0], ds[8 * h2 + 1]), pack_bf16(ds[8 * h2 + 2], ds[8 * h2 + 3]),
+                           pack_bf16(ds[8 * h2 + 4], ds[8 * h2 + 5]), pack_bf16(ds[8 * h2 + 6], ds[8 * h2 + 7]));
+          }
           fence_proxy_async_smem();
           tc_fence_before();
           mbar_arrive(&p_full[buf]);
@@ -756,45 +792,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         jp = j;
       }
       // epilogue of the unit: dK, dV rows, rounded to bf16. Each warp's 32 rows
-      // x 64 columns go through its own 4 KiB of the P^T / dS^T buffers (free:
-      // the unit's MMAs are complete and the pending dQ reduce-adds have read
-      // their staging), so that every global store covers four whole 128-byte
-      // row pieces.
+      // x 32 columns go through its own 2 KiB of the P^T buffers (free: the
+      // unit's MMAs are complete and the pending dQ reduce-adds have read their
+      // staging), so that every global store covers whole 64-byte row pieces.
       ok = ok && warp_wait(acc_full, (uint32_t)n & 1u, ab);
       if (lane == 0) bulk_wait_read_all();
-      asm volatile("bar.sync 1, %0;" ::"n"(SOFT_THREADS) : "memory");  // reached by every softmax thread
+      asm volatile("bar.sync 1, %0;" ::"n"(PIPE_SOFT_THREADS) : "memory");  // reached by every softmax thread
       if (ok) {
         tc_fence_after();
-        uint8_t* stg = smem + C::OFF_P + (q4 + 4 * half) * 4096;  // [32 rows][64 bf16], 16-byte chunks swizzled
-        const int64_t tstride = (int64_t)p.H * HD;                // elements between consecutive tokens
-        const int64_t col0 = (int64_t)x.h * HD + 64 * half;
+        uint8_t* stg = smem + C::OFF_P + w16 * 2048;        // [32 rows][32 bf16], 16-byte chunks swizzled
+        const int64_t tstride = (int64_t)p.H * HD;          // elements between consecutive tokens
+        const int64_t col0 = (int64_t)x.h * HD + 32 * cs;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {  // dK, then dV
-          uint32_t v[2][32];
-          const uint32_t tcol = (t == 0 ? C::T_DK : C::T_DV) + 64u * (uint32_t)half;
-          tmem_ld32(tmem + lane_off + tcol, v[0]);
-          tmem_ld32(tmem + lane_off + tcol + 32u, v[1]);
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + (t == 0 ? C::T_DK : C::T_DV) + 32u * (uint32_t)cs, v);
           tmem_wait_ld();
           if (t == 1) {  // both accumulators are in registers or stored: the next unit may overwrite them
             tc_fence_before();
             mbar_arrive(acc_empty);
           }
 #pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8) {
-            const uint32_t* a = &v[c8 >> 2][8 * (c8 & 3)];
-            *reinterpret_cast<uint4*>(stg + lane * 128 + ((c8 ^ (lane & 7)) << 4)) = make_uint4(
-                pack_bf16(__uint_as_float(a[0]), __uint_as_float(a[1])),
-                pack_bf16(__uint_as_float(a[2]), __uint_as_float(a[3])),
-                pack_bf16(__uint_as_float(a[4]), __uint_as_float(a[5])),
-                pack_bf16(__uint_as_float(a[6]), __uint_as_float(a[7])));
-          }
+          for (int c4 = 0; c4 < 4; ++c4)
+            *reinterpret_cast<uint4*>(stg + lane * 64 + ((c4 ^ ((lane >> 1) & 3)) << 4)) = make_uint4(
+                pack_bf16(__uint_as_float(v[8 * c4 + 0]), __uint_as_float(v[8 * c4 + 1])),
+                pack_bf16(__uint_as_float(v[8 * c4 + 2]), __uint_as_float(v[8 * c4 + 3])),
+                pack_bf16(__uint_as_float(v[8 * c4 + 4]), __uint_as_float(v[8 * c4 + 5])),
+                pack_bf16(__uint_as_float(v[8 * c4 + 6]), __uint_as_float(v[8 * c4 + 7])));
           __syncwarp();
           bf16* dst = t == 0 ? p.dk_bar : p.dv_bar;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int r = 4 * i + (lane >> 3), ch = lane & 7;  // row of the warp's 32, 16-byte chunk
-            const uint4 w = *reinterpret_cast<const uint4*>(stg + r * 128 + ((ch ^ (r & 7)) << 4));
-            const int key = x.kt + 32 * q4 + r;
+          for (int i = 0; i < 4; ++i) {
+            const int rr = 8 * i + (lane >> 2), ch = lane & 3;  // row of the warp's 32, 16-byte chunk
+            const uint4 w = *reinterpret_cast<const uint4*>(stg + rr * 64 + ((ch ^ ((rr >> 1) & 3)) << 4));
+            const int key = x.kt + 32 * q4 + rr;
             if (key < p.T)
               *reinterpret_cast<uint4*>(dst + ((int64_t)x.b * p.T + key) * tstride + col0 + 8 * ch) = w;
           }
@@ -804,7 +835,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     // the last drain stages into buffers the epilogue staged through: every warp
     // must be done with its epilogue first
-    asm volatile("bar.sync 1, %0;" ::"n"(SOFT_THREADS) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(PIPE_SOFT_THREADS) : "memory");
     if (g >= 1) drain_dq(g - 1, xp, jp);
     if (lane == 0) bulk_wait_all();  // dQ reductions complete before the CTA leaves
     __syncwarp();
@@ -828,8 +859,8 @@ cudaError_t launch_attn_bwd_tc(const SwaShape& s, const void* q_rot, const void*
   if ((e = make_tmap_tokens(&tk, k_bar, s.B, s.T, s.H, s.hd, 128)) != cudaSuccess) return e;
   if ((e = make_tmap_tokens(&tv, v_bar, s.B, s.T, s.H, s.hd, 128)) != cudaSuccess) return e;
   if ((e = make_tmap_tokens(&tdo, dout, s.B, s.T, s.H, s.hd, 128)) != cudaSuccess) return e;
-  CUtensorMap tdq;
-  if ((e = make_tmap_f32_tokens(&tdq, dq_acc, s.B, s.T, s.H, s.hd)) != cudaSuccess) return e;
+  CUtensorMap tdq;  // dQ reduce-add boxes: 32 query rows (head dim 64), 16 (pipelined kernel)
+  if ((e = make_tmap_f32_tokens(&tdq, dq_acc, s.B, s.T, s.H, s.hd, s.hd == 128 ? 16 : 32)) != cudaSuccess) return e;
   BwdParams p;
   p.B = s.B;
   p.T = s.T;
@@ -857,7 +888,7 @@ cudaError_t launch_attn_bwd_tc(const SwaShape& s, const void* q_rot, const void*
     auto k = attn_bwd_pipe_kernel<128>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PipeCfg<128>::SMEM);
     if (e != cudaSuccess) return e;
-    k<<<pgrid, NUM_THREADS, PipeCfg<128>::SMEM, st>>>(tq64, tk, tv, tdo64, tdq, pp);
+    k<<<pgrid, PIPE_THREADS, PipeCfg<128>::SMEM, st>>>(tq64, tk, tv, tdo64, tdq, pp);
   } else if (s.hd == 64) {
     auto k = attn_bwd_tc_kernel<64>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BwdCfg<64>::SMEM);

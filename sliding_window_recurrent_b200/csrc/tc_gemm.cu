@@ -470,9 +470,9 @@ cudaError_t make_tmap_bf16_2d_plain(CUtensorMap* m, const void* base, uint64_t i
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// fp32 [B,T,H,hd] token tensor, box {32 channels, 1 head, 32 rows, 1}, 128B
-// swizzle: the target of the dQ reduce-add of the attention backward.
-cudaError_t make_tmap_f32_tokens(CUtensorMap* m, void* base, int B, int T, int H, int hd) {
+// fp32 [B,T,H,hd] token tensor, box {32 channels, 1 head, box_rows rows, 1},
+// 128B swizzle: the target of the dQ reduce-add of the attention backward.
+cudaError_t make_tmap_f32_tokens(CUtensorMap* m, void* base, int B, int T, int H, int hd, uint32_t box_rows) {
   std::call_once(g_encode_once, [] {
     cudaDriverEntryPointQueryResult q;
     void* fn = nullptr;
@@ -483,7 +483,7 @@ cudaError_t make_tmap_f32_tokens(CUtensorMap* m, void* base, int B, int T, int H
   if (!g_encode) return cudaErrorNotSupported;
   const cuuint64_t dims[4] = {(cuuint64_t)hd, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
   const cuuint64_t strides[3] = {(cuuint64_t)hd * 4, (cuuint64_t)H * hd * 4, (cuuint64_t)T * H * hd * 4};
-  const cuuint32_t box[4] = {32, 1, 32, 1};
+  const cuuint32_t box[4] = {32, 1, box_rows, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
