@@ -386,21 +386,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // released at once) -> 4 KiB slices of the free P^T/dS^T buffer (g-1)&1 ->
 // one 32 x 32 fp32 TMA reduce-add per warp. Q/dO arrive through a 3-deep
 // ring; K/V once per unit.
-__device__ __forceinline__ void store_half_row(uint8_t* tile, int r, const float* x, int half) {
-  // 32 values (columns 32*half .. +31) of row r of a [rows x 64] bf16 tile in
-  // 128B-swizzled K-major layout (one 64-column chunk, 128 B per row).
-#pragma unroll
-  for (int gg = 0; gg < 4; ++gg) {
-    const int g = half * 4 + gg;
-    uint4 w;
-    w.x = pack_bf16(x[8 * gg + 0], x[8 * gg + 1]);
-    w.y = pack_bf16(x[8 * gg + 2], x[8 * gg + 3]);
-    w.z = pack_bf16(x[8 * gg + 4], x[8 * gg + 5]);
-    w.w = pack_bf16(x[8 * gg + 6], x[8 * gg + 7]);
-    *reinterpret_cast<uint4*>(tile + r * 128 + ((g ^ (r & 7)) << 4)) = w;
-  }
-}
-
 constexpr int PIPE_SOFT_WARPS = 16;                  // 4 per TMEM lane quarter
 constexpr int PIPE_SOFT_THREADS = 32 * PIPE_SOFT_WARPS;
 constexpr int PIPE_THREADS = 64 + PIPE_SOFT_THREADS;  // producer, MMA, softmax warps
