@@ -346,11 +346,19 @@ maglev_status maglev_decode_prefill(const maglev_swa_desc* desc, const void* sav
  *     of position j lives in slot j mod W. The call writes the new entry to slot
  *     p mod W (no other slot changes), then attends over the live slots
  *     (positions max(0, p-W+1)..p).
- *   out [B,H,hd] (out). */
+ *   out [B,H,hd] (out).
+ *   workspace: maglev_decode_workspace_bytes(desc) bytes of scratch. */
 maglev_status maglev_decode_step(const maglev_decode_desc* desc, const int64_t* pos,
                                  const void* q, const void* k, const void* v,
                                  const void* krec_rot, const void* vrec, const float* gate_logits,
-                                 void* k_ring, void* v_ring, void* out, void* stream);
+                                 void* k_ring, void* v_ring, void* out, void* workspace,
+                                 void* stream);
+
+/* Bytes of scratch memory maglev_decode_step needs (its `workspace`): the bf16
+ * path splits each (sequence, head) ring into two halves streamed by separate
+ * CTAs and keeps each half's partial softmax state there; 0 for the fp32 path
+ * (workspace may then be NULL). */
+size_t maglev_decode_workspace_bytes(const maglev_decode_desc* desc);
 
 #ifdef __cplusplus
 }

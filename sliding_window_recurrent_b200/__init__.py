@@ -74,7 +74,8 @@ _SIGS = {
     "maglev_memory_state": ([_I, _I, _I, _F, _I] + [_P] * 5, _I),
     "maglev_memory_state_bwd": ([_I, _I, _I, _I] + [_P] * 7, _I),
     "maglev_decode_mem_project": ([ctypes.POINTER(DecodeDesc)] + [_P] * 7, _I),
-    "maglev_decode_step": ([ctypes.POINTER(DecodeDesc)] + [_P] * 11, _I),
+    "maglev_decode_step": ([ctypes.POINTER(DecodeDesc)] + [_P] * 12, _I),
+    "maglev_decode_workspace_bytes": ([ctypes.POINTER(DecodeDesc)], _SZ),
     "maglev_decode_prefill": ([ctypes.POINTER(SwaDesc)] + [_P] * 4, _I),
     "maglev_wait_selftest": ([_P, _I, _I64, _P], _I),
     "maglev_lm_head_workspace_bytes": ([_I64, _I, _I], _SZ),
@@ -245,11 +246,15 @@ def maglev_decode_mem_project(desc, pos, m_prev, w_mk, w_mv, krec_rot, vrec, str
                                           _ptr(w_mv), _ptr(krec_rot), _ptr(vrec), _stream(stream)))
 
 
-def maglev_decode_step(desc, pos, q, k, v, krec_rot, vrec, gate_logits, k_ring, v_ring, out,
+def maglev_decode_workspace_bytes(desc) -> int:
+    return _lib.maglev_decode_workspace_bytes(ctypes.byref(desc))
+
+
+def maglev_decode_step(desc, pos, q, k, v, krec_rot, vrec, gate_logits, k_ring, v_ring, out, workspace,
                        stream=None):
     _check(_lib.maglev_decode_step(ctypes.byref(desc), _ptr(pos), _ptr(q), _ptr(k), _ptr(v),
                                    _ptr(krec_rot), _ptr(vrec), _ptr(gate_logits), _ptr(k_ring),
-                                   _ptr(v_ring), _ptr(out), _stream(stream)))
+                                   _ptr(v_ring), _ptr(out), _ptr(workspace), _stream(stream)))
 
 
 def maglev_decode_prefill(desc, saved, k_ring, v_ring, stream=None):

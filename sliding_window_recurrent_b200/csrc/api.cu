@@ -859,12 +859,18 @@ maglev_status maglev_decode_prefill(const maglev_swa_desc* d, const void* saved,
   return MAGLEV_OK;
 }
 
+size_t maglev_decode_workspace_bytes(const maglev_decode_desc* d) {
+  if (check_dec(d) != MAGLEV_OK) return 0;
+  return decode_workspace_bytes(dec_shape(d));
+}
+
 maglev_status maglev_decode_step(const maglev_decode_desc* d, const int64_t* pos, const void* q,
                                  const void* k, const void* v, const void* krec_rot,
                                  const void* vrec, const float* gate_logits, void* k_ring,
-                                 void* v_ring, void* out, void* stream) {
+                                 void* v_ring, void* out, void* workspace, void* stream) {
   maglev_status st = check_dec(d);
   if (st != MAGLEV_OK) return st;
+  if (decode_workspace_bytes(dec_shape(d)) > 0) NEED_PTR(workspace);
   NEED_PTR(pos);
   NEED_PTR(q);
   NEED_PTR(k);
@@ -882,8 +888,9 @@ maglev_status maglev_decode_step(const maglev_decode_desc* d, const int64_t* pos
   int* err = nullptr;
   st = status_word(&err, s);
   if (st != MAGLEV_OK) return st;
-  MAGLEV_LAUNCH(1, s, launch_decode_step(dec_shape(d), pos, q, k, v, krec_rot, vrec, gate_logits, k_ring,
-                                          v_ring, out, spin_limit_of(d->spin_limit), err, s),
+  const int nk = decode_workspace_bytes(dec_shape(d)) > 0 ? 2 : 1;  // split step + combine
+  MAGLEV_LAUNCH(nk, s, launch_decode_step(dec_shape(d), pos, q, k, v, krec_rot, vrec, gate_logits, k_ring,
+                                          v_ring, out, workspace, spin_limit_of(d->spin_limit), err, s),
                 "decode_step");
   return MAGLEV_OK;
 }

@@ -209,13 +209,24 @@ struct StreamCfg {
   static constexpr size_t SMEM = OFF_BAR + 256;
 };
 
+// Each (sequence, head) pair's ring is split into ST_SPLIT work units of
+// consecutive 128-slot chunks; units u = pair * ST_SPLIT + part are dealt to
+// the persistent CTAs with a stride of the grid, so that every SM streams about
+// the same number of chunks (whole pairs left the last of five waves 29% full
+// at 64 x 10 pairs on 148 SMs). A unit writes its partial softmax state (max
+// and sum in log2 units, unnormalised output) to the workspace; the unit that
+// holds slot p mod W also writes the new entry to the ring. decode_combine
+// merges the partials of each pair into its output.
+constexpr int ST_SPLIT = 2;
+
 template <int HD>
 __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, DecShape s,
     const int64_t* __restrict__ pos, const bf16* __restrict__ q, const bf16* __restrict__ k,
     const bf16* __restrict__ v, const bf16* __restrict__ krec, const bf16* __restrict__ vrec,
-    const float* __restrict__ gates, bf16* __restrict__ kring, bf16* __restrict__ vring, bf16* __restrict__ out,
-    float scale_log2, int64_t limit_ns, int* err, const __grid_constant__ RopeFreq rf) {
+    const float* __restrict__ gates, bf16* __restrict__ kring, bf16* __restrict__ vring,
+    float* __restrict__ part, int cpu_chunks, float scale_log2, int64_t limit_ns, int* err,
+    const __grid_constant__ RopeFreq rf) {
   using C = StreamCfg<HD>;
   constexpr int HALF = HD / 2;
   constexpr int LPR = HD / 8;                // lanes per row (16 B each)
@@ -235,12 +246,17 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
   __shared__ float wo[ST_WARPS][HD];
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int W = s.W;
-  const int npairs = s.B * s.H;
+  const int nunits = s.B * s.H * ST_SPLIT;
   const tc::Abort ab{abort_flag, err, limit_ns};
   // live slots of pair bh: positions max(0, p-W+1)..p
   auto live_of = [&](int bh) -> int {
     const int64_t p = pos[bh / s.H];
     return p < 0 ? 0 : (p >= W - 1 ? W : (int)p + 1);
+  };
+  // chunks [c0, c1) of unit u (cpu_chunks chunks per unit; may be empty)
+  auto range_of = [&](int u, int nchunks, int* c0, int* c1) {
+    *c0 = min(nchunks, (u % ST_SPLIT) * cpu_chunks);
+    *c1 = min(nchunks, *c0 + cpu_chunks);
   };
 
   if (tid == 0) {
@@ -266,9 +282,11 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
       uint32_t armed = 0, par = 0;
       int L = 0;
       bool ok = true;
-      for (int bh = blockIdx.x; bh < npairs && ok; bh += gridDim.x) {
-        const int nchunks = (live_of(bh) + ST_ROWS - 1) / ST_ROWS;
-        for (int j = 0; j < 2 * nchunks; ++j, ++L) {  // j = 2c: K_c, j = 2c+1: V_c
+      for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+        const int bh = u / ST_SPLIT;
+        int cb, ce;
+        range_of(u, (live_of(bh) + ST_ROWS - 1) / ST_ROWS, &cb, &ce);
+        for (int j = 2 * cb; j < 2 * ce; ++j, ++L) {  // j = 2c: K_c, j = 2c+1: V_c
           const int st = L % C::NSTAGE;
           const uint32_t ph = (uint32_t)(L / C::NSTAGE) & 1u;
           if (!tc::mbar_wait(&empty[st], ph ^ 1u, ab)) {
@@ -297,7 +315,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
     // entry (RoPE of the local key, gated mix), into buffer i&1 once the
     // compute warps are done with pair i-2
     int i = 0;
-    for (int bh = blockIdx.x; bh < npairs; bh += gridDim.x, ++i) {
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++i) {
+      const int bh = u / ST_SPLIT;
       const int buf = i & 1;
       if (i >= 2 && !tc::warp_wait(&prep_empty[buf], (uint32_t)((i - 2) >> 1) & 1u, ab)) break;
       const int h = bh % s.H;
@@ -357,17 +376,18 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
   int L = 0;
   bool ok = true;
   int i = 0;
-  for (int bh = blockIdx.x; bh < npairs; bh += gridDim.x, ++i) {
+  for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++i) {
+    const int bh = u / ST_SPLIT;
     const int buf = i & 1;
-    // the pair's q and new entry are ready (after an abort the pair is skipped)
+    // the pair's q and new entry are ready (after an abort the unit is skipped)
     ok = ok && tc::mbar_wait(&prep_full[buf], (uint32_t)(i >> 1) & 1u, ab);
     const int64_t p = ok ? (int64_t)ppos[buf] : -1;
-    const int64_t tok = (int64_t)bh * HD;
     const int64_t ring = (int64_t)bh * W * HD;
     const bool valid_pos = p >= 0;
     const int slot = valid_pos ? (int)(p % W) : -1;
     const int nlive = valid_pos ? (p >= W - 1 ? W : (int)p + 1) : 0;
-    const int nchunks = (nlive + ST_ROWS - 1) / ST_ROWS;  // as the producer counts them
+    int cb, ce;  // this unit's chunks, as the producer counts them
+    range_of(u, (nlive + ST_ROWS - 1) / ST_ROWS, &cb, &ce);
     const float* kn_b = kn[buf];
     const float* vn_b = vn[buf];
     float qv[8];
@@ -375,7 +395,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
     for (int e = 0; e < 8; ++e) qv[e] = qs[buf][cl + e];
     float m = -INFINITY, l = 0.f;  // log2 units, over the rows this lane-group has seen
     float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int c = 0; c < nchunks; ++c, L += 2) {
+    for (int c = cb; c < ce; ++c, L += 2) {
       if (!ok) continue;  // after an abort the remaining chunks are skipped
       const int sk = L % C::NSTAGE, sv = (L + 1) % C::NSTAGE;
       if (!tc::mbar_wait(&full[sk], (uint32_t)(L / C::NSTAGE) & 1u, ab)) {
@@ -477,7 +497,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
       wl[warp] = ok ? l : 0.f;
     }
     asm volatile("bar.sync 1, %0;" ::"n"(CT) : "memory");  // every warp's partial is in
-    // merge the warps; write the new entry now that the pair's copies have landed
+    // merge the warps into the unit's partial; the unit that holds the slot
+    // writes the new entry now that its copies have landed
     if (tid < HD) {
       float M = -INFINITY;
 #pragma unroll
@@ -489,8 +510,14 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
         Ls += a * wl[w];
         O += a * wo[w][tid];
       }
-      out[tok + tid] = from_f<bf16>(valid_pos && Ls > 0.f ? O / Ls : 0.f);
-      if (valid_pos && ok) {
+      float* pu = part + (int64_t)u * (HD + 2);
+      pu[2 + tid] = O;
+      if (tid == 0) {
+        pu[0] = M;
+        pu[1] = Ls;
+      }
+      const bool has_slot = valid_pos && slot / ST_ROWS >= cb && slot / ST_ROWS < ce;
+      if (has_slot && ok) {
         kring[ring + (int64_t)slot * HD + tid] = from_f<bf16>(kn_b[tid]);
         vring[ring + (int64_t)slot * HD + tid] = from_f<bf16>(vn_b[tid]);
       }
@@ -500,7 +527,34 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
   }
 }
 
+// out[pair] = the ST_SPLIT partials of the pair merged (zeros for an invalid
+// position or an empty window): one block of HD threads per pair.
+template <int HD>
+__global__ void __launch_bounds__(HD) decode_combine_kernel(int npairs, int H, const int64_t* __restrict__ pos,
+                                                            const float* __restrict__ part, bf16* __restrict__ out) {
+  const int bh = blockIdx.x, tid = threadIdx.x;
+  const float* pu = part + (int64_t)bh * ST_SPLIT * (HD + 2);
+  float M = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < ST_SPLIT; ++k) M = fmaxf(M, pu[k * (HD + 2)]);
+  float Ls = 0.f, O = 0.f;
+#pragma unroll
+  for (int k = 0; k < ST_SPLIT; ++k) {
+    const float m = pu[k * (HD + 2)];
+    const float a = m == -INFINITY ? 0.f : tc::ex2_fast(m - M);
+    Ls += a * pu[k * (HD + 2) + 1];
+    O += a * pu[k * (HD + 2) + 2 + tid];
+  }
+  const bool valid = pos[bh / H] >= 0;
+  out[(int64_t)bh * HD + tid] = from_f<bf16>(valid && Ls > 0.f ? O / Ls : 0.f);
+}
+
 }  // namespace
+
+size_t decode_workspace_bytes(const DecShape& s) {
+  if (s.dtype != 1 || (s.hd != 128 && s.hd != 64)) return 0;
+  return (size_t)s.B * s.H * ST_SPLIT * (s.hd + 2) * sizeof(float);
+}
 
 #define MAGLEV_DISPATCH2(DT, HDV, ...)                                                        \
   do {                                                                                       \
@@ -521,7 +575,7 @@ cudaError_t launch_rmsnorm_rope_rows(const DecShape& s, const int64_t* pos, void
 
 cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void* q, const void* k,
                                const void* v, const void* krec, const void* vrec,
-                               const float* gates, void* k_ring, void* v_ring, void* out,
+                               const float* gates, void* k_ring, void* v_ring, void* out, void* workspace,
                                int64_t limit_us, int* err, cudaStream_t st) {
   const float scale = 1.0f / sqrtf((float)s.hd);
   if (s.dtype == 1 && (s.hd == 128 || s.hd == 64)) {
@@ -538,7 +592,10 @@ cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void
     RopeFreq rf{};
     const double base = std::exp2(s.log2_base);
     for (int c = 0; c < s.hd / 2 && c < 64; ++c) rf.inv_freq[c] = std::pow(base, -2.0 * c / s.hd);
-    const unsigned grid = (unsigned)(s.B * s.H < num_sms() ? s.B * s.H : num_sms());  // persistent
+    const int nunits = s.B * s.H * ST_SPLIT;
+    const unsigned grid = (unsigned)(nunits < num_sms() ? nunits : num_sms());  // persistent
+    const int cpu_chunks = ((s.W + ST_ROWS - 1) / ST_ROWS + ST_SPLIT - 1) / ST_SPLIT;
+    float* part = static_cast<float*>(workspace);
     if (s.hd == 128) {
       auto kern = decode_stream_kernel<128>;
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -546,8 +603,10 @@ cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void
       if (e != cudaSuccess) return e;
       kern<<<grid, ST_THREADS, StreamCfg<128>::SMEM, st>>>(tk, tv, s, pos, (const bf16*)q, (const bf16*)k,
                                                                (const bf16*)v, (const bf16*)krec, (const bf16*)vrec,
-                                                               gates, (bf16*)k_ring, (bf16*)v_ring, (bf16*)out,
+                                                               gates, (bf16*)k_ring, (bf16*)v_ring, part, cpu_chunks,
                                                                scale_log2, limit_ns, err, rf);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      decode_combine_kernel<128><<<s.B * s.H, 128, 0, st>>>(s.B * s.H, s.H, pos, part, (bf16*)out);
     } else {
       auto kern = decode_stream_kernel<64>;
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -555,8 +614,10 @@ cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void
       if (e != cudaSuccess) return e;
       kern<<<grid, ST_THREADS, StreamCfg<64>::SMEM, st>>>(tk, tv, s, pos, (const bf16*)q, (const bf16*)k,
                                                               (const bf16*)v, (const bf16*)krec, (const bf16*)vrec,
-                                                              gates, (bf16*)k_ring, (bf16*)v_ring, (bf16*)out,
+                                                              gates, (bf16*)k_ring, (bf16*)v_ring, part, cpu_chunks,
                                                               scale_log2, limit_ns, err, rf);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      decode_combine_kernel<64><<<s.B * s.H, 64, 0, st>>>(s.B * s.H, s.H, pos, part, (bf16*)out);
     }
     return cudaGetLastError();
   }

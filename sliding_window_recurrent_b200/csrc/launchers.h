@@ -83,9 +83,11 @@ struct DecShape {
 };
 cudaError_t launch_rmsnorm_rope_rows(const DecShape& s, const int64_t* pos, void* x,
                                      cudaStream_t st);
+// Scratch of the split decode step: per work unit its partial softmax state.
+size_t decode_workspace_bytes(const DecShape& s);
 cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void* q, const void* k,
                                const void* v, const void* krec, const void* vrec,
-                               const float* gates, void* k_ring, void* v_ring, void* out,
+                               const float* gates, void* k_ring, void* v_ring, void* out, void* workspace,
                                int64_t limit_us, int* err, cudaStream_t st);
 
 // tcgen05 projection GEMMs (bf16 in/out, fp32 accumulation in TMEM).

@@ -9,6 +9,7 @@ import torch
 
 from . import (DecodeDesc, MAGLEV_BF16, MAGLEV_DR_WRITE, MAGLEV_F32, SwaDesc, maglev_consistency_loss,
                maglev_consistency_workspace_bytes, maglev_decode_mem_project, maglev_decode_step,
+               maglev_decode_workspace_bytes,
                maglev_inject_swa_bwd, maglev_inject_swa_fwd, maglev_swa_bwd_workspace_bytes,
                maglev_swa_saved_bytes)
 
@@ -85,11 +86,12 @@ class DecodeLayerState:
         self.krec = torch.empty(B, H, hd, dtype=td, device=device)
         self.vrec = torch.empty(B, H, hd, dtype=td, device=device)
         self.out = torch.empty(B, H, hd, dtype=td, device=device)
+        self.workspace = _bytes(maglev_decode_workspace_bytes(self.desc), device)
 
     def mem_project(self, pos, m_prev, w_mk, w_mv, stream=None):
         maglev_decode_mem_project(self.desc, pos, m_prev, w_mk, w_mv, self.krec, self.vrec, stream)
 
     def step(self, pos, q, k, v, gates, k_ring, v_ring, stream=None):
         maglev_decode_step(self.desc, pos, q, k, v, self.krec, self.vrec, gates, k_ring, v_ring,
-                           self.out, stream)
+                           self.out, self.workspace, stream)
         return self.out

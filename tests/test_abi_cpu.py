@@ -109,15 +109,15 @@ def test_bwd_and_loss_and_decode_validation():
     dd = mg.DecodeDesc(B=2, H=2, hd=64, d_mem=16, window=0, rope_base=1e4, rms_eps=1e-6,
                        inject=1, dtype=mg.MAGLEV_F32, spin_limit=0)
     with pytest.raises(mg.MaglevError):
-        mg.maglev_decode_step(dd, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, stream=0)
+        mg.maglev_decode_step(dd, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, stream=0)
     dd.window = 64
     dd.hd = 80
     with pytest.raises(mg.MaglevError) as e:
-        mg.maglev_decode_step(dd, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, stream=0)
+        mg.maglev_decode_step(dd, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, stream=0)
     assert e.value.status == mg.MAGLEV_ERR_UNSUPPORTED
     dd.hd = 64
     dd.B = 0
-    mg.maglev_decode_step(dd, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, stream=0)
+    mg.maglev_decode_step(dd, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, stream=0)
 
 
 def test_driver_modules_only_call_bound_entry_points():

@@ -54,6 +54,7 @@ class GpuDecoder:
         self.vrec = torch.empty_like(self.krec)
         self.out = [torch.empty_like(self.krec) for _ in range(L)]
         self.rstd = torch.empty(B, dtype=torch.float32, device="cuda")
+        self.ws = torch.empty(max(16, mg.maglev_decode_workspace_bytes(self.desc)), dtype=torch.uint8, device="cuda")
 
     def step(self, pos_t, qkv):
         mg.maglev_decode_mem_project(self.desc, pos_t, self.m, self.wk, self.wv, self.krec, self.vrec)
@@ -61,7 +62,7 @@ class GpuDecoder:
             q, k, v = qkv[l]
             kr, vr = self.rings[l]
             mg.maglev_decode_step(self.desc, pos_t, q, k, v, self.krec, self.vrec, self.gates_d[l], kr, vr,
-                                  self.out[l])
+                                  self.out[l], self.ws)
         mg.maglev_memory_state(B, 1, D, EPS, mg.MAGLEV_BF16, self.out[L - 1], self.m, None, self.rstd)
 
 
