@@ -290,10 +290,11 @@ def capture_graph(torch, fn):
 
 def run_layer_bench(torch, dist, rank, world, dev, steps, warmup, peaks, peaks_src, gpu_uuid):
     """The step's launches are captured in a CUDA graph and replayed for the
-    timed steps (no host gaps between the kernels). The library's per-launch
-    tracing is on while the graph is captured, so the CUDA events around every
-    kernel are nodes of the graph: after the timed replays they hold the
-    per-kernel durations of the last timed step."""
+    timed steps (no host gaps between the kernels). Right after the timed
+    replays, the same number of eager steps run with the library's per-launch
+    CUDA-event tracing on, on the launching stream: they give each kernel's
+    average duration (a kernel's own duration does not depend on the gaps
+    around it)."""
     import sliding_window_recurrent_b200 as mg
     c = LAYER
     x = make_layer_inputs(torch, dev, 1234 + rank)
@@ -302,21 +303,9 @@ def run_layer_bench(torch, dist, rank, world, dev, steps, warmup, peaks, peaks_s
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
-    s = torch.cuda.Stream()  # side-stream run before capture, as torch's graph capture wants
-    s.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(s):
-        step()
-    torch.cuda.current_stream().wait_stream(s)
-    torch.cuda.synchronize()
-    mg.maglev_profile_report()  # drop any earlier records
-    graph = torch.cuda.CUDAGraph()
-    mg.maglev_profile_enable(True)
     n0 = mg.maglev_launch_count()
-    with torch.cuda.graph(graph):
-        step()
-    per_step = mg.maglev_launch_count() - n0
-    mg.maglev_profile_enable(False)
-    torch.cuda.synchronize()
+    graph = capture_graph(torch, step)
+    per_step = (mg.maglev_launch_count() - n0) // 2  # the side-stream run and the capture
     for _ in range(warmup):
         graph.replay()
     torch.cuda.synchronize()
@@ -335,8 +324,14 @@ def run_layer_bench(torch, dist, rank, world, dev, steps, warmup, peaks, peaks_s
     torch.cuda.synchronize()
     launches = per_step * steps
     clocks = sampler.stop()
-    prof = aggregate_profile(mg.maglev_profile_report())  # the last timed replay's kernels
     del graph
+    mg.maglev_profile_report()  # drop any earlier records
+    mg.maglev_profile_enable(True)
+    for _ in range(steps):
+        step()
+    torch.cuda.synchronize()
+    mg.maglev_profile_enable(False)
+    prof = aggregate_profile(mg.maglev_profile_report())
     ms = e0.elapsed_time(e1) / steps
     ms_max = max_over_ranks(dist, ms, dev)
     if dist is not None:
@@ -365,7 +360,7 @@ def run_layer_bench(torch, dist, rank, world, dev, steps, warmup, peaks, peaks_s
         roof["spec_peak"] = SPEC_PEAKS[key]
         roof["frac_of_spec"] = round(roof["achieved"] / SPEC_PEAKS[key], 5)
         roof["avg_launch_ms"] = round(avg_ms, 5)
-        roof["duration_source"] = "CUDA events recorded by nodes of the replayed graph, last timed step"
+        roof["duration_source"] = "CUDA events around each launch, on its stream, over as many eager steps as timed"
         roof["work_per_launch"] = work
     kernels = {n: {"calls": v[0], "ms_total": round(v[1], 4), "share": round(v[1] / sum(w[1] for w in prof.values()), 4)}
                for n, v in sorted(prof.items(), key=lambda kv: -kv[1][1])}
