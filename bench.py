@@ -328,6 +328,9 @@ def run_layer_bench(torch, dist, rank, world, dev, steps, warmup, peaks, peaks_s
     mg.maglev_profile_report()  # drop any earlier records
     mg.maglev_profile_enable(True)
     for _ in range(steps):
+        # the GPU waits ~2 ms first, so that the host has queued the whole step
+        # and each event pair brackets its kernel alone, not a host gap
+        torch.cuda._sleep(4_000_000)
         step()
     torch.cuda.synchronize()
     mg.maglev_profile_enable(False)
@@ -464,6 +467,7 @@ def run_stack_bench(torch, dev, steps, warmup):
     launches = mg.maglev_launch_count() - n0
     ms = e0.elapsed_time(e1) / steps
     mg.maglev_profile_enable(True)
+    torch.cuda._sleep(20_000_000)  # the host queues the traced step while the GPU waits
     step()
     torch.cuda.synchronize()
     mg.maglev_profile_enable(False)
@@ -544,8 +548,10 @@ def run_decode_bench(torch, dev, steps, warmup, peaks):
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
-    # kernel-level roofline of decode_step from a traced eager step
+    # kernel-level roofline of decode_step from a traced eager step, queued
+    # behind a GPU-side delay so that each event pair brackets its kernel alone
     mg.maglev_profile_enable(True)
+    torch.cuda._sleep(4_000_000)
     one_step()
     torch.cuda.synchronize()
     mg.maglev_profile_enable(False)

@@ -347,7 +347,10 @@ maglev_status maglev_decode_prefill(const maglev_swa_desc* desc, const void* sav
  *     p mod W (no other slot changes), then attends over the live slots
  *     (positions max(0, p-W+1)..p).
  *   out [B,H,hd] (out).
- *   workspace: maglev_decode_workspace_bytes(desc) bytes of scratch. */
+ *   workspace: maglev_decode_workspace_bytes(desc) bytes of scratch, zero-filled
+ *     by the caller before its first use; every call that completes leaves it
+ *     zero-filled again (after a call that recorded MAGLEV_ERR_TIMEOUT, fill it
+ *     with zeros again). Calls that share a workspace must not overlap. */
 maglev_status maglev_decode_step(const maglev_decode_desc* desc, const int64_t* pos,
                                  const void* q, const void* k, const void* v,
                                  const void* krec_rot, const void* vrec, const float* gate_logits,
@@ -356,8 +359,8 @@ maglev_status maglev_decode_step(const maglev_decode_desc* desc, const int64_t* 
 
 /* Bytes of scratch memory maglev_decode_step needs (its `workspace`): the bf16
  * path splits each (sequence, head) ring into two halves streamed by separate
- * CTAs and keeps each half's partial softmax state there; 0 for the fp32 path
- * (workspace may then be NULL). */
+ * CTAs and keeps each half's partial softmax state and a per-pair counter
+ * there; 0 for the fp32 path (workspace may then be NULL). */
 size_t maglev_decode_workspace_bytes(const maglev_decode_desc* desc);
 
 #ifdef __cplusplus

@@ -888,8 +888,7 @@ maglev_status maglev_decode_step(const maglev_decode_desc* d, const int64_t* pos
   int* err = nullptr;
   st = status_word(&err, s);
   if (st != MAGLEV_OK) return st;
-  const int nk = decode_workspace_bytes(dec_shape(d)) > 0 ? 2 : 1;  // split step + combine
-  MAGLEV_LAUNCH(nk, s, launch_decode_step(dec_shape(d), pos, q, k, v, krec_rot, vrec, gate_logits, k_ring,
+  MAGLEV_LAUNCH(1, s, launch_decode_step(dec_shape(d), pos, q, k, v, krec_rot, vrec, gate_logits, k_ring,
                                           v_ring, out, workspace, spin_limit_of(d->spin_limit), err, s),
                 "decode_step");
   return MAGLEV_OK;

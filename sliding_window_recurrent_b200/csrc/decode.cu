@@ -214,9 +214,11 @@ struct StreamCfg {
 // the persistent CTAs with a stride of the grid, so that every SM streams about
 // the same number of chunks (whole pairs left the last of five waves 29% full
 // at 64 x 10 pairs on 148 SMs). A unit writes its partial softmax state (max
-// and sum in log2 units, unnormalised output) to the workspace; the unit that
-// holds slot p mod W also writes the new entry to the ring. decode_combine
-// merges the partials of each pair into its output.
+// and sum in log2 units, unnormalised output) to the workspace and counts
+// itself in the pair's counter; the last unit of the pair merges the partials
+// into the output and resets the counter to zero, so the workspace is all
+// zero again when the call ends. The unit that holds slot p mod W also writes
+// the new entry to the ring.
 constexpr int ST_SPLIT = 2;
 
 template <int HD>
@@ -225,8 +227,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
     const int64_t* __restrict__ pos, const bf16* __restrict__ q, const bf16* __restrict__ k,
     const bf16* __restrict__ v, const bf16* __restrict__ krec, const bf16* __restrict__ vrec,
     const float* __restrict__ gates, bf16* __restrict__ kring, bf16* __restrict__ vring,
-    float* __restrict__ part, int cpu_chunks, float scale_log2, int64_t limit_ns, int* err,
-    const __grid_constant__ RopeFreq rf) {
+    float* __restrict__ part, int* __restrict__ counters, bf16* __restrict__ out, int cpu_chunks,
+    float scale_log2, int64_t limit_ns, int* err, const __grid_constant__ RopeFreq rf) {
   using C = StreamCfg<HD>;
   constexpr int HALF = HD / 2;
   constexpr int LPR = HD / 8;                // lanes per row (16 B each)
@@ -244,6 +246,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
   __shared__ long long ppos[2];
   __shared__ float wm[ST_WARPS], wl[ST_WARPS];
   __shared__ float wo[ST_WARPS][HD];
+  __shared__ int last_unit;  // this unit completes its pair
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int W = s.W;
   const int nunits = s.B * s.H * ST_SPLIT;
@@ -521,39 +524,44 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
         kring[ring + (int64_t)slot * HD + tid] = from_f<bf16>(kn_b[tid]);
         vring[ring + (int64_t)slot * HD + tid] = from_f<bf16>(vn_b[tid]);
       }
+      __threadfence();  // the partial is visible before the pair's counter moves
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(CT) : "memory");  // the unit's partial is written and fenced
+    if (tid == 0) last_unit = atomicAdd(&counters[bh], 1) == ST_SPLIT - 1;
+    asm volatile("bar.sync 1, %0;" ::"n"(CT) : "memory");
+    if (last_unit) {  // every unit of the pair has counted itself: merge the partials
+      __threadfence();
+      if (tid < HD) {
+        const float* pp = part + (int64_t)bh * ST_SPLIT * (HD + 2);
+        float M = -INFINITY;
+#pragma unroll
+        for (int k2 = 0; k2 < ST_SPLIT; ++k2) M = fmaxf(M, __ldcg(pp + k2 * (HD + 2)));
+        float Ls = 0.f, O = 0.f;
+#pragma unroll
+        for (int k2 = 0; k2 < ST_SPLIT; ++k2) {
+          const float m2 = __ldcg(pp + k2 * (HD + 2));
+          const float a = m2 == -INFINITY ? 0.f : tc::ex2_fast(m2 - M);
+          Ls += a * __ldcg(pp + k2 * (HD + 2) + 1);
+          O += a * __ldcg(pp + k2 * (HD + 2) + 2 + tid);
+        }
+        out[(int64_t)bh * HD + tid] = from_f<bf16>(valid_pos && Ls > 0.f ? O / Ls : 0.f);
+      }
+      if (tid == 0) counters[bh] = 0;  // ready for the next call
     }
     asm volatile("bar.sync 1, %0;" ::"n"(CT) : "memory");  // q, new entry, partials free again
     if (tid == 0) tc::mbar_arrive(&prep_empty[buf]);           // the prep warp may refill buffer buf
   }
 }
 
-// out[pair] = the ST_SPLIT partials of the pair merged (zeros for an invalid
-// position or an empty window): one block of HD threads per pair.
-template <int HD>
-__global__ void __launch_bounds__(HD) decode_combine_kernel(int npairs, int H, const int64_t* __restrict__ pos,
-                                                            const float* __restrict__ part, bf16* __restrict__ out) {
-  const int bh = blockIdx.x, tid = threadIdx.x;
-  const float* pu = part + (int64_t)bh * ST_SPLIT * (HD + 2);
-  float M = -INFINITY;
-#pragma unroll
-  for (int k = 0; k < ST_SPLIT; ++k) M = fmaxf(M, pu[k * (HD + 2)]);
-  float Ls = 0.f, O = 0.f;
-#pragma unroll
-  for (int k = 0; k < ST_SPLIT; ++k) {
-    const float m = pu[k * (HD + 2)];
-    const float a = m == -INFINITY ? 0.f : tc::ex2_fast(m - M);
-    Ls += a * pu[k * (HD + 2) + 1];
-    O += a * pu[k * (HD + 2) + 2 + tid];
-  }
-  const bool valid = pos[bh / H] >= 0;
-  out[(int64_t)bh * HD + tid] = from_f<bf16>(valid && Ls > 0.f ? O / Ls : 0.f);
-}
-
 }  // namespace
 
+// [B*H*ST_SPLIT][hd + 2] fp32 partials, then [B*H] int pair counters.
+static size_t decode_part_bytes(const DecShape& s) {
+  return ((size_t)s.B * s.H * ST_SPLIT * (s.hd + 2) * sizeof(float) + 255) & ~(size_t)255;
+}
 size_t decode_workspace_bytes(const DecShape& s) {
   if (s.dtype != 1 || (s.hd != 128 && s.hd != 64)) return 0;
-  return (size_t)s.B * s.H * ST_SPLIT * (s.hd + 2) * sizeof(float);
+  return decode_part_bytes(s) + (size_t)s.B * s.H * sizeof(int);
 }
 
 #define MAGLEV_DISPATCH2(DT, HDV, ...)                                                        \
@@ -596,6 +604,7 @@ cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void
     const unsigned grid = (unsigned)(nunits < num_sms() ? nunits : num_sms());  // persistent
     const int cpu_chunks = ((s.W + ST_ROWS - 1) / ST_ROWS + ST_SPLIT - 1) / ST_SPLIT;
     float* part = static_cast<float*>(workspace);
+    int* counters = reinterpret_cast<int*>(static_cast<char*>(workspace) + decode_part_bytes(s));
     if (s.hd == 128) {
       auto kern = decode_stream_kernel<128>;
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -603,10 +612,8 @@ cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void
       if (e != cudaSuccess) return e;
       kern<<<grid, ST_THREADS, StreamCfg<128>::SMEM, st>>>(tk, tv, s, pos, (const bf16*)q, (const bf16*)k,
                                                                (const bf16*)v, (const bf16*)krec, (const bf16*)vrec,
-                                                               gates, (bf16*)k_ring, (bf16*)v_ring, part, cpu_chunks,
-                                                               scale_log2, limit_ns, err, rf);
-      if ((e = cudaGetLastError()) != cudaSuccess) return e;
-      decode_combine_kernel<128><<<s.B * s.H, 128, 0, st>>>(s.B * s.H, s.H, pos, part, (bf16*)out);
+                                                               gates, (bf16*)k_ring, (bf16*)v_ring, part, counters,
+                                                               (bf16*)out, cpu_chunks, scale_log2, limit_ns, err, rf);
     } else {
       auto kern = decode_stream_kernel<64>;
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -614,10 +621,8 @@ cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void
       if (e != cudaSuccess) return e;
       kern<<<grid, ST_THREADS, StreamCfg<64>::SMEM, st>>>(tk, tv, s, pos, (const bf16*)q, (const bf16*)k,
                                                               (const bf16*)v, (const bf16*)krec, (const bf16*)vrec,
-                                                              gates, (bf16*)k_ring, (bf16*)v_ring, part, cpu_chunks,
-                                                              scale_log2, limit_ns, err, rf);
-      if ((e = cudaGetLastError()) != cudaSuccess) return e;
-      decode_combine_kernel<64><<<s.B * s.H, 64, 0, st>>>(s.B * s.H, s.H, pos, part, (bf16*)out);
+                                                              gates, (bf16*)k_ring, (bf16*)v_ring, part, counters,
+                                                              (bf16*)out, cpu_chunks, scale_log2, limit_ns, err, rf);
     }
     return cudaGetLastError();
   }

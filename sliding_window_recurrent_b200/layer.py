@@ -86,7 +86,9 @@ class DecodeLayerState:
         self.krec = torch.empty(B, H, hd, dtype=td, device=device)
         self.vrec = torch.empty(B, H, hd, dtype=td, device=device)
         self.out = torch.empty(B, H, hd, dtype=td, device=device)
-        self.workspace = _bytes(maglev_decode_workspace_bytes(self.desc), device)
+        # zero-filled once; every completed step leaves it zero-filled
+        self.workspace = torch.zeros(max(16, maglev_decode_workspace_bytes(self.desc)), dtype=torch.uint8,
+                                     device=device)
 
     def mem_project(self, pos, m_prev, w_mk, w_mv, stream=None):
         maglev_decode_mem_project(self.desc, pos, m_prev, w_mk, w_mv, self.krec, self.vrec, stream)
