@@ -575,6 +575,45 @@ def run_decode_bench(torch, dev, steps, warmup, peaks):
                         f"{c['first_pos']} (after {warmup + 3} warm-up steps), CUDA graph"}
 
 
+def run_full_causal_bench(torch, dev, steps, warmup):
+    """One of the prefiller's full-causal layers (SLSL 'L': W = T = 2048, no
+    injection), B=8, 10 heads of 128: attention fwd + bwd as a replayed graph.
+    Work: 2,098,176 causal pairs per (b, h) x 4 hd flops forward, 2.5x backward."""
+    from sliding_window_recurrent_b200.layer import InjectedSWALayer
+    B, T, H, hd = STACK["B"], STACK["T"], STACK["H"], STACK["hd"]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1357)
+    rn = lambda: torch.randn(B, T, H, hd, generator=gen, device=dev).to(torch.bfloat16)
+    q, k, v, dout = rn(), rn(), rn(), rn()
+    L = InjectedSWALayer(B, T, H, hd, H * hd, T, dtype="bf16", inject=False, device=dev)
+
+    def step():
+        L.forward(q, k, v)
+        L.backward(k, v, dout)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    graph = capture_graph(torch, step)
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del graph
+    ms = e0.elapsed_time(e1) / steps
+    f = layer_flops(B, T, H, hd, H * hd, T)
+    fl = f["attn_fwd"] + f["attn_bwd"]
+    return {"value": round(fl / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
+            "gflop_per_step": round(fl / 1e9, 2),
+            "workload": f"prefiller full-causal layer (W = T = {T}, no injection) attention fwd+bwd incl. RoPE "
+                        f"and delta/unmix passes, B={B} H={H}x{hd}, bf16, CUDA graph"}
+
+
 def run_lm_head_bench(torch, dev, steps, warmup, peaks):
     """Softcapped LM head + CE, fwd+bwd: logits GEMM with the CE statistics in
     its epilogue, the loss and dz, then dm = dz U and dU = dz^T m."""
@@ -781,6 +820,10 @@ def main():
         dec = run_decode_bench(torch, dev, args.decode_steps, args.warmup, peaks)
         dec["tokens_per_s"] = job_rate(DECODE["B"], world, max_over_ranks(dist, dec["ms_per_step"], dev))
 
+    full = None
+    if not args.no_stack:
+        full = run_full_causal_bench(torch, dev, args.steps, args.warmup)
+
     lmh = None
     if not args.no_lm_head:
         lmh = run_lm_head_bench(torch, dev, max(3, args.steps // 4), args.warmup, peaks)
@@ -810,6 +853,7 @@ def main():
         "clocks": r["clocks"],
         "forward": fwd,
         "stack": stack,
+        "prefiller_full_causal_layer": full,
         "lm_head": lmh,
         "decode": None if dec is None else {
             "value": round(dec["tokens_per_s"], 1), "unit": "tokens/s", "ms_per_step": round(dec["ms_per_step"], 4),

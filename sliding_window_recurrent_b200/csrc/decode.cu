@@ -524,13 +524,17 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
         kring[ring + (int64_t)slot * HD + tid] = from_f<bf16>(kn_b[tid]);
         vring[ring + (int64_t)slot * HD + tid] = from_f<bf16>(vn_b[tid]);
       }
-      __threadfence();  // the partial is visible before the pair's counter moves
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(CT) : "memory");  // the unit's partial is written and fenced
-    if (tid == 0) last_unit = atomicAdd(&counters[bh], 1) == ST_SPLIT - 1;
+    asm volatile("bar.sync 1, %0;" ::"n"(CT) : "memory");  // the unit's partial is written
+    if (tid == 0) {
+      // release: the fence is cumulative, so it orders the CTA's partial (seen
+      // through the barrier) before the count; acquire on the last unit's side
+      __threadfence();
+      last_unit = atomicAdd(&counters[bh], 1) == ST_SPLIT - 1;
+      if (last_unit) __threadfence();
+    }
     asm volatile("bar.sync 1, %0;" ::"n"(CT) : "memory");
     if (last_unit) {  // every unit of the pair has counted itself: merge the partials
-      __threadfence();
       if (tid < HD) {
         const float* pp = part + (int64_t)bh * ST_SPLIT * (HD + 2);
         float M = -INFINITY;

@@ -548,8 +548,10 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
         if (q_armed & (1u << s)) mbar_drain(&q_full[s], (q_par >> s) & 1u, DRAIN_LIMIT_NS);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {
       // ------------------------------------------------------------ MMA issuer
+      // Every lane runs the loop and the waits, so descriptors and counters are
+      // warp-uniform; the elected lane issues each batch of MMAs and commits.
       constexpr uint32_t ID_S = idesc_bf16(128, 64, false, false);  // S^T, dP^T: 128 keys x 64 queries
       constexpr uint32_t ID_KV = idesc_bf16(128, HD, false, true);  // dV, dK: 128 keys x hd
       constexpr uint32_t ID_DQ = idesc_bf16(HD, 64, true, true);    // dQ^T: hd x 64 queries
@@ -561,34 +563,37 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
       // loaded S/dP of half-tile gs-1
       auto issue_sdp = [&](int gs) -> bool {
         const int s = gs % 3;
-        if (!mbar_wait(&q_full[s], (uint32_t)(gs / 3) & 1u, ab)) return false;
-        if (gs >= 1 && !mbar_wait(s_free, (uint32_t)(gs - 1) & 1u, ab)) return false;
+        if (!warp_wait(&q_full[s], (uint32_t)(gs / 3) & 1u, ab)) return false;
+        if (gs >= 1 && !warp_wait(s_free, (uint32_t)(gs - 1) & 1u, ab)) return false;
         tc_fence_after();
         const uint64_t qd = kmajor_desc(smem_u32(smem + C::OFF_Q + s * C::QH), 0);
         const uint64_t dod = kmajor_desc(smem_u32(smem + C::OFF_DO + s * C::QH), 0);
+        if (elect_one()) {
 #pragma unroll
-        for (int k16 = 0; k16 < HD / 16; ++k16) {
-          const uint32_t ka = (uint32_t)(k16 >> 2) * C::KCHUNK + (k16 & 3) * 32u;
-          const uint32_t qa = (uint32_t)(k16 >> 2) * C::QCHUNK + (k16 & 3) * 32u;
-          mma_ss(tmem + C::T_S, desc_at(kd0, ka), desc_at(qd, qa), ID_S, k16 > 0 ? 1u : 0u);
-        }
+          for (int k16 = 0; k16 < HD / 16; ++k16) {
+            const uint32_t ka = (uint32_t)(k16 >> 2) * C::KCHUNK + (k16 & 3) * 32u;
+            const uint32_t qa = (uint32_t)(k16 >> 2) * C::QCHUNK + (k16 & 3) * 32u;
+            mma_ss(tmem + C::T_S, desc_at(kd0, ka), desc_at(qd, qa), ID_S, k16 > 0 ? 1u : 0u);
+          }
 #pragma unroll
-        for (int k16 = 0; k16 < HD / 16; ++k16) {
-          const uint32_t ka = (uint32_t)(k16 >> 2) * C::KCHUNK + (k16 & 3) * 32u;
-          const uint32_t qa = (uint32_t)(k16 >> 2) * C::QCHUNK + (k16 & 3) * 32u;
-          mma_ss(tmem + C::T_DP, desc_at(vd0, ka), desc_at(dod, qa), ID_S, k16 > 0 ? 1u : 0u);
+          for (int k16 = 0; k16 < HD / 16; ++k16) {
+            const uint32_t ka = (uint32_t)(k16 >> 2) * C::KCHUNK + (k16 & 3) * 32u;
+            const uint32_t qa = (uint32_t)(k16 >> 2) * C::QCHUNK + (k16 & 3) * 32u;
+            mma_ss(tmem + C::T_DP, desc_at(vd0, ka), desc_at(dod, qa), ID_S, k16 > 0 ? 1u : 0u);
+          }
+          mma_commit(s_full);
         }
-        mma_commit(s_full);
+        __syncwarp();
         return true;
       };
       // dV, dK and dQ^T of half-tile gr (local index jr of unit nr), once the
       // softmax warps have stored its P / dS
       auto issue_rest = [&](int gr, int jr, int nr) -> bool {
         const int s = gr % 3, buf = gr & 1;
-        if (!mbar_wait(&p_full[buf], (uint32_t)(gr >> 1) & 1u, ab)) return false;
+        if (!warp_wait(&p_full[buf], (uint32_t)(gr >> 1) & 1u, ab)) return false;
         // the first dV/dK of a unit overwrites the accumulators: the previous
         // unit's epilogue must have read them
-        if (jr == 0 && !mbar_wait(acc_empty, ((uint32_t)nr & 1u) ^ 1u, ab)) return false;
+        if (jr == 0 && !warp_wait(acc_empty, ((uint32_t)nr & 1u) ^ 1u, ab)) return false;
         tc_fence_after();
         const uint32_t ds_addr = smem_u32(smem + C::OFF_DS + buf * C::PH);
         const uint64_t pd = kmajor_desc(smem_u32(smem + C::OFF_P + buf * C::PH), 0);
@@ -596,30 +601,36 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
         const uint64_t domn = sw128_desc(smem_u32(smem + C::OFF_DO + s * C::QH), (uint32_t)C::QCHUNK, 1024u);
         const uint64_t qmn = sw128_desc(smem_u32(smem + C::OFF_Q + s * C::QH), (uint32_t)C::QCHUNK, 1024u);
         const uint64_t dsmn = sw128_desc(ds_addr, (uint32_t)C::PH, 1024u);
+        if (elect_one()) {
 #pragma unroll
-        for (int k16 = 0; k16 < 4; ++k16)  // K = 64 queries
-          mma_ss(tmem + C::T_DV, desc_at(pd, k16 * 32u), desc_at(domn, k16 * 2048u), ID_KV,
-                 (jr > 0 || k16 > 0) ? 1u : 0u);
+          for (int k16 = 0; k16 < 4; ++k16)  // K = 64 queries
+            mma_ss(tmem + C::T_DV, desc_at(pd, k16 * 32u), desc_at(domn, k16 * 2048u), ID_KV,
+                   (jr > 0 || k16 > 0) ? 1u : 0u);
 #pragma unroll
-        for (int k16 = 0; k16 < 4; ++k16)
-          mma_ss(tmem + C::T_DK, desc_at(dsd, k16 * 32u), desc_at(qmn, k16 * 2048u), ID_KV,
-                 (jr > 0 || k16 > 0) ? 1u : 0u);
-        mma_commit(&q_empty[s]);
+          for (int k16 = 0; k16 < 4; ++k16)
+            mma_ss(tmem + C::T_DK, desc_at(dsd, k16 * 32u), desc_at(qmn, k16 * 2048u), ID_KV,
+                   (jr > 0 || k16 > 0) ? 1u : 0u);
+          mma_commit(&q_empty[s]);
+        }
+        __syncwarp();
         // DQ[buf] held dQ^T of half-tile gr-2: drained by now in practice
-        if (gr >= 2 && !mbar_wait(&dq_empty[buf], (uint32_t)((gr - 2) >> 1) & 1u, ab)) return false;
+        if (gr >= 2 && !warp_wait(&dq_empty[buf], (uint32_t)((gr - 2) >> 1) & 1u, ab)) return false;
         tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int k16 = 0; k16 < 8; ++k16)  // K = 128 keys
-          mma_ss(tmem + C::T_DQ + 64u * buf, desc_at(kmn, k16 * 2048u), desc_at(dsmn, k16 * 2048u), ID_DQ,
-                 k16 > 0 ? 1u : 0u);
-        mma_commit(&dq_full[buf]);
+          for (int k16 = 0; k16 < 8; ++k16)  // K = 128 keys
+            mma_ss(tmem + C::T_DQ + 64u * buf, desc_at(kmn, k16 * 2048u), desc_at(dsmn, k16 * 2048u), ID_DQ,
+                   k16 > 0 ? 1u : 0u);
+          mma_commit(&dq_full[buf]);
+        }
+        __syncwarp();
         return true;
       };
       int g = 0, n = 0;
       bool ok = true;
       for (int u = kunit_rank(pp, 0); u >= 0 && ok; u = kunit_rank(pp, ++n)) {
         const KUnit x = kunit_of(pp, u);
-        if (!mbar_wait(kv_full, (uint32_t)n & 1u, ab)) break;
+        if (!warp_wait(kv_full, (uint32_t)n & 1u, ab)) break;
         // S/dP of g+1 go to the tensor core ahead of dV/dK/dQ of g
         for (int j = 0; j < x.nh; ++j, ++g) {
           if (!issue_sdp(g) || (j > 0 && !issue_rest(g - 1, j - 1, n))) {
@@ -628,11 +639,17 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
           }
         }
         if (!ok || !issue_rest(g - 1, x.nh - 1, n)) break;
-        mma_commit(acc_full);
-        mma_commit(kv_empty);  // the next unit's K/V may overwrite this one's
+        if (elect_one()) {
+          mma_commit(acc_full);
+          mma_commit(kv_empty);  // the next unit's K/V may overwrite this one's
+        }
+        __syncwarp();
       }
-      mma_commit(drain);
-      mbar_drain(drain, 0, DRAIN_LIMIT_NS);
+      if (elect_one()) {  // the issuing lane's MMAs complete before TMEM is released
+        mma_commit(drain);
+        mbar_drain(drain, 0, DRAIN_LIMIT_NS);
+      }
+      __syncwarp();
     }
   } else {
     // -------------------------------------------------------------- softmax-backward / drains

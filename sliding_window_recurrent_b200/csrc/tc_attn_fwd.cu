@@ -206,8 +206,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {
       // ------------------------------------------------------------ MMA issuer
+      // Every lane runs the loop and the waits (warp-uniform descriptors and
+      // counters); the elected lane issues each batch of MMAs and commits.
       constexpr uint32_t ID_S = idesc_bf16(128, 64, false, false);  // 128 queries x 64 keys
       constexpr uint32_t ID_O = idesc_bf16(128, HD, false, true);   // 128 queries x hd
       // base descriptors: each MMA's operand is a constant offset from these
@@ -216,16 +218,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
       // S_gs = Q K_gs^T into S buffer gs&1; the K slot is released when it completes
       auto issue_s = [&](int gs) -> bool {
         const int s = gs & 1;
-        if (!mbar_wait(&k_full[s], (uint32_t)(gs >> 1) & 1u, ab)) return false;
+        if (!warp_wait(&k_full[s], (uint32_t)(gs >> 1) & 1u, ab)) return false;
         tc_fence_after();
         const uint64_t kd = kmajor_desc(smem_u32(smem + C::OFF_K + s * C::KH), 0);
+        if (elect_one()) {
 #pragma unroll
-        for (int k16 = 0; k16 < HD / 16; ++k16) {
-          mma_ss(tmem + C::T_S + 64u * (uint32_t)s, desc_at(qd, (uint32_t)(k16 >> 2) * C::QCHUNK + (k16 & 3) * 32u),
-                 desc_at(kd, (uint32_t)(k16 >> 2) * C::KCHUNK + (k16 & 3) * 32u), ID_S, k16 > 0 ? 1u : 0u);
+          for (int k16 = 0; k16 < HD / 16; ++k16) {
+            mma_ss(tmem + C::T_S + 64u * (uint32_t)s,
+                   desc_at(qd, (uint32_t)(k16 >> 2) * C::QCHUNK + (k16 & 3) * 32u),
+                   desc_at(kd, (uint32_t)(k16 >> 2) * C::KCHUNK + (k16 & 3) * 32u), ID_S, k16 > 0 ? 1u : 0u);
+          }
+          mma_commit(&s_full[s]);
+          mma_commit(&k_empty[s]);
         }
-        mma_commit(&s_full[s]);
-        mma_commit(&k_empty[s]);
+        __syncwarp();
         return true;
       };
       int g = 0, n = 0;
@@ -234,7 +240,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
         const Unit x = unit_of(p, u);
         // S buffer g&1 was last read by the softmax of half-tile g-2, whose
         // p_full this thread has waited for
-        if (!mbar_wait(q_full, (uint32_t)n & 1u, ab) || !issue_s(g)) break;
+        if (!warp_wait(q_full, (uint32_t)n & 1u, ab) || !issue_s(g)) break;
         for (int j = 0; j < x.n_half; ++j, ++g) {
           if (j + 1 < x.n_half) {
             if (!issue_s(g + 1)) {
@@ -242,33 +248,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
               break;
             }
           } else {
-            mma_commit(q_empty);  // every S of this unit has been issued
+            if (elect_one()) mma_commit(q_empty);  // every S of this unit has been issued
+            __syncwarp();
           }
-          if (!mbar_wait(p_full, (uint32_t)g & 1u, ab)) {
+          if (!warp_wait(p_full, (uint32_t)g & 1u, ab)) {
             ok = false;
             break;
           }
           // the first PV of a unit overwrites O: the previous unit's epilogue must be done
-          if (j == 0 && !mbar_wait(o_empty, ((uint32_t)n & 1u) ^ 1u, ab)) {
+          if (j == 0 && !warp_wait(o_empty, ((uint32_t)n & 1u) ^ 1u, ab)) {
             ok = false;
             break;
           }
-          if (!mbar_wait(&v_full[g & 1], (uint32_t)(g >> 1) & 1u, ab)) {
+          if (!warp_wait(&v_full[g & 1], (uint32_t)(g >> 1) & 1u, ab)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint64_t vmn = sw128_desc(smem_u32(smem + C::OFF_V + (g & 1) * C::KH), (uint32_t)C::KCHUNK, 1024u);
+          if (elect_one()) {
 #pragma unroll
-          for (int k16 = 0; k16 < 4; ++k16)  // K = 64 keys
-            mma_ss(tmem + C::T_O, desc_at(pd, k16 * 32u), desc_at(vmn, k16 * 2048u), ID_O,
-                   (j > 0 || k16 > 0) ? 1u : 0u);
-          mma_commit(&v_empty[g & 1]);
-          mma_commit(pv_done);
+            for (int k16 = 0; k16 < 4; ++k16)  // K = 64 keys
+              mma_ss(tmem + C::T_O, desc_at(pd, k16 * 32u), desc_at(vmn, k16 * 2048u), ID_O,
+                     (j > 0 || k16 > 0) ? 1u : 0u);
+            mma_commit(&v_empty[g & 1]);
+            mma_commit(pv_done);
+          }
+          __syncwarp();
         }
       }
-      mma_commit(drain);
-      mbar_drain(drain, 0, DRAIN_LIMIT_NS);
+      if (elect_one()) {  // the issuing lane's MMAs complete before TMEM is released
+        mma_commit(drain);
+        mbar_drain(drain, 0, DRAIN_LIMIT_NS);
+      }
+      __syncwarp();
     }
   } else {
     // -------------------------------------------------------------- softmax / epilogue

@@ -96,6 +96,19 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, int64
   }
 }
 
+// One lane of the (fully active) warp: the lowest, lane 0. A warp that runs
+// its issue loop on all lanes keeps descriptors and counters warp-uniform and
+// lets this lane alone issue the tensor-core instructions.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

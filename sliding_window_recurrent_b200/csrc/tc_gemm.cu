@@ -202,47 +202,56 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (armed & (1u << s)) mbar_drain(&full[s], (armed_parity >> s) & 1u, DRAIN_LIMIT_NS);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {
       // ------------------------------------------------------------ MMA issuer
+      // Every lane runs the loop and the waits (warp-uniform descriptors and
+      // counters); the elected lane issues each k-block's MMAs and commits.
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, ab)) break;
+        if (!warp_wait(&tempty[acc], acc_phase ^ 1, ab)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * C::ACC_STRIDE);
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&full[stage], phase, ab)) {
+          if (!warp_wait(&full[stage], phase, ab)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t b_addr = smem_u32(sB + stage * C::B_BYTES);
+          if (elect_one()) {
 #pragma unroll
-          for (int k16 = 0; k16 < BK / 16; ++k16) {
-            const uint64_t ad = A_MN ? mnmajor_desc(a_addr, k16) : kmajor_desc(a_addr, k16);
-            const uint64_t bd = B_MN ? mnmajor_desc(b_addr, k16) : kmajor_desc(b_addr, k16);
-            mma_ss(d_tmem, ad, bd, IDESC, (kb > 0 || k16 > 0) ? 1u : 0u);
+            for (int k16 = 0; k16 < BK / 16; ++k16) {
+              const uint64_t ad = A_MN ? mnmajor_desc(a_addr, k16) : kmajor_desc(a_addr, k16);
+              const uint64_t bd = B_MN ? mnmajor_desc(b_addr, k16) : kmajor_desc(b_addr, k16);
+              mma_ss(d_tmem, ad, bd, IDESC, (kb > 0 || k16 > 0) ? 1u : 0u);
+            }
+            mma_commit(&empty[stage]);
           }
-          mma_commit(&empty[stage]);
+          __syncwarp();
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        mma_commit(&tfull[acc]);
+        if (elect_one()) mma_commit(&tfull[acc]);
+        __syncwarp();
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1;
         }
       }
       // all issued MMAs must finish before TMEM is released
-      mma_commit(drain);
-      mbar_drain(drain, 0, DRAIN_LIMIT_NS);
+      if (elect_one()) {
+        mma_commit(drain);
+        mbar_drain(drain, 0, DRAIN_LIMIT_NS);
+      }
+      __syncwarp();
     }
   } else if constexpr (EPI == EPI_CE) {
     // -------------------------------------------------------------- CE epilogue
