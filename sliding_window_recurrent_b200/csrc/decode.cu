@@ -219,7 +219,7 @@ struct StreamCfg {
 // into the output and resets the counter to zero, so the workspace is all
 // zero again when the call ends. The unit that holds slot p mod W also writes
 // the new entry to the ring.
-constexpr int ST_SPLIT = 2;
+constexpr int ST_SPLIT = 2;  // the most units per pair (workspace size)
 
 template <int HD>
 __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
     const int64_t* __restrict__ pos, const bf16* __restrict__ q, const bf16* __restrict__ k,
     const bf16* __restrict__ v, const bf16* __restrict__ krec, const bf16* __restrict__ vrec,
     const float* __restrict__ gates, bf16* __restrict__ kring, bf16* __restrict__ vring,
-    float* __restrict__ part, int* __restrict__ counters, bf16* __restrict__ out, int cpu_chunks,
+    float* __restrict__ part, int* __restrict__ counters, bf16* __restrict__ out, int split, int cpu_chunks,
     float scale_log2, int64_t limit_ns, int* err, const __grid_constant__ RopeFreq rf) {
   using C = StreamCfg<HD>;
   constexpr int HALF = HD / 2;
@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
   __shared__ int last_unit;  // this unit completes its pair
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int W = s.W;
-  const int nunits = s.B * s.H * ST_SPLIT;
+  const int nunits = s.B * s.H * split;
   const tc::Abort ab{abort_flag, err, limit_ns};
   // live slots of pair bh: positions max(0, p-W+1)..p
   auto live_of = [&](int bh) -> int {
@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
   };
   // chunks [c0, c1) of unit u (cpu_chunks chunks per unit; may be empty)
   auto range_of = [&](int u, int nchunks, int* c0, int* c1) {
-    *c0 = min(nchunks, (u % ST_SPLIT) * cpu_chunks);
+    *c0 = min(nchunks, (u % split) * cpu_chunks);
     *c1 = min(nchunks, *c0 + cpu_chunks);
   };
 
@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
       int L = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
-        const int bh = u / ST_SPLIT;
+        const int bh = u / split;
         int cb, ce;
         range_of(u, (live_of(bh) + ST_ROWS - 1) / ST_ROWS, &cb, &ce);
         for (int j = 2 * cb; j < 2 * ce; ++j, ++L) {  // j = 2c: K_c, j = 2c+1: V_c
@@ -319,7 +319,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
     // compute warps are done with pair i-2
     int i = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++i) {
-      const int bh = u / ST_SPLIT;
+      const int bh = u / split;
       const int buf = i & 1;
       if (i >= 2 && !tc::warp_wait(&prep_empty[buf], (uint32_t)((i - 2) >> 1) & 1u, ab)) break;
       const int h = bh % s.H;
@@ -380,7 +380,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
   bool ok = true;
   int i = 0;
   for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++i) {
-    const int bh = u / ST_SPLIT;
+    const int bh = u / split;
     const int buf = i & 1;
     // the pair's q and new entry are ready (after an abort the unit is skipped)
     ok = ok && tc::mbar_wait(&prep_full[buf], (uint32_t)(i >> 1) & 1u, ab);
@@ -513,11 +513,15 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
         Ls += a * wl[w];
         O += a * wo[w][tid];
       }
-      float* pu = part + (int64_t)u * (HD + 2);
-      pu[2 + tid] = O;
-      if (tid == 0) {
-        pu[0] = M;
-        pu[1] = Ls;
+      if (split == 1) {  // the unit is the whole pair
+        out[(int64_t)bh * HD + tid] = from_f<bf16>(valid_pos && Ls > 0.f ? O / Ls : 0.f);
+      } else {
+        float* pu = part + (int64_t)u * (HD + 2);
+        pu[2 + tid] = O;
+        if (tid == 0) {
+          pu[0] = M;
+          pu[1] = Ls;
+        }
       }
       const bool has_slot = valid_pos && slot / ST_ROWS >= cb && slot / ST_ROWS < ce;
       if (has_slot && ok) {
@@ -525,24 +529,25 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
         vring[ring + (int64_t)slot * HD + tid] = from_f<bf16>(vn_b[tid]);
       }
     }
+    if (split > 1) {
     asm volatile("bar.sync 1, %0;" ::"n"(CT) : "memory");  // the unit's partial is written
     if (tid == 0) {
       // release: the fence is cumulative, so it orders the CTA's partial (seen
       // through the barrier) before the count; acquire on the last unit's side
       __threadfence();
-      last_unit = atomicAdd(&counters[bh], 1) == ST_SPLIT - 1;
+      last_unit = atomicAdd(&counters[bh], 1) == split - 1;
       if (last_unit) __threadfence();
     }
     asm volatile("bar.sync 1, %0;" ::"n"(CT) : "memory");
     if (last_unit) {  // every unit of the pair has counted itself: merge the partials
       if (tid < HD) {
-        const float* pp = part + (int64_t)bh * ST_SPLIT * (HD + 2);
+        const float* pp = part + (int64_t)bh * split * (HD + 2);
         float M = -INFINITY;
 #pragma unroll
-        for (int k2 = 0; k2 < ST_SPLIT; ++k2) M = fmaxf(M, __ldcg(pp + k2 * (HD + 2)));
+        for (int k2 = 0; k2 < split; ++k2) M = fmaxf(M, __ldcg(pp + k2 * (HD + 2)));
         float Ls = 0.f, O = 0.f;
 #pragma unroll
-        for (int k2 = 0; k2 < ST_SPLIT; ++k2) {
+        for (int k2 = 0; k2 < split; ++k2) {
           const float m2 = __ldcg(pp + k2 * (HD + 2));
           const float a = m2 == -INFINITY ? 0.f : tc::ex2_fast(m2 - M);
           Ls += a * __ldcg(pp + k2 * (HD + 2) + 1);
@@ -552,12 +557,16 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
       }
       if (tid == 0) counters[bh] = 0;  // ready for the next call
     }
+    }  // split > 1
     asm volatile("bar.sync 1, %0;" ::"n"(CT) : "memory");  // q, new entry, partials free again
     if (tid == 0) tc::mbar_arrive(&prep_empty[buf]);           // the prep warp may refill buffer buf
   }
 }
 
 }  // namespace
+
+// Work units per (sequence, head) pair.
+static int decode_split() { return 1; }
 
 // [B*H*ST_SPLIT][hd + 2] fp32 partials, then [B*H] int pair counters.
 static size_t decode_part_bytes(const DecShape& s) {
@@ -604,9 +613,10 @@ cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void
     RopeFreq rf{};
     const double base = std::exp2(s.log2_base);
     for (int c = 0; c < s.hd / 2 && c < 64; ++c) rf.inv_freq[c] = std::pow(base, -2.0 * c / s.hd);
-    const int nunits = s.B * s.H * ST_SPLIT;
+    const int split = decode_split();
+    const int nunits = s.B * s.H * split;
     const unsigned grid = (unsigned)(nunits < num_sms() ? nunits : num_sms());  // persistent
-    const int cpu_chunks = ((s.W + ST_ROWS - 1) / ST_ROWS + ST_SPLIT - 1) / ST_SPLIT;
+    const int cpu_chunks = ((s.W + ST_ROWS - 1) / ST_ROWS + split - 1) / split;
     float* part = static_cast<float*>(workspace);
     int* counters = reinterpret_cast<int*>(static_cast<char*>(workspace) + decode_part_bytes(s));
     if (s.hd == 128) {
@@ -617,7 +627,7 @@ cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void
       kern<<<grid, ST_THREADS, StreamCfg<128>::SMEM, st>>>(tk, tv, s, pos, (const bf16*)q, (const bf16*)k,
                                                                (const bf16*)v, (const bf16*)krec, (const bf16*)vrec,
                                                                gates, (bf16*)k_ring, (bf16*)v_ring, part, counters,
-                                                               (bf16*)out, cpu_chunks, scale_log2, limit_ns, err, rf);
+                                                               (bf16*)out, split, cpu_chunks, scale_log2, limit_ns, err, rf);
     } else {
       auto kern = decode_stream_kernel<64>;
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -626,7 +636,7 @@ cudaError_t launch_decode_step(const DecShape& s, const int64_t* pos, const void
       kern<<<grid, ST_THREADS, StreamCfg<64>::SMEM, st>>>(tk, tv, s, pos, (const bf16*)q, (const bf16*)k,
                                                               (const bf16*)v, (const bf16*)krec, (const bf16*)vrec,
                                                               gates, (bf16*)k_ring, (bf16*)v_ring, part, counters,
-                                                              (bf16*)out, cpu_chunks, scale_log2, limit_ns, err, rf);
+                                                              (bf16*)out, split, cpu_chunks, scale_log2, limit_ns, err, rf);
     }
     return cudaGetLastError();
   }

@@ -693,8 +693,8 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
       fence_proxy_async_smem();
       __syncwarp();
       const int q0 = xd.kt + 64 * jd + 16 * cs;
-      if (lane == 0 && q0 < p.T) {
-        tma_reduce_add_4d(&tmDQ, slice, 32 * q4, xd.h, q0, xd.b);
+      if (lane == 0) {  // one bulk group per drain, empty past the end of the sequence
+        if (q0 < p.T) tma_reduce_add_4d(&tmDQ, slice, 32 * q4, xd.h, q0, xd.b);
         bulk_commit();
       }
     };
@@ -714,7 +714,9 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
         const int qt = x.kt + 64 * j;
         float* lds = lds_all + buf * 128;  // [0,64) LSE*log2e, [64,128) Delta
         // the reduce-adds of half-tile g-2 have read their staging in buffer g&1
-        if (lane == 0) bulk_wait_read_all();
+        // (each warp's lane 0 commits one bulk group per drain: the latest one,
+        // of half-tile g-1, may still be reading buffer (g-1)&1)
+        if (lane == 0) bulk_wait_read_all_but_last();
         if (st < 128) lds[st] = pre;
         // every softmax thread reaches this barrier on every half-tile, aborted or not
         asm volatile("bar.sync 1, %0;" ::"n"(PIPE_SOFT_THREADS) : "memory");
