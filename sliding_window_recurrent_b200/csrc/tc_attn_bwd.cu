@@ -375,17 +375,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // 64-query half-tiles that see its keys (at most 10 for W = 512); g counts
 // half-tiles over all of the CTA's units.
 //   S^T_g  = K Q_g^T, dP^T_g = V dO_g^T   128 keys x 64 queries, TMEM S, DP (one each)
-//   P^T_g, dS^T_g                          bf16, shared memory buffer g&1
+//   P^T_g                                  bf16, TMEM PT[g&1] (the A operand of dV)
+//   dS^T_g                                 bf16, shared memory buffer g&1
 //   dV += P^T_g dO_g, dK += dS^T_g Q_g     TMEM accumulators (whole unit)
-//   dQ^T_g = K^T dS^T_g                    128 channels x 64 queries, TMEM DQ[g&1]
+//   dQ^T_g = K^T dS^T_g                    128 channels x 64 queries, TMEM DQ
 // The softmax warps release S / dP as soon as their tcgen05.ld of half-tile g
 // has completed, so the MMA warp issues S/dP of g+1 at once and the tensor
 // core computes it (and then dV/dK/dQ of g) while the softmax warps turn g's
 // scores into P and dS. After storing P/dS of g the softmax warps drain
-// dQ^T_{g-1} from its own TMEM columns: TMEM -> registers (DQ[(g-1)&1]
-// released at once) -> 4 KiB slices of the free P^T/dS^T buffer (g-1)&1 ->
-// one 32 x 32 fp32 TMA reduce-add per warp. Q/dO arrive through a 3-deep
-// ring; K/V once per unit.
+// dQ^T_{g-1}: TMEM -> registers (DQ released at once) -> the warp's 2 KiB
+// slice of a staging buffer of its own -> one 16 x 32 fp32 TMA reduce-add per
+// warp. An SM's reductions to global memory drain at only ~25 B/clk (the 32
+// KiB of a half-tile take ~1300 cycles); a slice is next written a whole
+// half-tile later. Q/dO arrive through a 3-deep ring; K/V once per unit.
 constexpr int PIPE_SOFT_WARPS = 16;                  // 4 per TMEM lane quarter
 constexpr int PIPE_SOFT_THREADS = 32 * PIPE_SOFT_WARPS;
 constexpr int PIPE_THREADS = 64 + PIPE_SOFT_THREADS;  // producer, MMA, softmax warps
@@ -404,13 +406,13 @@ struct PipeCfg {
   static constexpr int OFF_V = KV_TILE;
   static constexpr int OFF_Q = 2 * KV_TILE;
   static constexpr int OFF_DO = OFF_Q + NQ * QH;
-  static constexpr int OFF_P = OFF_DO + NQ * QH;  // [2]
-  static constexpr int OFF_DS = OFF_P + 2 * PH;   // [2]
+  static constexpr int OFF_X = OFF_DO + NQ * QH;  // dQ^T staging: 16 slices of 16 queries x 32 channels fp32
+  static constexpr int OFF_DS = OFF_X + 2 * PH;   // [2]
   static constexpr int OFF_LD = OFF_DS + 2 * PH;  // [2][128] floats: LSE*log2e (64), Delta (64)
   static constexpr int OFF_BAR = OFF_LD + 2 * 128 * 4;
   static constexpr size_t SMEM = OFF_BAR + 256;   // base is 1024-aligned (checked in the kernel)
-  // TMEM columns: S 64, dP 64, dQ 2 x 64, dV 128, dK 128
-  static constexpr uint32_t T_S = 0, T_DP = 64, T_DQ = 128, T_DV = 256, T_DK = 384;
+  // TMEM columns: S 64, dP 64, dQ 64, P^T 2 x 32 (bf16 pairs), dV 128, dK 128
+  static constexpr uint32_t T_S = 0, T_DP = 64, T_DQ = 128, T_PT = 192, T_DV = 256, T_DK = 384;
 };
 
 struct PipeParams {
@@ -461,8 +463,8 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
   uint64_t* s_full = bars + 8;     // S / dP of the current half-tile computed
   uint64_t* s_free = bars + 9;     // ... and loaded by every softmax thread
   uint64_t* p_full = bars + 10;    // [2]
-  uint64_t* dq_full = bars + 12;   // [2]
-  uint64_t* dq_empty = bars + 14;  // [2]
+  uint64_t* dq_full = bars + 12;
+  uint64_t* dq_empty = bars + 14;
   uint64_t* acc_full = bars + 16;
   uint64_t* acc_empty = bars + 17;
   uint64_t* drain = bars + 18;
@@ -481,11 +483,9 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, PIPE_SOFT_THREADS);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&p_full[s], PIPE_SOFT_THREADS);
-      mbar_init(&dq_full[s], 1);
-      mbar_init(&dq_empty[s], PIPE_SOFT_THREADS);
-    }
+    for (int s = 0; s < 2; ++s) mbar_init(&p_full[s], PIPE_SOFT_THREADS);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_empty, PIPE_SOFT_THREADS);
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, PIPE_SOFT_THREADS);
     mbar_init(drain, 1);
@@ -587,7 +587,7 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
         return true;
       };
       // dV, dK and dQ^T of half-tile gr (local index jr of unit nr), once the
-      // softmax warps have stored its P / dS
+      // softmax warps have stored its P^T (TMEM) / dS^T (shared memory)
       auto issue_rest = [&](int gr, int jr, int nr) -> bool {
         const int s = gr % 3, buf = gr & 1;
         if (!warp_wait(&p_full[buf], (uint32_t)(gr >> 1) & 1u, ab)) return false;
@@ -596,15 +596,15 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
         if (jr == 0 && !warp_wait(acc_empty, ((uint32_t)nr & 1u) ^ 1u, ab)) return false;
         tc_fence_after();
         const uint32_t ds_addr = smem_u32(smem + C::OFF_DS + buf * C::PH);
-        const uint64_t pd = kmajor_desc(smem_u32(smem + C::OFF_P + buf * C::PH), 0);
+        const uint32_t pt = tmem + C::T_PT + 32u * (uint32_t)buf;
         const uint64_t dsd = kmajor_desc(ds_addr, 0);
         const uint64_t domn = sw128_desc(smem_u32(smem + C::OFF_DO + s * C::QH), (uint32_t)C::QCHUNK, 1024u);
         const uint64_t qmn = sw128_desc(smem_u32(smem + C::OFF_Q + s * C::QH), (uint32_t)C::QCHUNK, 1024u);
         const uint64_t dsmn = sw128_desc(ds_addr, (uint32_t)C::PH, 1024u);
         if (elect_one()) {
 #pragma unroll
-          for (int k16 = 0; k16 < 4; ++k16)  // K = 64 queries
-            mma_ss(tmem + C::T_DV, desc_at(pd, k16 * 32u), desc_at(domn, k16 * 2048u), ID_KV,
+          for (int k16 = 0; k16 < 4; ++k16)  // K = 64 queries, 8 TMEM columns each
+            mma_ts(tmem + C::T_DV, pt + 8u * (uint32_t)k16, desc_at(domn, k16 * 2048u), ID_KV,
                    (jr > 0 || k16 > 0) ? 1u : 0u);
 #pragma unroll
           for (int k16 = 0; k16 < 4; ++k16)
@@ -613,15 +613,15 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
           mma_commit(&q_empty[s]);
         }
         __syncwarp();
-        // DQ[buf] held dQ^T of half-tile gr-2: drained by now in practice
-        if (gr >= 2 && !warp_wait(&dq_empty[buf], (uint32_t)((gr - 2) >> 1) & 1u, ab)) return false;
+        // DQ held dQ^T of half-tile gr-1, drained while dV / dK of gr run
+        if (gr >= 1 && !warp_wait(dq_empty, (uint32_t)(gr - 1) & 1u, ab)) return false;
         tc_fence_after();
         if (elect_one()) {
 #pragma unroll
           for (int k16 = 0; k16 < 8; ++k16)  // K = 128 keys
-            mma_ss(tmem + C::T_DQ + 64u * buf, desc_at(kmn, k16 * 2048u), desc_at(dsmn, k16 * 2048u), ID_DQ,
+            mma_ss(tmem + C::T_DQ, desc_at(kmn, k16 * 2048u), desc_at(dsmn, k16 * 2048u), ID_DQ,
                    k16 > 0 ? 1u : 0u);
-          mma_commit(&dq_full[buf]);
+          mma_commit(dq_full);
         }
         __syncwarp();
         return true;
@@ -664,37 +664,43 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     float* lds_all = reinterpret_cast<float*>(smem + C::OFF_LD);
     bool ok = true;
-    // LSE / Delta of half-tile g, loaded one half-tile ahead by threads 0..127
+    // LSE / Delta of half-tile g, loaded one half-tile ahead by threads 0..127.
+    // The loaded value is not touched until it is stored to shared memory a
+    // whole softmax step later, so no thread stalls on the load's latency.
     float pre = 0.f;
     auto fetch = [&](const KUnit& x, int j) {
       if (st < 128) {
         const int qi = x.kt + 64 * j + (st & 63);
         const int64_t lrow = ((int64_t)x.b * p.H + x.h) * p.T;
-        pre = qi < p.T ? (st < 64 ? p.lse[lrow + qi] * LOG2E : p.delta[lrow + qi]) : 0.f;
+        pre = 0.f;
+        if (qi < p.T) pre = __ldg((st < 64 ? p.lse : p.delta) + lrow + qi);
       }
     };
+    auto pre_scaled = [&]() { return st < 64 ? pre * LOG2E : pre; };  // LSE in log2 units
     // dQ^T of half-tile gd (unit xd, its local index jd): lanes are channels,
     // this warp's 16 columns are queries xd.kt + 64*jd + 16*cs ...
     auto drain_dq = [&](int gd, const KUnit& xd, int jd) {
-      const int buf = gd & 1;
-      ok = ok && warp_wait(&dq_full[buf], (uint32_t)(gd >> 1) & 1u, ab);
+      ok = ok && warp_wait(dq_full, (uint32_t)gd & 1u, ab);
       if (!ok) return;
       tc_fence_after();
       uint32_t v[16];
-      tmem_ld16(tmem + lane_off + C::T_DQ + 64u * (uint32_t)buf + 16u * (uint32_t)cs, v);
+      tmem_ld16(tmem + lane_off + C::T_DQ + 16u * (uint32_t)cs, v);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(&dq_empty[buf]);  // DQ[buf] may take dQ^T of half-tile gd + 2
+      mbar_arrive(dq_empty);  // DQ may take dQ^T of half-tile gd + 1
+      // the warp's reduce-add of half-tile gd-1 has read its slice
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
       // box of 16 query rows x 32 channels (128 B rows, 16-byte chunks swizzled by row)
-      uint8_t* slice = smem + (w16 < 8 ? C::OFF_P : C::OFF_DS) + buf * C::PH + (w16 & 7) * 2048;
+      uint8_t* slice = smem + C::OFF_X + w16 * 2048;
 #pragma unroll
       for (int c = 0; c < 16; ++c)
         *reinterpret_cast<uint32_t*>(slice + c * 128 + ((((lane >> 2) ^ (c & 7))) << 4) + (lane & 3) * 4) = v[c];
       fence_proxy_async_smem();
       __syncwarp();
       const int q0 = xd.kt + 64 * jd + 16 * cs;
-      if (lane == 0) {  // one bulk group per drain, empty past the end of the sequence
-        if (q0 < p.T) tma_reduce_add_4d(&tmDQ, slice, 32 * q4, xd.h, q0, xd.b);
+      if (lane == 0 && q0 < p.T) {  // none past the end of the sequence
+        tma_reduce_add_4d(&tmDQ, slice, 32 * q4, xd.h, q0, xd.b);
         bulk_commit();
       }
     };
@@ -704,6 +710,8 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
     {
       const int u0 = kunit_rank(pp, 0);
       if (u0 >= 0) fetch(kunit_of(pp, u0), 0);
+      if (st < 128) lds_all[st] = pre_scaled();  // LSE / Delta of half-tile 0
+      asm volatile("bar.sync 1, %0;" ::"n"(PIPE_SOFT_THREADS) : "memory");
     }
     for (int u = kunit_rank(pp, 0); u >= 0; u = kunit_rank(pp, ++n)) {
       const KUnit x = kunit_of(pp, u);
@@ -712,21 +720,15 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
       for (int j = 0; j < x.nh; ++j, ++g) {
         const int buf = g & 1;
         const int qt = x.kt + 64 * j;
-        float* lds = lds_all + buf * 128;  // [0,64) LSE*log2e, [64,128) Delta
-        // the reduce-adds of half-tile g-2 have read their staging in buffer g&1
-        // (each warp's lane 0 commits one bulk group per drain: the latest one,
-        // of half-tile g-1, may still be reading buffer (g-1)&1)
-        if (lane == 0) bulk_wait_read_all_but_last();
-        if (st < 128) lds[st] = pre;
-        // every softmax thread reaches this barrier on every half-tile, aborted or not
-        asm volatile("bar.sync 1, %0;" ::"n"(PIPE_SOFT_THREADS) : "memory");
-        if (j + 1 < x.nh) {
+        const float* lds = lds_all + buf * 128;  // [0,64) LSE*log2e, [64,128) Delta
+        if (j + 1 < x.nh) {  // LSE / Delta of half-tile g+1, stored below
           fetch(x, j + 1);
         } else {
           const int un = kunit_rank(pp, n + 1);
           if (un >= 0) fetch(kunit_of(pp, un), 0);
         }
         ok = ok && warp_wait(s_full, (uint32_t)g & 1u, ab);
+        float pt[16], ds[16];
         if (ok) {
           tc_fence_after();
           uint32_t sv[16], dv[16];
@@ -738,7 +740,6 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
           const int q0 = qt + 16 * cs;  // first query column of this warp
           // every (key, query) of this warp's 32 x 16 block inside the window
           const bool full = q0 >= kw + 31 && q0 + 15 <= kw + p.W - 1 && q0 + 15 <= p.T - 1 && kw + 31 < p.T;
-          float pt[16], ds[16];
           if (full) {
 #pragma unroll
             for (int e4 = 0; e4 < 4; ++e4) {
@@ -773,20 +774,31 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
               }
             }
           }
-          // buffer g&1: its MMAs (half-tile g-2) completed before dQ^T_{g-2} was drained.
-          // Row r, columns 16*cs .. +15: 16-byte chunks 2*cs and 2*cs + 1 of the 128 B row.
-          uint8_t* prow = smem + C::OFF_P + buf * C::PH + r * 128;
+        }
+        // Buffers g&1 (P^T in TMEM, dS^T in shared memory) held half-tile
+        // g-2, whose MMAs completed before dQ^T_{g-2} was drained. This
+        // barrier publishes LSE / Delta of g+1 into the other lds buffer, last
+        // read by every thread before the previous barrier.
+        if (st < 128) lds_all[(buf ^ 1) * 128 + st] = pre_scaled();
+        // every softmax thread reaches this barrier on every half-tile, aborted or not
+        asm volatile("bar.sync 1, %0;" ::"n"(PIPE_SOFT_THREADS) : "memory");
+        if (ok) {
+          // P^T row r (this lane's key), queries 16*cs .. +15 as 8 bf16 pairs
+          // in TMEM columns PT[buf] + 8*cs ..; dS^T into shared memory: 16-byte
+          // chunks 2*cs and 2*cs + 1 of the 128 B row.
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) pk[i] = pack_bf16(pt[2 * i], pt[2 * i + 1]);
+          tmem_st8(tmem + lane_off + C::T_PT + 32u * (uint32_t)buf + 8u * (uint32_t)cs, pk);
           uint8_t* drow = smem + C::OFF_DS + buf * C::PH + r * 128;
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
             const int chunk = ((2 * cs + h2) ^ (r & 7)) << 4;
-            *reinterpret_cast<uint4*>(prow + chunk) =
-                make_uint4(pack_bf16(pt[8 * h2 + 0], pt[8 * h2 + 1]), pack_bf16(pt[8 * h2 + 2], pt[8 * h2 + 3]),
-                           pack_bf16(pt[8 * h2 + 4], pt[8 * h2 + 5]), pack_bf16(pt[8 * h2 + 6], pt[8 * h2 + 7]));
             *reinterpret_cast<uint4*>(drow + chunk) =
                 make_uint4(pack_bf16(ds[8 * h2 + 0], ds[8 * h2 + 1]), pack_bf16(ds[8 * h2 + 2], ds[8 * h2 + 3]),
                            pack_bf16(ds[8 * h2 + 4], ds[8 * h2 + 5]), pack_bf16(ds[8 * h2 + 6], ds[8 * h2 + 7]));
           }
+          tmem_wait_st();
           fence_proxy_async_smem();
           tc_fence_before();
           mbar_arrive(&p_full[buf]);
@@ -796,15 +808,14 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
         jp = j;
       }
       // epilogue of the unit: dK, dV rows, rounded to bf16. Each warp's 32 rows
-      // x 32 columns go through its own 2 KiB of the P^T buffers (free: the
-      // unit's MMAs are complete and the pending dQ reduce-adds have read their
-      // staging), so that every global store covers whole 64-byte row pieces.
+      // x 32 columns go through its own 2 KiB of the dS^T buffers (free: the
+      // unit's MMAs are complete), so that every global store covers whole
+      // 64-byte row pieces.
       ok = ok && warp_wait(acc_full, (uint32_t)n & 1u, ab);
-      if (lane == 0) bulk_wait_read_all();
       asm volatile("bar.sync 1, %0;" ::"n"(PIPE_SOFT_THREADS) : "memory");  // reached by every softmax thread
       if (ok) {
         tc_fence_after();
-        uint8_t* stg = smem + C::OFF_P + w16 * 2048;        // [32 rows][32 bf16], 16-byte chunks swizzled
+        uint8_t* stg = smem + C::OFF_DS + w16 * 2048;       // [32 rows][32 bf16], 16-byte chunks swizzled
         const int64_t tstride = (int64_t)p.H * HD;          // elements between consecutive tokens
         const int64_t col0 = (int64_t)x.h * HD + 32 * cs;
 #pragma unroll
@@ -837,9 +848,6 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
         }
       }
     }
-    // the last drain stages into buffers the epilogue staged through: every warp
-    // must be done with its epilogue first
-    asm volatile("bar.sync 1, %0;" ::"n"(PIPE_SOFT_THREADS) : "memory");
     if (g >= 1) drain_dq(g - 1, xp, jp);
     if (lane == 0) bulk_wait_all();  // dQ reductions complete before the CTA leaves
     __syncwarp();

@@ -210,3 +210,45 @@ def test_prefill_from_prompt_then_decode(T):
                kr, vr)
     torch.cuda.synchronize()
     assert_close(host(o), f["out"][:, T], "bf16", f"decode at {T} after prefill")
+
+
+def test_decode_checkpoint_restore_bit_identical():
+    """The whole decode state is the rings, the position and m_{p-1}: run 3
+    steps, copy that state out, run 6 more (crossing p = 511 -> 512), restore
+    the copy and run the same 6 steps again. Every output and the final state
+    must be bit-identical between the two runs."""
+    seed = 47
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(seed)
+    m0 = synth.normal(seed, synth.TID["m_prev"], (B, D), sub=1 << 29)
+    G = GpuDecoder(seed, dev(m0))
+
+    def inputs():
+        return [tuple(torch.randn(B, H, HD, generator=gen, device="cuda").to(torch.bfloat16) for _ in range(3))
+                for _ in range(L)]
+
+    p0 = 507
+    for s in range(3):
+        G.step(torch.full((B,), p0 + s, dtype=torch.int64, device="cuda"), inputs())
+    saved = ([(kr.clone(), vr.clone()) for kr, vr in G.rings], G.m.clone(), p0 + 3)
+    steps = [inputs() for _ in range(6)]
+
+    def run():
+        outs = []
+        for s, qkv in enumerate(steps):
+            G.step(torch.full((B,), saved[2] + s, dtype=torch.int64, device="cuda"), qkv)
+            outs.append([o.clone() for o in G.out] + [G.m.clone()])
+        return outs, [(kr.clone(), vr.clone()) for kr, vr in G.rings]
+
+    first, rings1 = run()
+    for (kr, vr), (k0, v0) in zip(G.rings, saved[0]):
+        kr.copy_(k0)
+        vr.copy_(v0)
+    G.m.copy_(saved[1])
+    second, rings2 = run()
+    torch.cuda.synchronize()
+    for s, (a, b) in enumerate(zip(first, second)):
+        for i, (x, y) in enumerate(zip(a, b)):
+            assert torch.equal(x, y), (s, i)
+    for (k1, v1), (k2, v2) in zip(rings1, rings2):
+        assert torch.equal(k1, k2) and torch.equal(v1, v2)
