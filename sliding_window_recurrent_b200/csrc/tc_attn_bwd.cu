@@ -408,8 +408,8 @@ struct PipeCfg {
   static constexpr int OFF_DO = OFF_Q + NQ * QH;
   static constexpr int OFF_X = OFF_DO + NQ * QH;  // dQ^T staging: 16 slices of 16 queries x 32 channels fp32
   static constexpr int OFF_DS = OFF_X + 2 * PH;   // [2]
-  static constexpr int OFF_LD = OFF_DS + 2 * PH;  // [2][128] floats: LSE*log2e (64), Delta (64)
-  static constexpr int OFF_BAR = OFF_LD + 2 * 128 * 4;
+  static constexpr int OFF_LD = OFF_DS + 2 * PH;  // [16 warps][32] floats: LSE*log2e (16), Delta (16)
+  static constexpr int OFF_BAR = OFF_LD + 16 * 32 * 4;
   static constexpr size_t SMEM = OFF_BAR + 256;   // base is 1024-aligned (checked in the kernel)
   // TMEM columns: S 64, dP 64, dQ 64, P^T 2 x 32 (bf16 pairs), dV 128, dK 128
   static constexpr uint32_t T_S = 0, T_DP = 64, T_DQ = 128, T_PT = 192, T_DV = 256, T_DK = 384;
@@ -659,24 +659,27 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
     const int q4 = warp & 3;
     const int cs = (warp - 2) >> 2;
     const int r = q4 * 32 + lane;      // TMEM lane: key row (S^T, dV, dK) / channel (dQ^T)
-    const int st = threadIdx.x - 64;   // 0..511 among the softmax threads
     const int w16 = q4 + 4 * cs;       // this warp's 2 KiB staging slice
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    float* lds_all = reinterpret_cast<float*>(smem + C::OFF_LD);
+    // This warp's LSE (log2 units) and Delta of its 16 query columns of the
+    // current half-tile: lane l < 16 holds column l's LSE, lane 16 + l its Delta.
+    float* lds = reinterpret_cast<float*>(smem + C::OFF_LD) + 32 * w16;
     bool ok = true;
-    // LSE / Delta of half-tile g, loaded one half-tile ahead by threads 0..127.
-    // The loaded value is not touched until it is stored to shared memory a
-    // whole softmax step later, so no thread stalls on the load's latency.
+    // Each lane loads its value of the next half-tile one half-tile ahead and
+    // touches it only after the current half-tile's math, so no thread stalls
+    // on the load's latency and no warp waits for another.
     float pre = 0.f;
     auto fetch = [&](const KUnit& x, int j) {
-      if (st < 128) {
-        const int qi = x.kt + 64 * j + (st & 63);
-        const int64_t lrow = ((int64_t)x.b * p.H + x.h) * p.T;
-        pre = 0.f;
-        if (qi < p.T) pre = __ldg((st < 64 ? p.lse : p.delta) + lrow + qi);
-      }
+      const int qi = x.kt + 64 * j + 16 * cs + (lane & 15);
+      const int64_t lrow = ((int64_t)x.b * p.H + x.h) * p.T;
+      pre = 0.f;
+      if (qi < p.T) pre = __ldg((lane < 16 ? p.lse : p.delta) + lrow + qi);
     };
-    auto pre_scaled = [&]() { return st < 64 ? pre * LOG2E : pre; };  // LSE in log2 units
+    auto publish = [&]() {  // every lane of the warp has finished reading the previous values
+      __syncwarp();
+      lds[lane] = lane < 16 ? pre * LOG2E : pre;
+      __syncwarp();
+    };
     // dQ^T of half-tile gd (unit xd, its local index jd): lanes are channels,
     // this warp's 16 columns are queries xd.kt + 64*jd + 16*cs ...
     auto drain_dq = [&](int gd, const KUnit& xd, int jd) {
@@ -710,8 +713,7 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
     {
       const int u0 = kunit_rank(pp, 0);
       if (u0 >= 0) fetch(kunit_of(pp, u0), 0);
-      if (st < 128) lds_all[st] = pre_scaled();  // LSE / Delta of half-tile 0
-      asm volatile("bar.sync 1, %0;" ::"n"(PIPE_SOFT_THREADS) : "memory");
+      publish();  // LSE / Delta of half-tile 0
     }
     for (int u = kunit_rank(pp, 0); u >= 0; u = kunit_rank(pp, ++n)) {
       const KUnit x = kunit_of(pp, u);
@@ -720,7 +722,6 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
       for (int j = 0; j < x.nh; ++j, ++g) {
         const int buf = g & 1;
         const int qt = x.kt + 64 * j;
-        const float* lds = lds_all + buf * 128;  // [0,64) LSE*log2e, [64,128) Delta
         if (j + 1 < x.nh) {  // LSE / Delta of half-tile g+1, stored below
           fetch(x, j + 1);
         } else {
@@ -743,8 +744,8 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
           if (full) {
 #pragma unroll
             for (int e4 = 0; e4 < 4; ++e4) {
-              const float4 L = *reinterpret_cast<const float4*>(lds + 16 * cs + 4 * e4);
-              const float4 D = *reinterpret_cast<const float4*>(lds + 64 + 16 * cs + 4 * e4);
+              const float4 L = *reinterpret_cast<const float4*>(lds + 4 * e4);
+              const float4 D = *reinterpret_cast<const float4*>(lds + 16 + 4 * e4);
               const float Ls[4] = {L.x, L.y, L.z, L.w};
               const float Ds[4] = {D.x, D.y, D.z, D.w};
 #pragma unroll
@@ -760,8 +761,8 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
             const int hi = min(kj + p.W - 1, p.T - 1) - q0;
 #pragma unroll
             for (int e4 = 0; e4 < 4; ++e4) {
-              const float4 L = *reinterpret_cast<const float4*>(lds + 16 * cs + 4 * e4);
-              const float4 D = *reinterpret_cast<const float4*>(lds + 64 + 16 * cs + 4 * e4);
+              const float4 L = *reinterpret_cast<const float4*>(lds + 4 * e4);
+              const float4 D = *reinterpret_cast<const float4*>(lds + 16 + 4 * e4);
               const float Ls[4] = {L.x, L.y, L.z, L.w};
               const float Ds[4] = {D.x, D.y, D.z, D.w};
 #pragma unroll
@@ -775,13 +776,9 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
             }
           }
         }
+        publish();  // LSE / Delta of half-tile g+1
         // Buffers g&1 (P^T in TMEM, dS^T in shared memory) held half-tile
-        // g-2, whose MMAs completed before dQ^T_{g-2} was drained. This
-        // barrier publishes LSE / Delta of g+1 into the other lds buffer, last
-        // read by every thread before the previous barrier.
-        if (st < 128) lds_all[(buf ^ 1) * 128 + st] = pre_scaled();
-        // every softmax thread reaches this barrier on every half-tile, aborted or not
-        asm volatile("bar.sync 1, %0;" ::"n"(PIPE_SOFT_THREADS) : "memory");
+        // g-2, whose MMAs completed before this warp drained dQ^T_{g-2}.
         if (ok) {
           // P^T row r (this lane's key), queries 16*cs .. +15 as 8 bf16 pairs
           // in TMEM columns PT[buf] + 8*cs ..; dS^T into shared memory: 16-byte
@@ -812,7 +809,6 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
       // unit's MMAs are complete), so that every global store covers whole
       // 64-byte row pieces.
       ok = ok && warp_wait(acc_full, (uint32_t)n & 1u, ab);
-      asm volatile("bar.sync 1, %0;" ::"n"(PIPE_SOFT_THREADS) : "memory");  // reached by every softmax thread
       if (ok) {
         tc_fence_after();
         uint8_t* stg = smem + C::OFF_DS + w16 * 2048;       // [32 rows][32 bf16], 16-byte chunks swizzled
@@ -847,6 +843,9 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
           __syncwarp();
         }
       }
+      // the next unit's dS^T rows overwrite other warps' staging: every warp is
+      // past its epilogue first (reached by every softmax thread, aborted or not)
+      asm volatile("bar.sync 1, %0;" ::"n"(PIPE_SOFT_THREADS) : "memory");
     }
     if (g >= 1) drain_dq(g - 1, xp, jp);
     if (lane == 0) bulk_wait_all();  // dQ reductions complete before the CTA leaves
