@@ -528,10 +528,27 @@ cudaError_t run_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtenso
 
 }  // namespace
 
+// Two-SM (CTA pair) versions of the projection GEMMs (tc_gemm_pair.cu); they
+// return cudaErrorNotSupported when clusters of two cannot be launched.
+bool pair_gemm_supported(int D);
+cudaError_t launch_proj_fwd_pair(int64_t M, int D, int d, const void* m_shift, const void* w_mk, const void* w_mv,
+                                 void* Rk, void* Rv, int64_t spin_limit, int* err, cudaStream_t s);
+cudaError_t launch_proj_bwd_dm_pair(int64_t M, int D, int d, const void* dRk, const void* dRv, const void* w_mk,
+                                    const void* w_mv, void* dm, int64_t spin_limit, int* err, cudaStream_t s);
+cudaError_t launch_proj_bwd_dm_layers_pair(int64_t M, int D, int d, int L, const void* dRk, const void* dRv,
+                                           const void* w_mk, const void* w_mv, void* dm, int64_t spin_limit,
+                                           int* err, cudaStream_t s);
+cudaError_t launch_proj_bwd_dw_pair(int64_t M, int D, int d, const void* dRk, const void* dRv, const void* m_shift,
+                                    void* dwk, void* dwv, int64_t spin_limit, int* err, cudaStream_t s);
+
 // R_k | R_v [M, D] = m_shift [M, d] x W^T, W_mk / W_mv [D, d].
 cudaError_t launch_proj_fwd_tc(int64_t M, int D, int d, const void* m_shift, const void* w_mk,
                                const void* w_mv, void* Rk, void* Rv, int64_t spin_limit, int* err,
                                cudaStream_t s) {
+  if (pair_gemm_supported(D)) {
+    const cudaError_t pe = launch_proj_fwd_pair(M, D, d, m_shift, w_mk, w_mv, Rk, Rv, spin_limit, err, s);
+    if (pe != cudaErrorNotSupported) return pe;
+  }
   constexpr int BN = 256;
   CUtensorMap a, b0, b1;
   cudaError_t e;
@@ -558,6 +575,10 @@ cudaError_t launch_proj_fwd_tc(int64_t M, int D, int d, const void* m_shift, con
 cudaError_t launch_proj_bwd_dm_tc(int64_t M, int D, int d, const void* dRk, const void* dRv,
                                   const void* w_mk, const void* w_mv, void* dm, int64_t spin_limit,
                                   int* err, cudaStream_t s) {
+  if (pair_gemm_supported(D)) {
+    const cudaError_t pe = launch_proj_bwd_dm_pair(M, D, d, dRk, dRv, w_mk, w_mv, dm, spin_limit, err, s);
+    if (pe != cudaErrorNotSupported) return pe;
+  }
   constexpr int BN = 256;
   CUtensorMap a0, a1, b0, b1;
   cudaError_t e;
@@ -586,6 +607,11 @@ cudaError_t launch_proj_bwd_dm_tc(int64_t M, int D, int d, const void* dRk, cons
 cudaError_t launch_proj_bwd_dm_layers_tc(int64_t M, int D, int d, int L, const void* dRk, const void* dRv,
                                          const void* w_mk, const void* w_mv, void* dm, int64_t spin_limit,
                                          int* err, cudaStream_t s) {
+  if (pair_gemm_supported(D)) {
+    const cudaError_t pe =
+        launch_proj_bwd_dm_layers_pair(M, D, d, L, dRk, dRv, w_mk, w_mv, dm, spin_limit, err, s);
+    if (pe != cudaErrorNotSupported) return pe;
+  }
   constexpr int BN = 256;
   CUtensorMap a0, a1, b0, b1;
   cudaError_t e;
@@ -618,6 +644,10 @@ cudaError_t launch_proj_bwd_dm_layers_tc(int64_t M, int D, int d, int L, const v
 cudaError_t launch_proj_bwd_dw_tc(int64_t M, int D, int d, const void* dRk, const void* dRv,
                                   const void* m_shift, void* dwk, void* dwv, int64_t spin_limit,
                                   int* err, cudaStream_t s) {
+  if (pair_gemm_supported(D)) {
+    const cudaError_t pe = launch_proj_bwd_dw_pair(M, D, d, dRk, dRv, m_shift, dwk, dwv, spin_limit, err, s);
+    if (pe != cudaErrorNotSupported) return pe;
+  }
   constexpr int BN = 192;
   CUtensorMap a0, a1, b;
   cudaError_t e;

@@ -1,0 +1,482 @@
+// Two-SM tcgen05 GEMM for the shared memory projection of Maglev's recurrent
+// K/V injection and its backward ("Maglev: Sliding Recurrent Memory",
+// paper.rainbus.top, 方法步骤详情: k_rec and v_rec come from the projections
+// W_k^rec, W_v^rec shared by all layers):
+//   forward  R = m_shift [B*T, d] x [W_mk; W_mv]^T           -> R_k | R_v
+//   backward dm = [dR_k | dR_v] x [W_mk; W_mv]                (K = 2D)
+//            dW = [dR_k | dR_v]^T x m_shift                   (M = 2D)
+// and the per-layer projection's dm over layer-strided operands.
+//
+// A cluster of two CTAs on two SMs owns a 256 x 256 output tile: each CTA
+// TMA-loads its 128 rows of A and its 128 columns of B per 128-wide K block
+// into its own shared memory (no multicast), and the leader (even) CTA issues
+// tcgen05.mma.cta_group::2 (256 x 256 x 16), which reads both CTAs' operands
+// and accumulates each CTA's 128 rows in that CTA's TMEM. Per SM that is 64 KiB
+// of operands per 1024 MMA cycles (a one-SM 128 x 256 tile needs 1.5x that
+// per flop and is fed-bound at ~70%). Every operand arrives in 16 KiB boxes
+// ({64, 128}): L2 -> SM TMA throughput with 8 KiB boxes is a third lower.
+// Two TMEM accumulators per CTA let the epilogue of one tile run under the
+// next tile's MMAs.
+//
+// Roles per CTA (6 warps): warp 0 TMA producer, warp 1 MMA issuer (leader
+// only), warps 2-5 epilogue (TMEM -> bf16 -> 128-byte row pieces). Loads in
+// both CTAs count their bytes on the leader's stage barrier; the MMA commit
+// releases a stage / publishes an accumulator in both CTAs at once; each
+// epilogue warp returns its accumulator with an arrival on the leader's
+// barrier. Every mbarrier wait is bounded.
+#include <cuda.h>
+
+#include "launchers.h"
+#include "tc_common.cuh"
+
+namespace maglev {
+
+cudaError_t make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                              uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+cudaError_t make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+                              uint32_t box_inner, uint32_t box_mid);
+
+namespace {
+
+using namespace tc;
+
+constexpr int PM = 256;       // rows of a pair tile (128 per CTA)
+constexpr int PN = 256;       // columns of a pair tile (B: 128 per CTA)
+constexpr int PAIR_THREADS = 192;
+
+struct PairParams {
+  int M, N, K;
+  int tiles_m, tiles_n;
+  int a_switch_m, a_switch_k;  // rows / K index where operand A moves to map 1
+  int b_switch_n, b_switch_k;
+  int out_switch_m, out_switch_n;
+  int k_layers;  // > 0: A [k_layers][M][a_switch_k], B [k_layers][a_switch_k][N] (3-D maps), K = 2 L a_switch_k
+  void* out0;
+  void* out1;
+  int64_t ldo;
+  int64_t spin_limit;
+  int* err;
+};
+
+template <bool A_MN, bool B_MN>
+struct PairCfg {
+  // K block: 64 when both operands are K-major (one {64 K, 128 rows} box each,
+  // six 32 KiB stages); 128 when one is MN-major, whose 16 KiB box is
+  // {64 MN, 128 K} (three 64 KiB stages). A 16 KiB operand piece is
+  // K-major [128 rows x 64 K] (pieces along K) or MN-major [128 K x 64 MN]
+  // (pieces along MN).
+  static constexpr int PK = (A_MN || B_MN) ? 128 : 64;
+  static constexpr int A_BYTES = 128 * PK * 2;          // this CTA's 128 rows
+  static constexpr int B_BYTES = (PN / 2) * PK * 2;     // this CTA's 128 columns
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = PK == 64 ? 6 : 3;
+  static constexpr int PIECES = PK == 64 ? 1 : 2;       // 16 KiB pieces per operand per stage
+  static constexpr int TMEM_COLS = 512;                 // two 128 x 256 fp32 accumulators
+  static constexpr int ACC_STRIDE = 256;
+  static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
+  static constexpr int OFF_EPI = OFF_BAR + 256;         // 4 warps x [32 rows x 128 B] output staging
+  static constexpr size_t SMEM = 1024 + (size_t)OFF_EPI + 4 * 4096;
+};
+
+template <bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(PAIR_THREADS, 1)
+    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                        const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+                        PairParams p) {
+  using C = PairCfg<A_MN, B_MN>;
+  constexpr int STAGES = C::STAGES;
+  constexpr int PK = C::PK;
+  extern __shared__ uint8_t smem_raw[];
+  // the same offset in both CTAs: the pair MMA reads both CTAs' operands at one address
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);  // [STAGES], used in the leader
+  uint64_t* empty = full + STAGES;                                  // [STAGES]
+  uint64_t* tfull = empty + STAGES;                                 // [2]
+  uint64_t* tempty = tfull + 2;                                     // [2], used in the leader
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const Abort ab{abort_flag, p.err, p.spin_limit * 1000};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 8);  // one arrival per epilogue warp of both CTAs
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA0);
+    tma_prefetch_desc(&tmA1);
+    tma_prefetch_desc(&tmB0);
+    tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before any remote arrival or load
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_tiles = p.tiles_m * p.tiles_n;
+  const int pair = (int)blockIdx.x >> 1, npairs = (int)gridDim.x >> 1;
+  const int kblocks = (p.K + C::PK - 1) / C::PK;
+  constexpr uint32_t IDESC = idesc_bf16(PM, PN, A_MN, B_MN);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer (both CTAs)
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = pair; t < num_tiles && ok; t += npairs) {
+        const int tm = t % p.tiles_m, tn = t / p.tiles_m;
+        const int m0 = tm * PM + 128 * (int)rank;  // this CTA's A rows
+        const int n0 = tn * PN + 128 * (int)rank;  // this CTA's B columns
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, ab)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);  // both CTAs' bytes
+          const uint32_t bar = mapa_cluster(smem_u32(&full[stage]), 0);
+          uint8_t* dA = sA + stage * C::A_BYTES;
+          uint8_t* dB = sB + stage * C::B_BYTES;
+          const int k0 = kb * PK;
+          if constexpr (!A_MN && B_MN) {
+            if (p.k_layers > 0) {  // layer-strided K: (k or v, layer l, k within the layer)
+              const int LD = p.k_layers * p.a_switch_k;
+              const int which = k0 >= LD ? 1 : 0;
+              const int kr = k0 - which * LD;
+              const int l = kr / p.a_switch_k, kk = kr - l * p.a_switch_k;
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {  // A K-major, B MN-major: PK = 128
+                tma_load_3d_pair(dA + h * 16384, which ? &tmA1 : &tmA0, bar, kk + 64 * h, m0, l);
+                tma_load_3d_pair(dB + h * 16384, which ? &tmB1 : &tmB0, bar, n0 + 64 * h, kk, l);
+              }
+              if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1;
+              }
+              continue;
+            }
+          }
+          // operand A: this CTA's 128 rows; halves along K (K-major) or M (MN-major).
+          // The k / v switches fall on multiples of 128 (checked by the host).
+          {
+            const bool second = (p.a_switch_m > 0 && m0 >= p.a_switch_m) || (p.a_switch_k > 0 && k0 >= p.a_switch_k);
+            const CUtensorMap* m = second ? &tmA1 : &tmA0;
+            const int mm = (p.a_switch_m > 0 && m0 >= p.a_switch_m) ? m0 - p.a_switch_m : m0;
+            const int kk = (p.a_switch_k > 0 && k0 >= p.a_switch_k) ? k0 - p.a_switch_k : k0;
+#pragma unroll
+            for (int h = 0; h < C::PIECES; ++h)
+              tma_load_2d_pair(dA + h * 16384, m, bar, A_MN ? mm + 64 * h : kk + 64 * h, A_MN ? kk : mm);
+          }
+          // operand B: this CTA's 128 columns; halves along K (K-major) or N (MN-major)
+          {
+            const bool second = (p.b_switch_n > 0 && n0 >= p.b_switch_n) || (p.b_switch_k > 0 && k0 >= p.b_switch_k);
+            const CUtensorMap* m = second ? &tmB1 : &tmB0;
+            const int nn = (p.b_switch_n > 0 && n0 >= p.b_switch_n) ? n0 - p.b_switch_n : n0;
+            const int kk = (p.b_switch_k > 0 && k0 >= p.b_switch_k) ? k0 - p.b_switch_k : k0;
+#pragma unroll
+            for (int h = 0; h < C::PIECES; ++h)
+              tma_load_2d_pair(dB + h * 16384, m, bar, B_MN ? nn + 64 * h : kk + 64 * h, B_MN ? kk : nn);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // Every stage this CTA filled has been consumed (so its loads have landed)
+      // before the CTA may exit: wait for the release of the last fill of each.
+      for (int s = 0; s < STAGES; ++s) {
+        mbar_drain(&empty[stage], phase ^ 1, DRAIN_LIMIT_NS);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (leader) {
+      // ------------------------------------------------------------ MMA issuer (leader CTA)
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = pair; t < num_tiles && ok; t += npairs) {
+        if (!warp_wait(&tempty[acc], acc_phase ^ 1, ab)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * C::ACC_STRIDE);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!warp_wait(&full[stage], phase, ab)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * C::B_BYTES);
+          if (elect_one()) {
+#pragma unroll
+            for (int k16 = 0; k16 < PK / 16; ++k16) {
+              // K-major: half k16 / 4, 32 bytes per 16 K inside it; MN-major: 16 K rows
+              // of 128 B per step, the two MN halves 16 KiB apart
+              const uint32_t koff = (uint32_t)(k16 >> 2) * 16384u + (uint32_t)(k16 & 3) * 32u;
+              const uint64_t ad = A_MN ? sw128_desc(a_addr + (uint32_t)k16 * 2048u, 16384u, 1024u)
+                                       : sw128_desc(a_addr + koff, 16u, 1024u);
+              const uint64_t bd = B_MN ? sw128_desc(b_addr + (uint32_t)k16 * 2048u, 16384u, 1024u)
+                                       : sw128_desc(b_addr + koff, 16u, 1024u);
+              mma_ss_pair(d_tmem, ad, bd, IDESC, (kb > 0 || k16 > 0) ? 1u : 0u);
+            }
+            mma_commit_pair_both(&empty[stage]);  // the stage is free in both CTAs
+          }
+          __syncwarp();
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        if (elect_one()) mma_commit_pair_both(&tfull[acc]);  // both CTAs' halves of the tile are ready
+        __syncwarp();
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      // all issued MMAs finish before either CTA releases its TMEM
+      if (elect_one()) {
+        mma_commit_pair(drain);
+        mbar_drain(drain, 0, DRAIN_LIMIT_NS);
+      }
+      __syncwarp();
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue (both CTAs)
+    // This CTA's 128 rows of the tile, 64 columns at a time: TMEM -> bf16 ->
+    // the warp's 4 KiB of staging (16-byte chunks swizzled by row) -> read back
+    // so that each warp-wide store covers four whole 128-byte row pieces.
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    uint8_t* stg = smem + C::OFF_EPI + q * 4096;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = pair; t < num_tiles; t += npairs) {
+      const int tm = t % p.tiles_m, tn = t / p.tiles_m;
+      const int m0 = tm * PM + 128 * (int)rank, n0 = tn * PN;
+      if (!warp_wait(&tfull[acc], acc_phase, ab)) break;
+      tc_fence_after();
+      bf16* out = static_cast<bf16*>(p.out0);
+      int om0 = m0 + q * 32;  // first row of this warp in the output tensor
+      if (p.out_switch_m > 0 && m0 >= p.out_switch_m) {
+        out = static_cast<bf16*>(p.out1);
+        om0 -= p.out_switch_m;
+      }
+#pragma unroll 1
+      for (int c0 = 0; c0 < PN; c0 += 64) {
+        uint32_t r[2][32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::ACC_STRIDE + c0), r[0]);
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::ACC_STRIDE + c0 + 32), r[1]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          uint4 v;
+          v.x = pack_bf16(__uint_as_float(r[j >> 2][8 * (j & 3) + 0]), __uint_as_float(r[j >> 2][8 * (j & 3) + 1]));
+          v.y = pack_bf16(__uint_as_float(r[j >> 2][8 * (j & 3) + 2]), __uint_as_float(r[j >> 2][8 * (j & 3) + 3]));
+          v.z = pack_bf16(__uint_as_float(r[j >> 2][8 * (j & 3) + 4]), __uint_as_float(r[j >> 2][8 * (j & 3) + 5]));
+          v.w = pack_bf16(__uint_as_float(r[j >> 2][8 * (j & 3) + 6]), __uint_as_float(r[j >> 2][8 * (j & 3) + 7]));
+          *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) = v;
+        }
+        __syncwarp();
+        // 64 columns [col0, col0 + 64): this tensor, or the second one past out_switch_n
+        const int col0 = n0 + c0;
+        bf16* o = out;
+        int ocol0 = col0, n_lim = p.N;
+        if (p.out_switch_n > 0) {
+          if (col0 >= p.out_switch_n) {
+            o = static_cast<bf16*>(p.out1);
+            ocol0 -= p.out_switch_n;
+          } else {
+            n_lim = p.out_switch_n;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 4 * i + (lane >> 3), j = lane & 7;  // row of the warp's 32, 16-byte chunk
+          const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 128 + ((j ^ (rr & 7)) << 4));
+          if (m0 + q * 32 + rr < p.M && col0 + 8 * j + 8 <= n_lim)
+            *reinterpret_cast<uint4*>(o + (int64_t)(om0 + rr) * p.ldo + ocol0 + 8 * j) = v;
+        }
+        __syncwarp();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_cluster(smem_u32(&tempty[acc]), 0));  // the leader may reuse it
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+  __syncthreads();
+  cluster_sync_all();  // neither CTA releases TMEM / leaves while the pair still uses it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+namespace {
+
+// Largest number of two-CTA clusters of this kernel that can be resident at
+// once (0 when clusters cannot be launched), cached per instantiation.
+template <bool A_MN, bool B_MN>
+int max_pairs() {
+  static int cached = -1;
+  if (cached >= 0) return cached;
+  using C = PairCfg<A_MN, B_MN>;
+  auto kern = tc_gemm_pair_kernel<A_MN, B_MN>;
+  int n = 0;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 74, 1, 1);
+    cfg.blockDim = dim3(PAIR_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, (void*)kern, &cfg) != cudaSuccess) n = 0;
+  }
+  (void)cudaGetLastError();
+  cached = n;
+  return n;
+}
+
+template <bool A_MN, bool B_MN>
+cudaError_t run_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0, const CUtensorMap& b1,
+                     PairParams p, cudaStream_t s) {
+  using C = PairCfg<A_MN, B_MN>;
+  const int cap = max_pairs<A_MN, B_MN>();
+  if (cap < 1) return cudaErrorNotSupported;
+  const int tiles = p.tiles_m * p.tiles_n;
+  const int pairs = tiles < cap ? tiles : cap;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(PAIR_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<A_MN, B_MN>, a0, a1, b0, b1, p);
+}
+
+PairParams pair_params(int M, int N, int K, int64_t ldo, int64_t spin_limit, int* err) {
+  PairParams p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.tiles_m = (M + PM - 1) / PM;
+  p.tiles_n = (N + PN - 1) / PN;
+  p.ldo = ldo;
+  p.spin_limit = spin_limit;
+  p.err = err;
+  return p;
+}
+
+}  // namespace
+
+// The pair kernels move between the k and v operands only at multiples of 128
+// (a CTA's rows / columns, a K block): D must be a multiple of 128; otherwise
+// the caller uses the one-SM kernels.
+bool pair_gemm_supported(int D) { return D % 128 == 0; }
+
+// R_k | R_v [M, D] = m_shift [M, d] x W^T, W_mk / W_mv [D, d].
+cudaError_t launch_proj_fwd_pair(int64_t M, int D, int d, const void* m_shift, const void* w_mk, const void* w_mv,
+                                 void* Rk, void* Rv, int64_t spin_limit, int* err, cudaStream_t s) {
+  CUtensorMap a, b0, b1;
+  cudaError_t e;
+  if ((e = make_tmap_bf16_2d(&a, m_shift, d, M, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&b0, w_mk, d, D, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&b1, w_mv, d, D, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
+  PairParams p = pair_params((int)M, 2 * D, d, D, spin_limit, err);
+  p.b_switch_n = D;
+  p.out_switch_n = D;
+  p.out0 = Rk;
+  p.out1 = Rv;
+  return run_pair<false, false>(a, a, b0, b1, p, s);
+}
+
+// dm [M, d] = dR_k [M, D] W_mk [D, d] + dR_v W_mv (K = 2D, B operand N-contiguous).
+cudaError_t launch_proj_bwd_dm_pair(int64_t M, int D, int d, const void* dRk, const void* dRv, const void* w_mk,
+                                    const void* w_mv, void* dm, int64_t spin_limit, int* err, cudaStream_t s) {
+  CUtensorMap a0, a1, b0, b1;
+  cudaError_t e;
+  if ((e = make_tmap_bf16_2d(&a0, dRk, D, M, (uint64_t)D * 2, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&a1, dRv, D, M, (uint64_t)D * 2, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&b0, w_mk, d, D, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&b1, w_mv, d, D, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
+  PairParams p = pair_params((int)M, d, 2 * D, d, spin_limit, err);
+  p.a_switch_k = D;
+  p.b_switch_k = D;
+  p.out0 = dm;
+  p.out1 = dm;
+  return run_pair<false, true>(a0, a1, b0, b1, p, s);
+}
+
+// dm [M, d] = sum over L layers of dR_k^l W_mk^l + dR_v^l W_mv^l (layer-strided, K = 2 L D).
+cudaError_t launch_proj_bwd_dm_layers_pair(int64_t M, int D, int d, int L, const void* dRk, const void* dRv,
+                                           const void* w_mk, const void* w_mv, void* dm, int64_t spin_limit,
+                                           int* err, cudaStream_t s) {
+  CUtensorMap a0, a1, b0, b1;
+  cudaError_t e;
+  if ((e = make_tmap_bf16_3d(&a0, dRk, D, M, L, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_3d(&a1, dRv, D, M, L, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_3d(&b0, w_mk, d, D, L, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_3d(&b1, w_mv, d, D, L, 64, 128)) != cudaSuccess) return e;
+  PairParams p = pair_params((int)M, d, 2 * L * D, d, spin_limit, err);
+  p.a_switch_k = D;
+  p.b_switch_k = D;
+  p.k_layers = L;
+  p.out0 = dm;
+  p.out1 = dm;
+  return run_pair<false, true>(a0, a1, b0, b1, p, s);
+}
+
+// dW_mk | dW_mv [D, d] = dR^T [D, M] m_shift [M, d] (A and B both M-contiguous in memory).
+cudaError_t launch_proj_bwd_dw_pair(int64_t M, int D, int d, const void* dRk, const void* dRv, const void* m_shift,
+                                    void* dwk, void* dwv, int64_t spin_limit, int* err, cudaStream_t s) {
+  CUtensorMap a0, a1, b;
+  cudaError_t e;
+  if ((e = make_tmap_bf16_2d(&a0, dRk, D, M, (uint64_t)D * 2, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&a1, dRv, D, M, (uint64_t)D * 2, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&b, m_shift, d, M, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
+  PairParams p = pair_params(2 * D, d, (int)M, d, spin_limit, err);
+  p.a_switch_m = D;
+  p.out_switch_m = D;
+  p.out0 = dwk;
+  p.out1 = dwv;
+  return run_pair<true, true>(a0, a1, b, b, p, s);
+}
+
+}  // namespace maglev
