@@ -101,14 +101,17 @@ __device__ __forceinline__ float row_sum(float x) {
 }
 
 // cos / sin of position p times inv_freq (double) for 8 pairs, reduced to
-// [-pi, pi] in double before the float sincos.
+// [-pi, pi] in double before the hardware sin / cos (__sincosf: absolute error
+// about 2^-21 on [-pi, pi], far below the bf16 and fp32 tolerances of the
+// rotated values, and two special-function instructions instead of a full
+// range-reduced sincosf per pair).
 __device__ __forceinline__ void rope8(int64_t p, const double* inv_freq, int c0, float* cs, float* sn) {
   const double two_pi = 6.283185307179586476925286766559;
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     double ang = (double)p * inv_freq[c0 + e];
     ang -= two_pi * rint(ang * 0.15915494309189533577);
-    sincosf((float)ang, &sn[e], &cs[e]);
+    __sincosf((float)ang, &sn[e], &cs[e]);
   }
 }
 

@@ -9,49 +9,88 @@ namespace maglev {
 namespace {
 
 constexpr int LOSS_THREADS = 256;
-constexpr int LOSS_U = 4;                                 // 8-element vectors per thread
-constexpr int64_t LOSS_CHUNK = 8 * LOSS_THREADS * LOSS_U;  // elements per block
+constexpr int LOSS_U = 2;             // 8-element vectors per thread per round
+constexpr int LOSS_MAX_BLOCKS = 592;  // persistent grid: 4 blocks on each of 148 SMs
 
-// Block b covers elements [b * LOSS_CHUNK, (b + 1) * LOSS_CHUNK): each thread
-// puts all of its loads (LOSS_U vectors of m, m' and, when accumulating, dm)
-// in flight before any arithmetic, then writes dm, dm' and adds its squares.
+// 8 elements in their stored form, so that a thread puts all its loads of a
+// round in flight before any arithmetic.
 template <typename T>
-__global__ void __launch_bounds__(LOSS_THREADS) loss_partial_kernel(
+struct Raw8L;
+template <>
+struct Raw8L<bf16> {
+  uint4 u;
+  __device__ __forceinline__ void load(const bf16* p) { u = *reinterpret_cast<const uint4*>(p); }
+  __device__ __forceinline__ void to(float* x) const {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      x[2 * i] = f.x;
+      x[2 * i + 1] = f.y;
+    }
+  }
+};
+template <>
+struct Raw8L<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* p) {
+    a = *reinterpret_cast<const float4*>(p);
+    b = *reinterpret_cast<const float4*>(p + 4);
+  }
+  __device__ __forceinline__ void to(float* x) const {
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+};
+
+// Block b walks rounds r = b, b + G, ... (G blocks); round r covers vectors
+// [r * 256 * U, (r + 1) * 256 * U). Each thread loads all U vectors of m, m'
+// and, when accumulating, dm of its round before any arithmetic, then writes
+// dm, dm' and adds its squares; the block's partial is the sum over its rounds
+// in a fixed order, so the loss is bitwise reproducible for a given size.
+template <typename T>
+__global__ void __launch_bounds__(LOSS_THREADS, sizeof(T) == 2 ? 4 : 2) loss_partial_kernel(
     const T* __restrict__ m, const T* __restrict__ mt, int64_t n, float scale_grad,
     T* __restrict__ dm, T* __restrict__ dmt, int accumulate, float* __restrict__ partials) {
   __shared__ float red[LOSS_THREADS / 32];
-  const int64_t lo = (int64_t)blockIdx.x * LOSS_CHUNK;
   float acc = 0.f;
   if ((n & 7) == 0) {
-    float a[LOSS_U][8], b[LOSS_U][8], d[LOSS_U][8];
+    const int64_t nv = n >> 3;
     const bool rd = dm != nullptr && accumulate;
+    for (int64_t r0 = (int64_t)blockIdx.x * LOSS_THREADS * LOSS_U; r0 < nv;
+         r0 += (int64_t)gridDim.x * LOSS_THREADS * LOSS_U) {
+      Raw8L<T> a[LOSS_U], b[LOSS_U], d[LOSS_U];
 #pragma unroll
-    for (int u = 0; u < LOSS_U; ++u) {
-      const int64_t i = lo + 8 * ((int64_t)u * LOSS_THREADS + threadIdx.x);
-      if (i < n) {
-        load8f(m + i, a[u]);
-        load8f(mt + i, b[u]);
-        if (rd) load8f(dm + i, d[u]);
+      for (int u = 0; u < LOSS_U; ++u) {
+        const int64_t i = r0 + (int64_t)u * LOSS_THREADS + threadIdx.x;
+        if (i < nv) {
+          a[u].load(m + 8 * i);
+          b[u].load(mt + 8 * i);
+          if (rd) d[u].load(dm + 8 * i);
+        }
       }
-    }
 #pragma unroll
-    for (int u = 0; u < LOSS_U; ++u) {
-      const int64_t i = lo + 8 * ((int64_t)u * LOSS_THREADS + threadIdx.x);
-      if (i >= n) continue;
+      for (int u = 0; u < LOSS_U; ++u) {
+        const int64_t i = r0 + (int64_t)u * LOSS_THREADS + threadIdx.x;
+        if (i >= nv) continue;
+        float x[8], y[8], z[8];
+        a[u].to(x);
+        b[u].to(y);
+        if (rd) d[u].to(z);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float diff = a[u][e] - b[u][e];
-        acc = fmaf(diff, diff, acc);
-        const float g = scale_grad * diff;
-        a[u][e] = rd ? d[u][e] + g : g;
-        b[u][e] = -g;
+        for (int e = 0; e < 8; ++e) {
+          const float diff = x[e] - y[e];
+          acc = fmaf(diff, diff, acc);
+          const float g = scale_grad * diff;
+          x[e] = rd ? z[e] + g : g;
+          y[e] = -g;
+        }
+        if (dm) store8f(dm + 8 * i, x);
+        if (dmt) store8f(dmt + 8 * i, y);
       }
-      if (dm) store8f(dm + i, a[u]);
-      if (dmt) store8f(dmt + i, b[u]);
     }
   } else {
-    const int64_t hi = min(n, lo + LOSS_CHUNK);
-    for (int64_t i = lo + threadIdx.x; i < hi; i += LOSS_THREADS) {
+    for (int64_t i = (int64_t)blockIdx.x * LOSS_THREADS + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * LOSS_THREADS) {
       const float diff = to_f(m[i]) - to_f(mt[i]);
       acc = fmaf(diff, diff, acc);
       const float g = scale_grad * diff;
@@ -88,8 +127,9 @@ __global__ void __launch_bounds__(LOSS_THREADS) loss_final_kernel(const float* _
 }  // namespace
 
 int loss_partial_blocks(int64_t n) {
-  const int64_t b = (n + LOSS_CHUNK - 1) / LOSS_CHUNK;
-  return (int)(b < 1 ? 1 : b);
+  const int64_t per = (n & 7) == 0 ? 8 * LOSS_THREADS * LOSS_U : LOSS_THREADS;  // elements per round
+  const int64_t b = (n + per - 1) / per;
+  return (int)(b < 1 ? 1 : (b > LOSS_MAX_BLOCKS ? LOSS_MAX_BLOCKS : b));
 }
 
 cudaError_t launch_consistency_loss(const void* m, const void* mt, int64_t rows, int d, int dtype,
