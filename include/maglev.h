@@ -45,7 +45,11 @@ typedef enum {
   MAGLEV_ERR_INVALID_ARG = 1,
   MAGLEV_ERR_UNSUPPORTED = 2,
   MAGLEV_ERR_CUDA = 3,
-  MAGLEV_ERR_TIMEOUT = 4
+  MAGLEV_ERR_TIMEOUT = 4,
+  /* Only from a library built with -DMAGLEV_DEBUG (libmaglev_debug.so): an
+   * in-kernel index check failed; the access was skipped. Reported through
+   * maglev_device_status like MAGLEV_ERR_TIMEOUT. */
+  MAGLEV_ERR_BOUNDS = 5
 } maglev_status;
 
 typedef enum { MAGLEV_F32 = 0, MAGLEV_BF16 = 1 } maglev_dtype;

@@ -14,10 +14,12 @@ import os
 import re
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmaglev.so")
+# MAGLEV_DEBUG=1 selects the debug build (in-kernel index checks that record
+# MAGLEV_ERR_BOUNDS), libmaglev_debug.so from `build.py --debug`.
+LIB_PATH = os.path.join(_HERE, "libmaglev_debug.so" if os.environ.get("MAGLEV_DEBUG") == "1" else "libmaglev.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "maglev.h")
 
-MAGLEV_OK, MAGLEV_ERR_INVALID_ARG, MAGLEV_ERR_UNSUPPORTED, MAGLEV_ERR_CUDA, MAGLEV_ERR_TIMEOUT = range(5)
+MAGLEV_OK, MAGLEV_ERR_INVALID_ARG, MAGLEV_ERR_UNSUPPORTED, MAGLEV_ERR_CUDA, MAGLEV_ERR_TIMEOUT, MAGLEV_ERR_BOUNDS = range(6)
 MAGLEV_F32, MAGLEV_BF16 = 0, 1
 MAGLEV_DR_WRITE, MAGLEV_DR_FIRST, MAGLEV_DR_ADD, MAGLEV_DR_LAST = range(4)
 

@@ -1,9 +1,12 @@
 """Build libmaglev.so in-tree for sm_100a with nvcc.
 
-    python -m sliding_window_recurrent_b200.build [--force] [--ptxas-verbose]
+    python -m sliding_window_recurrent_b200.build [--force] [--ptxas-verbose] [--debug]
 
 Objects go to _build/ at the repo root; the shared library lands next to this
-file so that it travels with the source tree.
+file so that it travels with the source tree. --debug builds
+libmaglev_debug.so with -DMAGLEV_DEBUG: in-kernel index checks that record
+MAGLEV_ERR_BOUNDS in the device status word and skip the access (the binding
+loads it when MAGLEV_DEBUG=1).
 """
 from __future__ import annotations
 
@@ -20,6 +23,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmaglev.so")
+LIB_DEBUG = os.path.join(PKG, "libmaglev_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
@@ -46,19 +50,22 @@ def _newest(paths):
     return max((os.path.getmtime(p) for p in paths), default=0.0)
 
 
-def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = False, debug: bool = False) -> str:
+    bdir = os.path.join(BUILD, "debug") if debug else BUILD
+    lib = LIB_DEBUG if debug else LIB
+    flags = NVCC_FLAGS + (["-DMAGLEV_DEBUG"] if debug else [])
+    os.makedirs(bdir, exist_ok=True)
     cc = nvcc()
     hdr_time = _newest(headers())
     jobs = []
     objs = []
     for src in sources():
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(bdir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         stale = force or not os.path.exists(obj) or os.path.getmtime(obj) < max(
             os.path.getmtime(src), hdr_time)
         if stale:
-            cmd = [cc] + NVCC_FLAGS + (["-Xptxas", "-v"] if ptxas_verbose else []) + ["-c", src, "-o", obj]
+            cmd = [cc] + flags + (["-Xptxas", "-v"] if ptxas_verbose else []) + ["-c", src, "-o", obj]
             jobs.append((src, cmd))
 
     def run(job):
@@ -74,18 +81,19 @@ def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = False)
                     raise RuntimeError(f"nvcc failed on {os.path.basename(src)}")
                 if ptxas_verbose or (r.stderr.strip() and not quiet):
                     sys.stderr.write(r.stderr)
-    if force or jobs or not os.path.exists(LIB) or os.path.getmtime(LIB) < _newest(objs):
-        cmd = [cc] + ARCH + ["-shared", "-o", LIB] + objs
+    if force or jobs or not os.path.exists(lib) or os.path.getmtime(lib) < _newest(objs):
+        cmd = [cc] + ARCH + ["-shared", "-o", lib] + objs
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)
-            raise RuntimeError("link of libmaglev.so failed")
-    return LIB
+            raise RuntimeError(f"link of {os.path.basename(lib)} failed")
+    return lib
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--ptxas-verbose", action="store_true")
+    ap.add_argument("--debug", action="store_true")
     a = ap.parse_args()
-    print(build(force=a.force, ptxas_verbose=a.ptxas_verbose))
+    print(build(force=a.force, ptxas_verbose=a.ptxas_verbose, debug=a.debug))

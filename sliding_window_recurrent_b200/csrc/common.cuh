@@ -74,10 +74,23 @@ __device__ __forceinline__ void rope_cos_sin(int64_t p, int c, int hd, double lo
 }
 
 // Device status word (per device, defined in api.cu); kernels receive its address.
-enum { DEV_OK = 0, DEV_TIMEOUT = 4 };
+enum { DEV_OK = 0, DEV_TIMEOUT = 4, DEV_BOUNDS = 5 };
 
 __device__ __forceinline__ void record_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
 }
+
+// Index checks of the debug build (compiled with -DMAGLEV_DEBUG): a false
+// condition records MAGLEV_ERR_BOUNDS in the status word and the caller skips
+// the access; nothing traps. In the release build the check is `true`.
+#ifdef MAGLEV_DEBUG
+__device__ __forceinline__ bool debug_check(int* err, bool cond) {
+  if (!cond) record_error(err, DEV_BOUNDS);
+  return cond;
+}
+#define MAGLEV_CHECK(err, cond) ::maglev::debug_check((err), (cond))
+#else
+#define MAGLEV_CHECK(err, cond) true
+#endif
 
 }  // namespace maglev

@@ -292,6 +292,11 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
         for (int j = 2 * cb; j < 2 * ce; ++j, ++L) {  // j = 2c: K_c, j = 2c+1: V_c
           const int st = L % C::NSTAGE;
           const uint32_t ph = (uint32_t)(L / C::NSTAGE) & 1u;
+          if (!MAGLEV_CHECK(err, (j >> 1) * ST_ROWS < W && bh < s.B * s.H)) {  // every role stops
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
           if (!tc::mbar_wait(&empty[st], ph ^ 1u, ab)) {
             ok = false;
             break;
@@ -524,7 +529,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) decode_stream_kernel(
         }
       }
       const bool has_slot = valid_pos && slot / ST_ROWS >= cb && slot / ST_ROWS < ce;
-      if (has_slot && ok) {
+      if (has_slot && ok && MAGLEV_CHECK(err, slot >= 0 && slot < W && bh < s.B * s.H)) {
         kring[ring + (int64_t)slot * HD + tid] = from_f<bf16>(kn_b[tid]);
         vring[ring + (int64_t)slot * HD + tid] = from_f<bf16>(vn_b[tid]);
       }

@@ -702,7 +702,7 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
       fence_proxy_async_smem();
       __syncwarp();
       const int q0 = xd.kt + 64 * jd + 16 * cs;
-      if (lane == 0 && q0 < p.T) {  // none past the end of the sequence
+      if (lane == 0 && q0 < p.T && MAGLEV_CHECK(p.err, q0 >= 0 && xd.h < p.H && xd.b < p.B)) {  // none past the end
         tma_reduce_add_4d(&tmDQ, slice, 32 * q4, xd.h, q0, xd.b);
         bulk_commit();
       }
@@ -837,7 +837,7 @@ __global__ void __launch_bounds__(PIPE_THREADS, 1)
             const int rr = 8 * i + (lane >> 2), ch = lane & 3;  // row of the warp's 32, 16-byte chunk
             const uint4 w = *reinterpret_cast<const uint4*>(stg + rr * 64 + ((ch ^ ((rr >> 1) & 3)) << 4));
             const int key = x.kt + 32 * q4 + rr;
-            if (key < p.T)
+            if (key < p.T && MAGLEV_CHECK(p.err, x.b < p.B && col0 + 8 * ch + 8 <= tstride))
               *reinterpret_cast<uint4*>(dst + ((int64_t)x.b * p.T + key) * tstride + col0 + 8 * ch) = w;
           }
           __syncwarp();

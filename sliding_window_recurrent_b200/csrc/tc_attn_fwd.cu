@@ -419,7 +419,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
         for (int k = 0; k < 8; ++k) {
           const int rr = 4 * k + (lane >> 3), j = lane & 7;  // row of the warp's 32, 16-byte chunk
           const uint4 w = *reinterpret_cast<const uint4*>(stg + rr * 128 + ((j ^ (rr & 7)) << 4));
-          if (i_lo + rr < p.T) *reinterpret_cast<uint4*>(obase + rr * tstride + 64 * c + 8 * j) = w;
+          if (i_lo + rr < p.T && MAGLEV_CHECK(p.err, i_lo + rr >= 0 && x.b < p.B && x.h < p.H))
+            *reinterpret_cast<uint4*>(obase + rr * tstride + 64 * c + 8 * j) = w;
         }
         __syncwarp();
       }

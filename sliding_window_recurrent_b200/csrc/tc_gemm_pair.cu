@@ -314,7 +314,8 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
         for (int i = 0; i < 8; ++i) {
           const int rr = 4 * i + (lane >> 3), j = lane & 7;  // row of the warp's 32, 16-byte chunk
           const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 128 + ((j ^ (rr & 7)) << 4));
-          if (m0 + q * 32 + rr < p.M && col0 + 8 * j + 8 <= n_lim)
+          if (m0 + q * 32 + rr < p.M && col0 + 8 * j + 8 <= n_lim &&
+              MAGLEV_CHECK(p.err, om0 + rr >= 0 && ocol0 >= 0 && ocol0 + 8 * j + 8 <= p.ldo))
             *reinterpret_cast<uint4*>(o + (int64_t)(om0 + rr) * p.ldo + ocol0 + 8 * j) = v;
         }
         __syncwarp();

@@ -132,3 +132,13 @@ def test_driver_modules_only_call_bound_entry_points():
         for name in set(re.findall(r"\b(maglev_[a-z0-9_]+)\(", src)):
             assert hasattr(mod, name), (mod.__name__, name)
             assert hasattr(mg, name), name
+
+
+def test_debug_build_exports_every_symbol():
+    """The debug build (-DMAGLEV_DEBUG: in-kernel index checks that record
+    MAGLEV_ERR_BOUNDS) is a drop-in for the release library."""
+    path = _build.build(quiet=True, debug=True)
+    lib = ctypes.CDLL(path)
+    for n in mg.header_symbols():
+        assert hasattr(lib, n), n
+    assert mg.MAGLEV_ERR_BOUNDS == 5
