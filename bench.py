@@ -51,11 +51,10 @@ SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 # figures "traffic_source": "stored ncu capture", since they are not measured
 # during the run.
 NCU_TRAFFIC: dict[str, dict] = {
-    "attn_bwd_tc": {"bytes": 162984960, "src": "tc_attn_bwd.cu", "src_sha": "ff592e916e291f26"},
-    "attn_fwd_tc": {"bytes": 68273920, "src": "tc_attn_fwd.cu", "src_sha": "e2b9ee99ddfc1ff6"},
-    "decode_step": {"bytes": 172034048, "src": "decode.cu", "src_sha": "3d9fef6b5a1a20e3"},
+    "attn_bwd_tc": {"bytes": 164081408, "src": "tc_attn_bwd.cu", "src_sha": "1673693a89fbd72f"},
+    "attn_fwd_tc": {"bytes": 63595264, "src": "tc_attn_fwd.cu", "src_sha": "cdc1badd0e6a9b5c"},
+    "decode_step": {"bytes": 171966464, "src": "decode.cu", "src_sha": "188f1e09ac4c8bae"},
 }
-
 
 def stored_traffic(name: str):
     """The stored ncu DRAM bytes of `name` if taken on its current source, else None."""
