@@ -117,6 +117,7 @@ def kernel_work(name: str, cfg: dict) -> tuple[float, str]:
         "mem_project_tc": (f["proj_fwd"], "flop"),
         "mem_project_bwd_dm_tc": (f["proj_fwd"], "flop"),
         "mem_project_bwd_dw_tc": (f["proj_fwd"], "flop"),
+        "mem_project_bwd_tc": (2 * f["proj_fwd"], "flop"),  # dm and dW in one launch
         # reads q, k, v, R_k, R_v; writes q_rot, k_bar, v_bar (bf16)
         "inject_prep": (B * T * D * 2.0 * (5 + 3), "byte"),
         # reads dq_rot (fp32), dk_bar, dv_bar, k, v, R_k, R_v (bf16); writes dq, dk, dv, dR_k, dR_v

@@ -201,8 +201,11 @@ maglev_status maglev_inject_swa_bwd(const maglev_swa_desc* desc, const void* k, 
                                     void* workspace, void* stream);
 
 /* a6 -- backward of the shared memory projection.
- *   dm_shift [B,T,d_mem] = dR_k W_mk + dR_v W_mv (overwritten);
- *   dw_mk, dw_mv [D,d_mem] = dR^T m_shift summed over all B*T rows (overwritten). */
+ *   dm_shift [B,T,d_mem] = dR_k W_mk + dR_v W_mv (overwritten; NULL: not computed);
+ *   dw_mk, dw_mv [D,d_mem] = dR^T m_shift summed over all B*T rows (overwritten;
+ *     NULL as a pair: not computed).
+ * With all three outputs, bf16, d_mem % 8 == 0 and H*hd % 128 == 0, both
+ * products run in one launch on SM pairs. */
 maglev_status maglev_mem_project_bwd(const maglev_swa_desc* desc, const void* m_shift,
                                      const void* w_mk, const void* w_mv, const void* dR_k,
                                      const void* dR_v, void* dm_shift, void* dw_mk, void* dw_mv,

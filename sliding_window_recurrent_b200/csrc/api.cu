@@ -217,6 +217,13 @@ maglev_status run_mem_project_bwd(const maglev_swa_desc* d, const void* m, const
   maglev_status stw = status_word(&err, st);
   if (stw != MAGLEV_OK) return stw;
   const bool tc = d->dtype == MAGLEV_BF16 && K % 8 == 0;
+  if (dm && dwk && dwv && tc && proj_bwd_grouped_available(M, (int)D, (int)K)) {
+    MAGLEV_LAUNCH(1, st, launch_proj_bwd_grouped_pair(M, (int)D, (int)K, dRk, dRv, wk, wv, m, dm, dwk, dwv,
+                                                      spin_limit_of(d->spin_limit), err, st),
+                  "mem_project_bwd_tc");
+    dm = nullptr;
+    dwk = dwv = nullptr;
+  }
   if (dm && tc && D % 64 == 0) {
     MAGLEV_LAUNCH(1, st, launch_proj_bwd_dm_tc(M, (int)D, (int)K, dRk, dRv, wk, wv, dm,
                                                spin_limit_of(d->spin_limit), err, st),

@@ -108,6 +108,12 @@ cudaError_t launch_proj_bwd_dm_layers_tc(int64_t M, int D, int d, int L, const v
 cudaError_t launch_proj_bwd_dw_tc(int64_t M, int D, int d, const void* dRk, const void* dRv,
                                   const void* m_shift, void* dwk, void* dwv, int64_t spin_limit,
                                   int* err, cudaStream_t s);
+// dW and dm of the shared projection in one launch on SM pairs (tc_gemm_pair.cu),
+// when proj_bwd_grouped_available says it can run.
+bool proj_bwd_grouped_available(int64_t M, int D, int d);
+cudaError_t launch_proj_bwd_grouped_pair(int64_t M, int D, int d, const void* dRk, const void* dRv, const void* w_mk,
+                                         const void* w_mv, const void* m_shift, void* dm, void* dwk, void* dwv,
+                                         int64_t spin_limit, int* err, cudaStream_t s);
 int num_sms();
 
 // tcgen05 banded attention backward: dk_bar, dv_bar (bf16, rounded from the

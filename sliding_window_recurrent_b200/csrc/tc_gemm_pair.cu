@@ -8,8 +8,8 @@
 // and the per-layer projection's dm over layer-strided operands.
 //
 // A cluster of two CTAs on two SMs owns a 256 x 256 output tile: each CTA
-// TMA-loads its 128 rows of A and its 128 columns of B per 128-wide K block
-// into its own shared memory (no multicast), and the leader (even) CTA issues
+// TMA-loads its 128 rows of A and its 128 columns of B per K block into its
+// own shared memory (no multicast), and the leader (even) CTA issues
 // tcgen05.mma.cta_group::2 (256 x 256 x 16), which reads both CTAs' operands
 // and accumulates each CTA's 128 rows in that CTA's TMEM. Per SM that is 64 KiB
 // of operands per 1024 MMA cycles (a one-SM 128 x 256 tile needs 1.5x that
@@ -18,6 +18,13 @@
 // Two TMEM accumulators per CTA let the epilogue of one tile run under the
 // next tile's MMAs.
 //
+// One launch may carry two GEMMs (the backward's dm and dW both read dR, and
+// neither fills the 74 SM pairs of a B200 evenly on its own: dm is 160 tiles
+// of 20 K blocks, 2.16 waves; dW 50 tiles of 64 K blocks). The host then
+// deals the tiles of both longest first, each to the pair with the least work
+// so far, and passes every pair its list: 100 K-block times for the two
+// instead of 60 + 64 back to back.
+//
 // Roles per CTA (6 warps): warp 0 TMA producer, warp 1 MMA issuer (leader
 // only), warps 2-5 epilogue (TMEM -> bf16 -> 128-byte row pieces). Loads in
 // both CTAs count their bytes on the leader's stage barrier; the MMA commit
@@ -25,6 +32,12 @@
 // epilogue warp returns its accumulator with an arrival on the leader's
 // barrier. Every mbarrier wait is bounded.
 #include <cuda.h>
+
+#include <algorithm>
+#include <functional>
+#include <queue>
+#include <utility>
+#include <vector>
 
 #include "launchers.h"
 #include "tc_common.cuh"
@@ -43,34 +56,56 @@ using namespace tc;
 constexpr int PM = 256;       // rows of a pair tile (128 per CTA)
 constexpr int PN = 256;       // columns of a pair tile (B: 128 per CTA)
 constexpr int PAIR_THREADS = 192;
+constexpr int PAIR_MAX_PAIRS = 80;   // schedule table (a B200 holds 74 pairs)
+constexpr int PAIR_MAX_ITEMS = 512;  // tiles of a scheduled launch
 
-struct PairParams {
+// One GEMM of a launch: out [M, N] bf16 = A [M, K] x B [K, N], fp32 in TMEM.
+// A is K-major (rows of K contiguous) or MN-major (a_mn: columns of M
+// contiguous); B likewise with N (b_mn). The k / v halves of the projections
+// live in two tensors: A moves to its second map at row a_switch_m or K index
+// a_switch_k, B at column b_switch_n or K index b_switch_k, the output at row
+// out_switch_m or column out_switch_n (0: no switch).
+struct PairProblem {
   int M, N, K;
-  int tiles_m, tiles_n;
-  int a_switch_m, a_switch_k;  // rows / K index where operand A moves to map 1
+  int tiles_m, tiles_n, kblocks;
+  int a_mn, b_mn;
+  int a_switch_m, a_switch_k;
   int b_switch_n, b_switch_k;
   int out_switch_m, out_switch_n;
   int k_layers;  // > 0: A [k_layers][M][a_switch_k], B [k_layers][a_switch_k][N] (3-D maps), K = 2 L a_switch_k
   void* out0;
   void* out1;
   int64_t ldo;
-  int64_t spin_limit;
-  int* err;
 };
 
-template <bool A_MN, bool B_MN>
+struct PairMaps {
+  CUtensorMap a0, a1, b0, b1;
+};
+
+struct PairParams {
+  PairProblem pr[2];
+  int tiles0;   // items [0, tiles0) are problem 0's tiles, [tiles0, n_items) problem 1's
+  int n_items;
+  int sched;    // 1: pair i runs order[first[i] .. first[i + 1]); 0: items i, i + pairs, ...
+  int64_t spin_limit;
+  int* err;
+  uint16_t first[PAIR_MAX_PAIRS + 1];
+  uint16_t order[PAIR_MAX_ITEMS];
+};
+
+template <int PK>
 struct PairCfg {
   // K block: 64 when both operands are K-major (one {64 K, 128 rows} box each,
   // six 32 KiB stages); 128 when one is MN-major, whose 16 KiB box is
   // {64 MN, 128 K} (three 64 KiB stages). A 16 KiB operand piece is
   // K-major [128 rows x 64 K] (pieces along K) or MN-major [128 K x 64 MN]
   // (pieces along MN).
-  static constexpr int PK = (A_MN || B_MN) ? 128 : 64;
+  static_assert(PK == 64 || PK == 128, "K block of 64 or 128");
   static constexpr int A_BYTES = 128 * PK * 2;          // this CTA's 128 rows
   static constexpr int B_BYTES = (PN / 2) * PK * 2;     // this CTA's 128 columns
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = PK == 64 ? 6 : 3;
-  static constexpr int PIECES = PK == 64 ? 1 : 2;       // 16 KiB pieces per operand per stage
+  static constexpr int PIECES = PK / 64;                // 16 KiB pieces per operand per stage
   static constexpr int TMEM_COLS = 512;                 // two 128 x 256 fp32 accumulators
   static constexpr int ACC_STRIDE = 256;
   static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
@@ -78,14 +113,36 @@ struct PairCfg {
   static constexpr size_t SMEM = 1024 + (size_t)OFF_EPI + 4 * 4096;
 };
 
-template <bool A_MN, bool B_MN>
+// The i-th item (tile) of this pair, or -1 past its last.
+__device__ __forceinline__ int pair_item(const PairParams& p, int pair, int npairs, int i) {
+  if (p.sched) {
+    const int k = (int)p.first[pair] + i;
+    return k < (int)p.first[pair + 1] ? (int)p.order[k] : -1;
+  }
+  const int t = pair + i * npairs;
+  return t < p.n_items ? t : -1;
+}
+
+struct PairTile {
+  int prob, tm, tn;
+};
+
+__device__ __forceinline__ PairTile pair_tile(const PairParams& p, int item) {
+  PairTile t;
+  t.prob = item >= p.tiles0 ? 1 : 0;
+  const int r = item - (t.prob ? p.tiles0 : 0);
+  const int tiles_m = p.pr[t.prob].tiles_m;
+  t.tm = r % tiles_m;
+  t.tn = r / tiles_m;
+  return t;
+}
+
+template <int PK>
 __global__ void __launch_bounds__(PAIR_THREADS, 1)
-    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-                        const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
-                        PairParams p) {
-  using C = PairCfg<A_MN, B_MN>;
+    tc_gemm_pair_kernel(const __grid_constant__ PairMaps mp0, const __grid_constant__ PairMaps mp1,
+                        const __grid_constant__ PairParams p) {
+  using C = PairCfg<PK>;
   constexpr int STAGES = C::STAGES;
-  constexpr int PK = C::PK;
   extern __shared__ uint8_t smem_raw[];
   // the same offset in both CTAs: the pair MMA reads both CTAs' operands at one address
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -116,10 +173,16 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tmA0);
-    tma_prefetch_desc(&tmA1);
-    tma_prefetch_desc(&tmB0);
-    tma_prefetch_desc(&tmB1);
+    tma_prefetch_desc(&mp0.a0);
+    tma_prefetch_desc(&mp0.a1);
+    tma_prefetch_desc(&mp0.b0);
+    tma_prefetch_desc(&mp0.b1);
+    if (p.tiles0 < p.n_items) {
+      tma_prefetch_desc(&mp1.a0);
+      tma_prefetch_desc(&mp1.a1);
+      tma_prefetch_desc(&mp1.b0);
+      tma_prefetch_desc(&mp1.b1);
+    }
   }
   if (warp == 1) tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
   __syncthreads();
@@ -127,10 +190,7 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int num_tiles = p.tiles_m * p.tiles_n;
   const int pair = (int)blockIdx.x >> 1, npairs = (int)gridDim.x >> 1;
-  const int kblocks = (p.K + C::PK - 1) / C::PK;
-  constexpr uint32_t IDESC = idesc_bf16(PM, PN, A_MN, B_MN);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -138,11 +198,15 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int t = pair; t < num_tiles && ok; t += npairs) {
-        const int tm = t % p.tiles_m, tn = t / p.tiles_m;
-        const int m0 = tm * PM + 128 * (int)rank;  // this CTA's A rows
-        const int n0 = tn * PN + 128 * (int)rank;  // this CTA's B columns
-        for (int kb = 0; kb < kblocks; ++kb) {
+      for (int i = 0; ok; ++i) {
+        const int item = pair_item(p, pair, npairs, i);
+        if (item < 0) break;
+        const PairTile tl = pair_tile(p, item);
+        const PairProblem& pr = p.pr[tl.prob];
+        const PairMaps& mp = tl.prob ? mp1 : mp0;
+        const int m0 = tl.tm * PM + 128 * (int)rank;  // this CTA's A rows
+        const int n0 = tl.tn * PN + 128 * (int)rank;  // this CTA's B columns
+        for (int kb = 0; kb < pr.kblocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, ab)) {
             ok = false;
             break;
@@ -152,44 +216,45 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
           uint8_t* dA = sA + stage * C::A_BYTES;
           uint8_t* dB = sB + stage * C::B_BYTES;
           const int k0 = kb * PK;
-          if constexpr (!A_MN && B_MN) {
-            if (p.k_layers > 0) {  // layer-strided K: (k or v, layer l, k within the layer)
-              const int LD = p.k_layers * p.a_switch_k;
+          bool done = false;
+          if constexpr (PK == 128) {
+            if (pr.k_layers > 0) {  // layer-strided K (A K-major, B MN-major): (k or v, layer l, k within the layer)
+              const int LD = pr.k_layers * pr.a_switch_k;
               const int which = k0 >= LD ? 1 : 0;
               const int kr = k0 - which * LD;
-              const int l = kr / p.a_switch_k, kk = kr - l * p.a_switch_k;
+              const int l = kr / pr.a_switch_k, kk = kr - l * pr.a_switch_k;
 #pragma unroll
-              for (int h = 0; h < 2; ++h) {  // A K-major, B MN-major: PK = 128
-                tma_load_3d_pair(dA + h * 16384, which ? &tmA1 : &tmA0, bar, kk + 64 * h, m0, l);
-                tma_load_3d_pair(dB + h * 16384, which ? &tmB1 : &tmB0, bar, n0 + 64 * h, kk, l);
+              for (int h = 0; h < 2; ++h) {
+                tma_load_3d_pair(dA + h * 16384, which ? &mp.a1 : &mp.a0, bar, kk + 64 * h, m0, l);
+                tma_load_3d_pair(dB + h * 16384, which ? &mp.b1 : &mp.b0, bar, n0 + 64 * h, kk, l);
               }
-              if (++stage == STAGES) {
-                stage = 0;
-                phase ^= 1;
-              }
-              continue;
+              done = true;
             }
           }
-          // operand A: this CTA's 128 rows; halves along K (K-major) or M (MN-major).
-          // The k / v switches fall on multiples of 128 (checked by the host).
-          {
-            const bool second = (p.a_switch_m > 0 && m0 >= p.a_switch_m) || (p.a_switch_k > 0 && k0 >= p.a_switch_k);
-            const CUtensorMap* m = second ? &tmA1 : &tmA0;
-            const int mm = (p.a_switch_m > 0 && m0 >= p.a_switch_m) ? m0 - p.a_switch_m : m0;
-            const int kk = (p.a_switch_k > 0 && k0 >= p.a_switch_k) ? k0 - p.a_switch_k : k0;
+          if (!done) {
+            // operand A: this CTA's 128 rows; pieces along K (K-major) or M (MN-major).
+            // The k / v switches fall on multiples of 128 (checked by the host).
+            {
+              const bool sw_m = pr.a_switch_m > 0 && m0 >= pr.a_switch_m;
+              const bool sw_k = pr.a_switch_k > 0 && k0 >= pr.a_switch_k;
+              const CUtensorMap* m = (sw_m || sw_k) ? &mp.a1 : &mp.a0;
+              const int mm = sw_m ? m0 - pr.a_switch_m : m0;
+              const int kk = sw_k ? k0 - pr.a_switch_k : k0;
 #pragma unroll
-            for (int h = 0; h < C::PIECES; ++h)
-              tma_load_2d_pair(dA + h * 16384, m, bar, A_MN ? mm + 64 * h : kk + 64 * h, A_MN ? kk : mm);
-          }
-          // operand B: this CTA's 128 columns; halves along K (K-major) or N (MN-major)
-          {
-            const bool second = (p.b_switch_n > 0 && n0 >= p.b_switch_n) || (p.b_switch_k > 0 && k0 >= p.b_switch_k);
-            const CUtensorMap* m = second ? &tmB1 : &tmB0;
-            const int nn = (p.b_switch_n > 0 && n0 >= p.b_switch_n) ? n0 - p.b_switch_n : n0;
-            const int kk = (p.b_switch_k > 0 && k0 >= p.b_switch_k) ? k0 - p.b_switch_k : k0;
+              for (int h = 0; h < C::PIECES; ++h)
+                tma_load_2d_pair(dA + h * 16384, m, bar, pr.a_mn ? mm + 64 * h : kk + 64 * h, pr.a_mn ? kk : mm);
+            }
+            // operand B: this CTA's 128 columns; pieces along K (K-major) or N (MN-major)
+            {
+              const bool sw_n = pr.b_switch_n > 0 && n0 >= pr.b_switch_n;
+              const bool sw_k = pr.b_switch_k > 0 && k0 >= pr.b_switch_k;
+              const CUtensorMap* m = (sw_n || sw_k) ? &mp.b1 : &mp.b0;
+              const int nn = sw_n ? n0 - pr.b_switch_n : n0;
+              const int kk = sw_k ? k0 - pr.b_switch_k : k0;
 #pragma unroll
-            for (int h = 0; h < C::PIECES; ++h)
-              tma_load_2d_pair(dB + h * 16384, m, bar, B_MN ? nn + 64 * h : kk + 64 * h, B_MN ? kk : nn);
+              for (int h = 0; h < C::PIECES; ++h)
+                tma_load_2d_pair(dB + h * 16384, m, bar, pr.b_mn ? nn + 64 * h : kk + 64 * h, pr.b_mn ? kk : nn);
+            }
           }
           if (++stage == STAGES) {
             stage = 0;
@@ -215,11 +280,16 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int t = pair; t < num_tiles && ok; t += npairs) {
+      for (int i = 0; ok; ++i) {
+        const int item = pair_item(p, pair, npairs, i);
+        if (item < 0) break;
+        const PairProblem& pr = p.pr[pair_tile(p, item).prob];
+        const bool a_mn = pr.a_mn != 0, b_mn = pr.b_mn != 0;
+        const uint32_t idesc = idesc_bf16(PM, PN, a_mn, b_mn);
         if (!warp_wait(&tempty[acc], acc_phase ^ 1, ab)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * C::ACC_STRIDE);
-        for (int kb = 0; kb < kblocks; ++kb) {
+        for (int kb = 0; kb < pr.kblocks; ++kb) {
           if (!warp_wait(&full[stage], phase, ab)) {
             ok = false;
             break;
@@ -230,14 +300,14 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
           if (elect_one()) {
 #pragma unroll
             for (int k16 = 0; k16 < PK / 16; ++k16) {
-              // K-major: half k16 / 4, 32 bytes per 16 K inside it; MN-major: 16 K rows
-              // of 128 B per step, the two MN halves 16 KiB apart
+              // K-major: piece k16 / 4, 32 bytes per 16 K inside it; MN-major: 16 K rows
+              // of 128 B per step, the two MN pieces 16 KiB apart
               const uint32_t koff = (uint32_t)(k16 >> 2) * 16384u + (uint32_t)(k16 & 3) * 32u;
-              const uint64_t ad = A_MN ? sw128_desc(a_addr + (uint32_t)k16 * 2048u, 16384u, 1024u)
+              const uint64_t ad = a_mn ? sw128_desc(a_addr + (uint32_t)k16 * 2048u, 16384u, 1024u)
                                        : sw128_desc(a_addr + koff, 16u, 1024u);
-              const uint64_t bd = B_MN ? sw128_desc(b_addr + (uint32_t)k16 * 2048u, 16384u, 1024u)
+              const uint64_t bd = b_mn ? sw128_desc(b_addr + (uint32_t)k16 * 2048u, 16384u, 1024u)
                                        : sw128_desc(b_addr + koff, 16u, 1024u);
-              mma_ss_pair(d_tmem, ad, bd, IDESC, (kb > 0 || k16 > 0) ? 1u : 0u);
+              mma_ss_pair(d_tmem, ad, bd, idesc, (kb > 0 || k16 > 0) ? 1u : 0u);
             }
             mma_commit_pair_both(&empty[stage]);  // the stage is free in both CTAs
           }
@@ -271,16 +341,19 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
     uint8_t* stg = smem + C::OFF_EPI + q * 4096;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = pair; t < num_tiles; t += npairs) {
-      const int tm = t % p.tiles_m, tn = t / p.tiles_m;
-      const int m0 = tm * PM + 128 * (int)rank, n0 = tn * PN;
+    for (int i = 0;; ++i) {
+      const int item = pair_item(p, pair, npairs, i);
+      if (item < 0) break;
+      const PairTile tl = pair_tile(p, item);
+      const PairProblem& pr = p.pr[tl.prob];
+      const int m0 = tl.tm * PM + 128 * (int)rank, n0 = tl.tn * PN;
       if (!warp_wait(&tfull[acc], acc_phase, ab)) break;
       tc_fence_after();
-      bf16* out = static_cast<bf16*>(p.out0);
+      bf16* out = static_cast<bf16*>(pr.out0);
       int om0 = m0 + q * 32;  // first row of this warp in the output tensor
-      if (p.out_switch_m > 0 && m0 >= p.out_switch_m) {
-        out = static_cast<bf16*>(p.out1);
-        om0 -= p.out_switch_m;
+      if (pr.out_switch_m > 0 && m0 >= pr.out_switch_m) {
+        out = static_cast<bf16*>(pr.out1);
+        om0 -= pr.out_switch_m;
       }
 #pragma unroll 1
       for (int c0 = 0; c0 < PN; c0 += 64) {
@@ -301,22 +374,22 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
         // 64 columns [col0, col0 + 64): this tensor, or the second one past out_switch_n
         const int col0 = n0 + c0;
         bf16* o = out;
-        int ocol0 = col0, n_lim = p.N;
-        if (p.out_switch_n > 0) {
-          if (col0 >= p.out_switch_n) {
-            o = static_cast<bf16*>(p.out1);
-            ocol0 -= p.out_switch_n;
+        int ocol0 = col0, n_lim = pr.N;
+        if (pr.out_switch_n > 0) {
+          if (col0 >= pr.out_switch_n) {
+            o = static_cast<bf16*>(pr.out1);
+            ocol0 -= pr.out_switch_n;
           } else {
-            n_lim = p.out_switch_n;
+            n_lim = pr.out_switch_n;
           }
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int rr = 4 * i + (lane >> 3), j = lane & 7;  // row of the warp's 32, 16-byte chunk
+        for (int k = 0; k < 8; ++k) {
+          const int rr = 4 * k + (lane >> 3), j = lane & 7;  // row of the warp's 32, 16-byte chunk
           const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 128 + ((j ^ (rr & 7)) << 4));
-          if (m0 + q * 32 + rr < p.M && col0 + 8 * j + 8 <= n_lim &&
-              MAGLEV_CHECK(p.err, om0 + rr >= 0 && ocol0 >= 0 && ocol0 + 8 * j + 8 <= p.ldo))
-            *reinterpret_cast<uint4*>(o + (int64_t)(om0 + rr) * p.ldo + ocol0 + 8 * j) = v;
+          if (m0 + q * 32 + rr < pr.M && col0 + 8 * j + 8 <= n_lim &&
+              MAGLEV_CHECK(p.err, om0 + rr >= 0 && ocol0 >= 0 && ocol0 + 8 * j + 8 <= pr.ldo))
+            *reinterpret_cast<uint4*>(o + (int64_t)(om0 + rr) * pr.ldo + ocol0 + 8 * j) = v;
         }
         __syncwarp();
       }
@@ -343,12 +416,12 @@ namespace {
 
 // Largest number of two-CTA clusters of this kernel that can be resident at
 // once (0 when clusters cannot be launched), cached per instantiation.
-template <bool A_MN, bool B_MN>
+template <int PK>
 int max_pairs() {
   static int cached = -1;
   if (cached >= 0) return cached;
-  using C = PairCfg<A_MN, B_MN>;
-  auto kern = tc_gemm_pair_kernel<A_MN, B_MN>;
+  using C = PairCfg<PK>;
+  auto kern = tc_gemm_pair_kernel<PK>;
   int n = 0;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM) == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
@@ -365,18 +438,47 @@ int max_pairs() {
     if (cudaOccupancyMaxActiveClusters(&n, (void*)kern, &cfg) != cudaSuccess) n = 0;
   }
   (void)cudaGetLastError();
-  cached = n;
-  return n;
+  cached = n < PAIR_MAX_PAIRS ? n : PAIR_MAX_PAIRS;
+  return cached;
 }
 
-template <bool A_MN, bool B_MN>
-cudaError_t run_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0, const CUtensorMap& b1,
-                     PairParams p, cudaStream_t s) {
-  using C = PairCfg<A_MN, B_MN>;
-  const int cap = max_pairs<A_MN, B_MN>();
+// Longest processing time first: items in decreasing K-block count (ties in
+// item order), each to the pair with the least work so far (ties to the lower
+// pair); a pair runs its items in the order they were dealt.
+void lpt_schedule(PairParams& p, int pairs) {
+  std::vector<int> items(p.n_items);
+  for (int i = 0; i < p.n_items; ++i) items[i] = i;
+  auto cost = [&](int it) { return p.pr[it >= p.tiles0 ? 1 : 0].kblocks; };
+  std::stable_sort(items.begin(), items.end(), [&](int x, int y) { return cost(x) > cost(y); });
+  using Load = std::pair<int64_t, int>;  // (work so far, pair)
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+  for (int i = 0; i < pairs; ++i) heap.push({0, i});
+  std::vector<std::vector<uint16_t>> lists(pairs);
+  for (int it : items) {
+    Load l = heap.top();
+    heap.pop();
+    lists[l.second].push_back((uint16_t)it);
+    heap.push({l.first + cost(it), l.second});
+  }
+  int k = 0;
+  for (int i = 0; i < pairs; ++i) {
+    p.first[i] = (uint16_t)k;
+    for (uint16_t it : lists[i]) p.order[k++] = it;
+  }
+  p.first[pairs] = (uint16_t)k;
+  p.sched = 1;
+}
+
+template <int PK>
+cudaError_t run_pair(const PairMaps& m0, const PairMaps& m1, PairParams& p, bool schedule, cudaStream_t s) {
+  using C = PairCfg<PK>;
+  const int cap = max_pairs<PK>();
   if (cap < 1) return cudaErrorNotSupported;
-  const int tiles = p.tiles_m * p.tiles_n;
-  const int pairs = tiles < cap ? tiles : cap;
+  const int pairs = p.n_items < cap ? p.n_items : cap;
+  if (schedule) {
+    if (p.n_items > PAIR_MAX_ITEMS) return cudaErrorNotSupported;
+    lpt_schedule(p, pairs);
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.blockDim = dim3(PAIR_THREADS, 1, 1);
@@ -389,20 +491,64 @@ cudaError_t run_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUtenso
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<A_MN, B_MN>, a0, a1, b0, b1, p);
+  return cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<PK>, m0, m1, p);
 }
 
-PairParams pair_params(int M, int N, int K, int64_t ldo, int64_t spin_limit, int* err) {
+PairProblem pair_problem(int M, int N, int K, bool a_mn, bool b_mn, int64_t ldo) {
+  PairProblem q{};
+  q.M = M;
+  q.N = N;
+  q.K = K;
+  q.tiles_m = (M + PM - 1) / PM;
+  q.tiles_n = (N + PN - 1) / PN;
+  q.kblocks = (K + ((a_mn || b_mn) ? 128 : 64) - 1) / ((a_mn || b_mn) ? 128 : 64);
+  q.a_mn = a_mn ? 1 : 0;
+  q.b_mn = b_mn ? 1 : 0;
+  q.ldo = ldo;
+  return q;
+}
+
+PairParams pair_params(const PairProblem& q0, int64_t spin_limit, int* err) {
   PairParams p{};
-  p.M = M;
-  p.N = N;
-  p.K = K;
-  p.tiles_m = (M + PM - 1) / PM;
-  p.tiles_n = (N + PN - 1) / PN;
-  p.ldo = ldo;
+  p.pr[0] = q0;
+  p.pr[1] = q0;
+  p.tiles0 = q0.tiles_m * q0.tiles_n;
+  p.n_items = p.tiles0;
   p.spin_limit = spin_limit;
   p.err = err;
   return p;
+}
+
+// Problem and maps of dm [M, d] = dR_k [M, D] W_mk [D, d] + dR_v W_mv (K = 2D, B N-contiguous).
+cudaError_t dm_problem(int64_t M, int D, int d, const void* dRk, const void* dRv, const void* w_mk,
+                       const void* w_mv, void* dm, PairMaps& mp, PairProblem& q) {
+  cudaError_t e;
+  if ((e = make_tmap_bf16_2d(&mp.a0, dRk, D, M, (uint64_t)D * 2, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&mp.a1, dRv, D, M, (uint64_t)D * 2, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&mp.b0, w_mk, d, D, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&mp.b1, w_mv, d, D, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
+  q = pair_problem((int)M, d, 2 * D, false, true, d);
+  q.a_switch_k = D;
+  q.b_switch_k = D;
+  q.out0 = dm;
+  q.out1 = dm;
+  return cudaSuccess;
+}
+
+// Problem and maps of dW_mk | dW_mv [D, d] = dR^T [D, M] m_shift [M, d] (A and B both M-contiguous).
+cudaError_t dw_problem(int64_t M, int D, int d, const void* dRk, const void* dRv, const void* m_shift, void* dwk,
+                       void* dwv, PairMaps& mp, PairProblem& q) {
+  cudaError_t e;
+  if ((e = make_tmap_bf16_2d(&mp.a0, dRk, D, M, (uint64_t)D * 2, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&mp.a1, dRv, D, M, (uint64_t)D * 2, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&mp.b0, m_shift, d, M, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
+  mp.b1 = mp.b0;
+  q = pair_problem(2 * D, d, (int)M, true, true, d);
+  q.a_switch_m = D;
+  q.out_switch_m = D;
+  q.out0 = dwk;
+  q.out1 = dwv;
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -415,69 +561,85 @@ bool pair_gemm_supported(int D) { return D % 128 == 0; }
 // R_k | R_v [M, D] = m_shift [M, d] x W^T, W_mk / W_mv [D, d].
 cudaError_t launch_proj_fwd_pair(int64_t M, int D, int d, const void* m_shift, const void* w_mk, const void* w_mv,
                                  void* Rk, void* Rv, int64_t spin_limit, int* err, cudaStream_t s) {
-  CUtensorMap a, b0, b1;
+  PairMaps mp;
   cudaError_t e;
-  if ((e = make_tmap_bf16_2d(&a, m_shift, d, M, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
-  if ((e = make_tmap_bf16_2d(&b0, w_mk, d, D, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
-  if ((e = make_tmap_bf16_2d(&b1, w_mv, d, D, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
-  PairParams p = pair_params((int)M, 2 * D, d, D, spin_limit, err);
-  p.b_switch_n = D;
-  p.out_switch_n = D;
-  p.out0 = Rk;
-  p.out1 = Rv;
-  return run_pair<false, false>(a, a, b0, b1, p, s);
+  if ((e = make_tmap_bf16_2d(&mp.a0, m_shift, d, M, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&mp.b0, w_mk, d, D, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&mp.b1, w_mv, d, D, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
+  mp.a1 = mp.a0;
+  PairProblem q = pair_problem((int)M, 2 * D, d, false, false, D);
+  q.b_switch_n = D;
+  q.out_switch_n = D;
+  q.out0 = Rk;
+  q.out1 = Rv;
+  PairParams p = pair_params(q, spin_limit, err);
+  return run_pair<64>(mp, mp, p, false, s);
 }
 
 // dm [M, d] = dR_k [M, D] W_mk [D, d] + dR_v W_mv (K = 2D, B operand N-contiguous).
 cudaError_t launch_proj_bwd_dm_pair(int64_t M, int D, int d, const void* dRk, const void* dRv, const void* w_mk,
                                     const void* w_mv, void* dm, int64_t spin_limit, int* err, cudaStream_t s) {
-  CUtensorMap a0, a1, b0, b1;
+  PairMaps mp;
+  PairProblem q;
   cudaError_t e;
-  if ((e = make_tmap_bf16_2d(&a0, dRk, D, M, (uint64_t)D * 2, 64, 128)) != cudaSuccess) return e;
-  if ((e = make_tmap_bf16_2d(&a1, dRv, D, M, (uint64_t)D * 2, 64, 128)) != cudaSuccess) return e;
-  if ((e = make_tmap_bf16_2d(&b0, w_mk, d, D, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
-  if ((e = make_tmap_bf16_2d(&b1, w_mv, d, D, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
-  PairParams p = pair_params((int)M, d, 2 * D, d, spin_limit, err);
-  p.a_switch_k = D;
-  p.b_switch_k = D;
-  p.out0 = dm;
-  p.out1 = dm;
-  return run_pair<false, true>(a0, a1, b0, b1, p, s);
+  if ((e = dm_problem(M, D, d, dRk, dRv, w_mk, w_mv, dm, mp, q)) != cudaSuccess) return e;
+  PairParams p = pair_params(q, spin_limit, err);
+  return run_pair<128>(mp, mp, p, false, s);
 }
 
 // dm [M, d] = sum over L layers of dR_k^l W_mk^l + dR_v^l W_mv^l (layer-strided, K = 2 L D).
 cudaError_t launch_proj_bwd_dm_layers_pair(int64_t M, int D, int d, int L, const void* dRk, const void* dRv,
                                            const void* w_mk, const void* w_mv, void* dm, int64_t spin_limit,
                                            int* err, cudaStream_t s) {
-  CUtensorMap a0, a1, b0, b1;
+  PairMaps mp;
   cudaError_t e;
-  if ((e = make_tmap_bf16_3d(&a0, dRk, D, M, L, 64, 128)) != cudaSuccess) return e;
-  if ((e = make_tmap_bf16_3d(&a1, dRv, D, M, L, 64, 128)) != cudaSuccess) return e;
-  if ((e = make_tmap_bf16_3d(&b0, w_mk, d, D, L, 64, 128)) != cudaSuccess) return e;
-  if ((e = make_tmap_bf16_3d(&b1, w_mv, d, D, L, 64, 128)) != cudaSuccess) return e;
-  PairParams p = pair_params((int)M, d, 2 * L * D, d, spin_limit, err);
-  p.a_switch_k = D;
-  p.b_switch_k = D;
-  p.k_layers = L;
-  p.out0 = dm;
-  p.out1 = dm;
-  return run_pair<false, true>(a0, a1, b0, b1, p, s);
+  if ((e = make_tmap_bf16_3d(&mp.a0, dRk, D, M, L, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_3d(&mp.a1, dRv, D, M, L, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_3d(&mp.b0, w_mk, d, D, L, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_3d(&mp.b1, w_mv, d, D, L, 64, 128)) != cudaSuccess) return e;
+  PairProblem q = pair_problem((int)M, d, 2 * L * D, false, true, d);
+  q.a_switch_k = D;
+  q.b_switch_k = D;
+  q.k_layers = L;
+  q.out0 = dm;
+  q.out1 = dm;
+  PairParams p = pair_params(q, spin_limit, err);
+  return run_pair<128>(mp, mp, p, false, s);
 }
 
 // dW_mk | dW_mv [D, d] = dR^T [D, M] m_shift [M, d] (A and B both M-contiguous in memory).
 cudaError_t launch_proj_bwd_dw_pair(int64_t M, int D, int d, const void* dRk, const void* dRv, const void* m_shift,
                                     void* dwk, void* dwv, int64_t spin_limit, int* err, cudaStream_t s) {
-  CUtensorMap a0, a1, b;
+  PairMaps mp;
+  PairProblem q;
   cudaError_t e;
-  if ((e = make_tmap_bf16_2d(&a0, dRk, D, M, (uint64_t)D * 2, 64, 128)) != cudaSuccess) return e;
-  if ((e = make_tmap_bf16_2d(&a1, dRv, D, M, (uint64_t)D * 2, 64, 128)) != cudaSuccess) return e;
-  if ((e = make_tmap_bf16_2d(&b, m_shift, d, M, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
-  PairParams p = pair_params(2 * D, d, (int)M, d, spin_limit, err);
-  p.a_switch_m = D;
-  p.out_switch_m = D;
-  p.out0 = dwk;
-  p.out1 = dwv;
-  return run_pair<true, true>(a0, a1, b, b, p, s);
+  if ((e = dw_problem(M, D, d, dRk, dRv, m_shift, dwk, dwv, mp, q)) != cudaSuccess) return e;
+  PairParams p = pair_params(q, spin_limit, err);
+  return run_pair<128>(mp, mp, p, false, s);
+}
+
+// Whether launch_proj_bwd_grouped_pair can run dW and dm of these sizes.
+bool proj_bwd_grouped_available(int64_t M, int D, int d) {
+  if (!pair_gemm_supported(D) || max_pairs<128>() < 1) return false;
+  const int64_t tiles = ((2 * (int64_t)D + PM - 1) / PM + (M + PM - 1) / PM) * (((int64_t)d + PN - 1) / PN);
+  return tiles <= PAIR_MAX_ITEMS;
+}
+
+// dW and dm in one launch, their tiles dealt longest first over the SM pairs.
+// cudaErrorNotSupported when clusters cannot be launched or the two have more
+// than 512 tiles; the caller then launches them one by one.
+cudaError_t launch_proj_bwd_grouped_pair(int64_t M, int D, int d, const void* dRk, const void* dRv, const void* w_mk,
+                                         const void* w_mv, const void* m_shift, void* dm, void* dwk, void* dwv,
+                                         int64_t spin_limit, int* err, cudaStream_t s) {
+  PairMaps mw, mm;
+  PairProblem qw, qm;
+  cudaError_t e;
+  if ((e = dw_problem(M, D, d, dRk, dRv, m_shift, dwk, dwv, mw, qw)) != cudaSuccess) return e;
+  if ((e = dm_problem(M, D, d, dRk, dRv, w_mk, w_mv, dm, mm, qm)) != cudaSuccess) return e;
+  PairParams p = pair_params(qw, spin_limit, err);
+  p.pr[1] = qm;
+  p.n_items = p.tiles0 + qm.tiles_m * qm.tiles_n;
+  return run_pair<128>(mw, mm, p, true, s);
 }
 
 }  // namespace maglev

@@ -241,6 +241,36 @@ def test_accumulated_memory_gradient_over_layers(dtype, hd, n_layers):
     assert_close(host(dRv), want_v, dtype, "dR_v sum")
 
 
+# --------------------------------------------------------------------------- projection backward alone
+@pytest.mark.parametrize("which", ["both", "dm", "dw"])
+def test_mem_project_bwd_outputs(which):
+    """maglev_mem_project_bwd on its own: dm_shift and dW together (one launch
+    that deals the tiles of both over the SM pairs) and each alone (a launch of
+    its own), with ragged rows (B*T = 600, K of dW not a multiple of the K block)
+    and ragged columns (d = 384, half a pair tile past 256)."""
+    B, T, H, hd, d = 2, 300, 2, 128, 384
+    D = H * hd
+    seed = 77
+    m = synth.normal(seed, 901, (B, T, d))
+    wk = synth.normal(seed, 902, (D, d), std=d ** -0.5)
+    wv = synth.normal(seed, 903, (D, d), std=d ** -0.5)
+    dRk = synth.normal(seed, 904, (B, T, D))
+    dRv = synth.normal(seed, 905, (B, T, D))
+    L = InjectedSWALayer(B, T, H, hd, d, 64, dtype="bf16")
+    dm = torch.full((B, T, d), float("nan"), dtype=torch.bfloat16, device="cuda") if which != "dw" else None
+    dwk = torch.full((D, d), float("nan"), dtype=torch.bfloat16, device="cuda") if which != "dm" else None
+    dwv = torch.full((D, d), float("nan"), dtype=torch.bfloat16, device="cuda") if which != "dm" else None
+    mg.maglev_mem_project_bwd(L.desc, dev(m), dev(wk), dev(wv), dev(dRk), dev(dRv), dm, dwk, dwv)
+    torch.cuda.synchronize()
+    ref_dm, ref_dwk, ref_dwv = oracle.mem_project_backward(m.f64, wk.f64, wv.f64, dRk.f64, dRv.f64)
+    if dm is not None:
+        assert_close(host(dm), ref_dm, "bf16", "dm_shift")
+    if dwk is not None:
+        assert_close(host(dwk), ref_dwk, "bf16", "dw_mk")
+        assert_close(host(dwv), ref_dwv, "bf16", "dw_mv")
+    assert mg.maglev_device_status() == 0
+
+
 # --------------------------------------------------------------------------- consistency loss
 @pytest.mark.parametrize("dtype,rows,d", [("f32", 256, 128), ("bf16", 8192, 1280), ("bf16", 3, 17)])
 def test_consistency_loss(dtype, rows, d):
