@@ -119,14 +119,15 @@ struct RopeTable {
   double inv_freq[64];  // base^(-2c/hd), c < hd/2
 };
 
+// One (row, u) item of prep: thread gid of a grid that covers B*T*H rows with
+// hd/16 threads each (gid past the end: a thread that only joins the row sums).
 template <typename T, int HD>
-__global__ void __launch_bounds__(256) prep_vec_kernel(SwaShape s, RopeTable rt, const T* __restrict__ q,
-                                                       const T* __restrict__ k, const T* __restrict__ v,
-                                                       const T* __restrict__ Rk, const T* __restrict__ Rv,
-                                                       const float* __restrict__ gates, T* __restrict__ qr,
-                                                       T* __restrict__ kb, T* __restrict__ vb) {
+__device__ __forceinline__ void prep_item(int64_t gid, const SwaShape& s, const RopeTable& rt,
+                                          const T* __restrict__ q, const T* __restrict__ k,
+                                          const T* __restrict__ v, const T* __restrict__ Rk,
+                                          const T* __restrict__ Rv, const float* __restrict__ gates,
+                                          T* __restrict__ qr, T* __restrict__ kb, T* __restrict__ vb) {
   constexpr int HALF = HD / 2, TPR = HD / 16;
-  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t row = gid / TPR;
   const int u = (int)(gid % TPR);
   const int64_t nrows = (int64_t)s.B * s.T * s.H;
@@ -136,10 +137,26 @@ __global__ void __launch_bounds__(256) prep_vec_kernel(SwaShape s, RopeTable rt,
   const int t = (int)((rr / s.H) % s.T);
   const int64_t p = (int64_t)s.pos0 + t;
   const int64_t b1 = rr * HD + 8 * u, b2 = b1 + HALF;
+  // every load first; the RoPE angles are computed while they are in flight
+  Raw8<T> q1r{}, q2r{}, k1r{}, k2r{}, v1r{}, v2r{}, r1r{}, r2r{}, w1r{}, w2r{};
+  if (live) {
+    q1r = raw8(q + b1);
+    q2r = raw8(q + b2);
+    k1r = raw8(k + b1);
+    k2r = raw8(k + b2);
+    v1r = raw8(v + b1);
+    v2r = raw8(v + b2);
+    if (s.inject) {
+      r1r = raw8(Rk + b1);
+      r2r = raw8(Rk + b2);
+      w1r = raw8(Rv + b1);
+      w2r = raw8(Rv + b2);
+    }
+  }
   float cs[8], sn[8];
   rope8(p, rt.inv_freq, 8 * u, cs, sn);
   if (live) {
-    const V8 q1 = load8(q + b1), q2 = load8(q + b2);
+    const V8 q1 = cvt8(q1r), q2 = cvt8(q2r);
     V8 o1, o2;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -149,9 +166,9 @@ __global__ void __launch_bounds__(256) prep_vec_kernel(SwaShape s, RopeTable rt,
     store8(qr + b1, o1);
     store8(qr + b2, o2);
   }
-  V8 k1 = {}, k2 = {};
-  if (live) {
-    const V8 a = load8(k + b1), c = load8(k + b2);
+  V8 k1, k2;
+  {
+    const V8 a = cvt8(k1r), c = cvt8(k2r);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       k1.x[e] = a.x[e] * cs[e] - c.x[e] * sn[e];
@@ -162,19 +179,15 @@ __global__ void __launch_bounds__(256) prep_vec_kernel(SwaShape s, RopeTable rt,
     if (live) {
       store8(kb + b1, k1);
       store8(kb + b2, k2);
-      store8(vb + b1, load8(v + b1));
-      store8(vb + b2, load8(v + b2));
+      store8(vb + b1, cvt8(v1r));
+      store8(vb + b2, cvt8(v2r));
     }
     return;
   }
-  V8 r1 = {}, r2 = {};
+  const V8 r1 = cvt8(r1r), r2 = cvt8(r2r);
   float ss = 0.f;
-  if (live) {
-    r1 = load8(Rk + b1);
-    r2 = load8(Rk + b2);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) ss += r1.x[e] * r1.x[e] + r2.x[e] * r2.x[e];
-  }
+  for (int e = 0; e < 8; ++e) ss += r1.x[e] * r1.x[e] + r2.x[e] * r2.x[e];
   ss = row_sum<TPR>(ss);
   if (!live) return;
   const float rinv = rsqrtf(ss / HD + s.eps);
@@ -189,7 +202,7 @@ __global__ void __launch_bounds__(256) prep_vec_kernel(SwaShape s, RopeTable rt,
   }
   store8(kb + b1, o1);
   store8(kb + b2, o2);
-  const V8 va = load8(v + b1), vc = load8(v + b2), ra = load8(Rv + b1), rc = load8(Rv + b2);
+  const V8 va = cvt8(v1r), vc = cvt8(v2r), ra = cvt8(w1r), rc = cvt8(w2r);
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     o1.x[e] = gvl * va.x[e] + gvr * ra.x[e];
@@ -199,15 +212,30 @@ __global__ void __launch_bounds__(256) prep_vec_kernel(SwaShape s, RopeTable rt,
   store8(vb + b2, o2);
 }
 
+// Persistent: the grid fills the SMs once and each thread strides over the
+// items (the stride is a multiple of the block, so a warp's lanes stay in
+// step and its row sums see whole rows).
 template <typename T, int HD>
-__global__ void __launch_bounds__(256, sizeof(T) == 2 ? 2 : 1) unmix_vec_kernel(
-    SwaShape s, RopeTable rt, const T* __restrict__ dkb, const T* __restrict__ dvb,
+__global__ void __launch_bounds__(256) prep_vec_kernel(SwaShape s, RopeTable rt, const T* __restrict__ q,
+                                                       const T* __restrict__ k, const T* __restrict__ v,
+                                                       const T* __restrict__ Rk, const T* __restrict__ Rv,
+                                                       const float* __restrict__ gates, T* __restrict__ qr,
+                                                       T* __restrict__ kb, T* __restrict__ vb) {
+  const int64_t total = (int64_t)s.B * s.T * s.H * (HD / 16);
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < total; base += stride)
+    prep_item<T, HD>(base + threadIdx.x, s, rt, q, k, v, Rk, Rv, gates, qr, kb, vb);
+}
+
+// One (row, u) item of unmix (as prep_item).
+template <typename T, int HD>
+__device__ __forceinline__ void unmix_item(
+    int64_t gid, const SwaShape& s, const RopeTable& rt, const T* __restrict__ dkb, const T* __restrict__ dvb,
     const T* __restrict__ k, const T* __restrict__ v, const T* __restrict__ Rk, const T* __restrict__ Rv,
     const float* __restrict__ gates, T* __restrict__ dk, T* __restrict__ dv, T* __restrict__ dRk,
     T* __restrict__ dRv, float* __restrict__ accRk, float* __restrict__ accRv, int dr_mode,
     float* __restrict__ gpart, const float* __restrict__ dq_acc, T* __restrict__ dq) {
   constexpr int HALF = HD / 2, TPR = HD / 16;
-  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t row = gid / TPR;
   const int u = (int)(gid % TPR);
   const int64_t nrows = (int64_t)s.B * s.T * s.H;
@@ -370,6 +398,23 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 2 : 1) unmix_vec_kernel(
   }
 }
 
+// Persistent, as prep_vec_kernel; two blocks per SM for bf16 (measured: one
+// block at up to 255 registers without spills ran 6% slower, and a version
+// whose 128 registers spilled freshly loaded values ran 20% slower).
+template <typename T, int HD>
+__global__ void __launch_bounds__(256, sizeof(T) == 2 ? 2 : 1) unmix_vec_kernel(
+    SwaShape s, RopeTable rt, const T* __restrict__ dkb, const T* __restrict__ dvb,
+    const T* __restrict__ k, const T* __restrict__ v, const T* __restrict__ Rk, const T* __restrict__ Rv,
+    const float* __restrict__ gates, T* __restrict__ dk, T* __restrict__ dv, T* __restrict__ dRk,
+    T* __restrict__ dRv, float* __restrict__ accRk, float* __restrict__ accRv, int dr_mode,
+    float* __restrict__ gpart, const float* __restrict__ dq_acc, T* __restrict__ dq) {
+  const int64_t total = (int64_t)s.B * s.T * s.H * (HD / 16);
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < total; base += stride)
+    unmix_item<T, HD>(base + threadIdx.x, s, rt, dkb, dvb, k, v, Rk, Rv, gates, dk, dv, dRk, dRv, accRk, accRv,
+                      dr_mode, gpart, dq_acc, dq);
+}
+
 // Delta[b,h,t] = dout . out over hd; also zeroes the fp32 dq accumulator rows.
 template <typename T, int HD>
 __global__ void __launch_bounds__(256) delta_vec_kernel(SwaShape s, const T* __restrict__ out,
@@ -437,6 +482,31 @@ inline unsigned blocks_for(const SwaShape& s, int tpr) {
   return (unsigned)((threads + 255) / 256);
 }
 
+// Grid of a persistent element-wise kernel: as many 256-thread blocks as are
+// resident on all SMs at once (cached per kernel), or fewer if the items run out.
+template <typename Kern>
+unsigned persistent_blocks(Kern kern, int& cached_per_sm, const SwaShape& s, int tpr) {
+  if (cached_per_sm < 1) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 256, 0) != cudaSuccess || n < 1) n = 1;
+    (void)cudaGetLastError();
+    cached_per_sm = n;
+  }
+  const unsigned cap = (unsigned)(num_sms() * cached_per_sm);
+  const unsigned want = blocks_for(s, tpr);
+  return want < cap ? want : cap;
+}
+template <typename T, int HD>
+unsigned prep_blocks(const SwaShape& s) {
+  static int per_sm = 0;
+  return persistent_blocks(prep_vec_kernel<T, HD>, per_sm, s, HD / 16);
+}
+template <typename T, int HD>
+unsigned unmix_blocks(const SwaShape& s) {
+  static int per_sm = 0;
+  return persistent_blocks(unmix_vec_kernel<T, HD>, per_sm, s, HD / 16);
+}
+
 }  // namespace
 
 #define MAGLEV_EW_DISPATCH(DT, HDV, ...)                                                        \
@@ -453,7 +523,7 @@ cudaError_t launch_prep(const SwaShape& s, const void* q, const void* k, const v
                         cudaStream_t st) {
   const RopeTable rt = rope_table(s);
   MAGLEV_EW_DISPATCH(s.dtype, s.hd,
-                     prep_vec_kernel<T, HD><<<blocks_for(s, HD / 16), 256, 0, st>>>(
+                     prep_vec_kernel<T, HD><<<prep_blocks<T, HD>(s), 256, 0, st>>>(
                          s, rt, (const T*)q, (const T*)k, (const T*)v, (const T*)Rk, (const T*)Rv, gates,
                          (T*)q_rot, (T*)k_bar, (T*)v_bar));
   return cudaGetLastError();
@@ -465,7 +535,7 @@ cudaError_t launch_unmix(const SwaShape& s, const void* dk_bar, const void* dv_b
                          const float* dq_acc, void* dq, cudaStream_t st) {
   const RopeTable rt = rope_table(s);
   MAGLEV_EW_DISPATCH(s.dtype, s.hd,
-                     unmix_vec_kernel<T, HD><<<blocks_for(s, HD / 16), 256, 0, st>>>(
+                     unmix_vec_kernel<T, HD><<<unmix_blocks<T, HD>(s), 256, 0, st>>>(
                          s, rt, (const T*)dk_bar, (const T*)dv_bar, (const T*)k, (const T*)v, (const T*)Rk, (const T*)Rv, gates,
                          (T*)dk, (T*)dv, (T*)dRk, (T*)dRv, accRk, accRv, dr_mode, gpart, dq_acc, (T*)dq));
   return cudaGetLastError();
