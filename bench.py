@@ -372,34 +372,56 @@ def run_layer_bench(torch, dist, rank, world, dev, steps, warmup, peaks, peaks_s
 
 
 def run_layer_e2e(torch, dev, steps, warmup, step):
-    """Same step with inputs copied in from pinned host memory and the loss and
-    parameter gradients copied out, every step, inside the timed region."""
-    x = step.x
+    """Same step with every step's inputs copied in from pinned host memory and
+    the loss and parameter gradients copied out, inside the timed region. As an
+    input pipeline that prefetches does, step i+1's inputs are copied on their
+    own stream into a second set of device buffers while step i computes: each
+    step waits for its own inputs, and a buffer set is refilled only after the
+    step that last read it has finished. The results are read back after every
+    step, on the compute stream."""
     names = ("q", "k", "v", "m_shift", "target", "dout", "w_mk", "w_mv", "gates")
-    host = {n: x[n].cpu().pin_memory() for n in names}
+    host = {n: step.x[n].cpu().pin_memory() for n in names}
     L = step.L
     outs = [L.loss, L.dw_mk, L.dw_mv, L.dgate]
     host_out = [o.cpu().pin_memory() for o in outs]
     h2d = sum(host[n].numel() * host[n].element_size() for n in names)
     d2h = sum(o.numel() * o.element_size() for o in outs)
-    stream = torch.cuda.current_stream()
+    compute = torch.cuda.current_stream()
+    copy = torch.cuda.Stream(device=dev)
+    sets = [dict(step.x), {n: torch.empty_like(t) for n, t in step.x.items()}]
+    douts = [step.dout_total, torch.empty_like(step.dout_total)]
+    ready = [torch.cuda.Event(), torch.cuda.Event()]
+    done = [torch.cuda.Event(), torch.cuda.Event()]
+    used = [False, False]
+    x0, dout0 = step.x, step.dout_total
 
-    def e2e_step():
-        for n in names:  # this step's dO lands in the buffer the step accumulates into
-            (step.dout_total if n == "dout" else x[n]).copy_(host[n], non_blocking=True)
+    def e2e_step(i):
+        s = i % 2
+        if used[s]:
+            copy.wait_event(done[s])  # the step that last read this set has finished
+        with torch.cuda.stream(copy):
+            for n in names:  # this step's dO lands in the buffer the step accumulates into
+                (douts[s] if n == "dout" else sets[s][n]).copy_(host[n], non_blocking=True)
+            ready[s].record(copy)
+        compute.wait_event(ready[s])
+        step.x, step.dout_total = sets[s], douts[s]
         step()
         for o, h in zip(outs, host_out):
             h.copy_(o, non_blocking=True)
+        done[s].record(compute)
+        used[s] = True
 
-    for _ in range(max(1, warmup)):
-        e2e_step()
+    for i in range(max(1, warmup)):
+        e2e_step(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(compute)
+    copy.wait_event(e0)  # every timed copy starts after e0
+    for i in range(steps):
+        e2e_step(i)
+    e1.record(compute)
     torch.cuda.synchronize()
+    step.x, step.dout_total = x0, dout0
     return e0.elapsed_time(e1) / steps, h2d, d2h
 
 
