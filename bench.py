@@ -124,6 +124,8 @@ def kernel_work(name: str, cfg: dict) -> tuple[float, str]:
         "unmix": (B * T * D * (4 + 6 * 2 + 5 * 2.0), "byte"),
         # reads m, m', dm; writes dm (the layer step accumulates into dO)
         "consistency_loss": (B * T * D * 2.0 * 4, "byte"),
+        # the same, plus the zeroed fp32 dQ accumulator (Delta itself is B*H*T floats)
+        "consistency_loss_prep": (B * T * D * 12.0, "byte"),
         # reads O, dO (bf16); zeroes the fp32 dQ accumulator
         "attn_delta": (B * T * D * (2.0 * 2 + 4), "byte"),
     }
@@ -255,11 +257,11 @@ class LayerStep:
         self.dout_total = inputs["dout"].clone()
 
     def __call__(self):
-        x, L, D = self.x, self.L, self.D
+        x, L = self.x, self.L
         L.forward(x["q"], x["k"], x["v"], x["gates"], x["m_shift"], x["w_mk"], x["w_mv"])
-        L.consistency(L.out.view(-1, D), x["target"].view(-1, D), LAYER["lam"],
-                      dm=self.dout_total.view(-1, D), accumulate_dm=True)
-        L.backward(x["k"], x["v"], self.dout_total, x["gates"], x["m_shift"], x["w_mk"], x["w_mv"])
+        # the loss of the layer's own output, with the backward's first pass (Delta, dQ accumulator)
+        L.consistency_prepare_bwd(x["target"], LAYER["lam"], self.dout_total)
+        L.backward(x["k"], x["v"], self.dout_total, x["gates"], x["m_shift"], x["w_mk"], x["w_mv"], prepared=True)
 
 
 def aggregate_profile(rows):

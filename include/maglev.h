@@ -175,6 +175,12 @@ typedef enum {
   MAGLEV_DR_LAST = 3
 } maglev_dr_mode;
 
+/* Or'd into dR_mode of maglev_inject_swa_bwd: the backward workspace already
+ * holds Delta and the zeroed dQ accumulator for this out and dout, written by
+ * maglev_consistency_loss_prepare_bwd, so the backward skips its own first
+ * pass over out and dout. */
+#define MAGLEV_BWD_PREPARED 16
+
 /* a6 -- backward of maglev_inject_swa_fwd (chain rule of the forward above).
  *   Inputs: the forward's k, v, R_k, R_v, gate_logits, out, lse, saved, and
  *   dout [B,T,H,hd] = dL/dout.
@@ -183,7 +189,8 @@ typedef enum {
  *     NULL in modes FIRST and ADD, and when inject == 0.
  *   dR_acc_k, dR_acc_v [B,T,D] fp32: the running sums, written (FIRST), updated
  *     (ADD) or read (LAST); unused (may be NULL) in mode WRITE.
- *   dR_mode: a maglev_dr_mode value.
+ *   dR_mode: a maglev_dr_mode value, with MAGLEV_BWD_PREPARED or'd in when
+ *     maglev_consistency_loss_prepare_bwd has run on this out, dout and workspace.
  *   dgate_logits [4,H] fp32 ([2,H] with shared_kv_gates; out, overwritten);
  *     NULL when inject == 0.
  *   m_shift, w_mk, w_mv, dm_shift, dw_mk, dw_mv: if m_shift != NULL the call
@@ -266,6 +273,28 @@ maglev_status maglev_consistency_loss(const void* m, const void* m_target, int64
                                       int dtype, float lambda, float inv_count, float* loss,
                                       void* dm, void* dm_target, int accumulate_dm,
                                       void* workspace, void* stream);
+
+/* a7 fused with the first pass of a6, for a layer whose own output feeds the
+ * consistency loss ([rainbus] 方法步骤详情: the loss on m; the backward of the
+ * banded attention needs Delta_i = sum_c out_ic dout_ic per query row and head).
+ * In one pass over out, m_target and dout it computes what
+ * maglev_consistency_loss(m = out, dm = dout, accumulate_dm = 1) computes, the
+ * same loss bit for bit and the same updated dout, and writes into the layer's
+ * backward workspace Delta from the updated, stored dout and (bf16) the zeroed
+ * fp32 dQ accumulator: what maglev_inject_swa_bwd's first pass writes. Call
+ * maglev_inject_swa_bwd next on the same out, dout and workspace with
+ * MAGLEV_BWD_PREPARED or'd into dR_mode.
+ *   desc: the layer's descriptor (B, T, H, hd, dtype).
+ *   out, m_target [B,T,H,hd] of dtype; dout [B,T,H,hd] (in/out).
+ *   lambda, inv_count, loss: as in maglev_consistency_loss (d = H*hd).
+ *   bwd_workspace: maglev_swa_bwd_workspace_bytes(desc) bytes;
+ *   loss_workspace: maglev_consistency_workspace_bytes(B*T, H*hd) bytes.
+ * Errors: as maglev_consistency_loss, and the descriptor checks of the layer
+ * calls. */
+maglev_status maglev_consistency_loss_prepare_bwd(const maglev_swa_desc* desc, const void* out,
+                                                  const void* m_target, float lambda, float inv_count,
+                                                  float* loss, void* dout, void* bwd_workspace,
+                                                  void* loss_workspace, void* stream);
 
 /* Scratch-free variant of maglev_consistency_loss, for callers that cannot
  * allocate device memory: e.g. a plugin or custom-op interface that hands over

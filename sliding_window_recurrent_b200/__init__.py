@@ -22,6 +22,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "maglev.h")
 MAGLEV_OK, MAGLEV_ERR_INVALID_ARG, MAGLEV_ERR_UNSUPPORTED, MAGLEV_ERR_CUDA, MAGLEV_ERR_TIMEOUT, MAGLEV_ERR_BOUNDS = range(6)
 MAGLEV_F32, MAGLEV_BF16 = 0, 1
 MAGLEV_DR_WRITE, MAGLEV_DR_FIRST, MAGLEV_DR_ADD, MAGLEV_DR_LAST = range(4)
+MAGLEV_BWD_PREPARED = 16
 
 
 class MaglevError(RuntimeError):
@@ -72,6 +73,7 @@ _SIGS = {
     "maglev_mem_project_bwd": ([ctypes.POINTER(SwaDesc)] + [_P] * 9, _I),
     "maglev_mem_project_bwd_layers": ([ctypes.POINTER(SwaDesc), _I] + [_P] * 9, _I),
     "maglev_consistency_loss": ([_P, _P, _I64, _I, _I, _F, _F, _P, _P, _P, _I, _P, _P], _I),
+    "maglev_consistency_loss_prepare_bwd": ([ctypes.POINTER(SwaDesc), _P, _P, _F, _F, _P, _P, _P, _P, _P], _I),
     "maglev_consistency_loss_noalloc": ([_P, _P, _I64, _I, _I, _F, _F, _P, _P, _P, _I, _P], _I),
     "maglev_memory_state": ([_I, _I, _I, _F, _I] + [_P] * 5, _I),
     "maglev_memory_state_bwd": ([_I, _I, _I, _I] + [_P] * 7, _I),
@@ -222,6 +224,13 @@ def maglev_consistency_loss(m, m_target, rows, d, dtype, lam, inv_count, loss, d
                                         float(lam), float(inv_count), _ptr(loss), _ptr(dm),
                                         _ptr(dm_target), int(accumulate_dm), _ptr(workspace),
                                         _stream(stream)))
+
+
+def maglev_consistency_loss_prepare_bwd(desc, out, m_target, lam, inv_count, loss, dout, bwd_workspace,
+                                        loss_workspace, stream=None):
+    _check(_lib.maglev_consistency_loss_prepare_bwd(ctypes.byref(desc), _ptr(out), _ptr(m_target), float(lam),
+                                                    float(inv_count), _ptr(loss), _ptr(dout),
+                                                    _ptr(bwd_workspace), _ptr(loss_workspace), _stream(stream)))
 
 
 def maglev_consistency_loss_noalloc(m, m_target, rows, d, dtype, lam, inv_count, loss, dm, dm_target,

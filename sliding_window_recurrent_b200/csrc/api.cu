@@ -470,6 +470,10 @@ maglev_status maglev_inject_swa_bwd(const maglev_swa_desc* d, const void* k, con
   NEED_PTR(dk);
   NEED_PTR(dv);
   NEED_PTR(workspace);
+  // Delta and the zeroed dQ accumulator already in the workspace
+  // (maglev_consistency_loss_prepare_bwd on this out and dout)
+  const bool prepared = (dR_mode & MAGLEV_BWD_PREPARED) != 0;
+  dR_mode &= ~MAGLEV_BWD_PREPARED;
   if (dR_mode < MAGLEV_DR_WRITE || dR_mode > MAGLEV_DR_LAST)
     return fail(MAGLEV_ERR_INVALID_ARG, "dR_mode %d is not a maglev_dr_mode", dR_mode);
   if (!d->inject) dR_mode = MAGLEV_DR_WRITE;
@@ -513,7 +517,7 @@ maglev_status maglev_inject_swa_bwd(const maglev_swa_desc* d, const void* k, con
   void* dvb = at<char>(workspace, Wk.dvb);
   float* gpart = at<float>(workspace, Wk.gpart);
   float* dq_acc = d->dtype == MAGLEV_BF16 ? at<float>(workspace, Wk.dq_acc) : nullptr;
-  MAGLEV_LAUNCH(1, s, launch_attn_delta(sh, out, dout, delta, dq_acc, s), "attn_delta");
+  if (!prepared) MAGLEV_LAUNCH(1, s, launch_attn_delta(sh, out, dout, delta, dq_acc, s), "attn_delta");
   if (d->dtype == MAGLEV_BF16) {
     int* err = nullptr;
     st = status_word(&err, s);
@@ -658,6 +662,36 @@ maglev_status maglev_consistency_loss(const void* m, const void* m_target, int64
                                                loss, dm, dm_target, accumulate_dm ? 1 : 0,
                                                static_cast<float*>(workspace), s),
                 "consistency_loss");
+  return MAGLEV_OK;
+}
+
+maglev_status maglev_consistency_loss_prepare_bwd(const maglev_swa_desc* d, const void* out,
+                                                  const void* m_target, float lambda, float inv_count,
+                                                  float* loss, void* dout, void* bwd_workspace,
+                                                  void* loss_workspace, void* stream) {
+  maglev_status st = check_swa(d);
+  if (st != MAGLEV_OK) return st;
+  if (!std::isfinite(lambda) || !std::isfinite(inv_count) || inv_count < 0)
+    return fail(MAGLEV_ERR_INVALID_ARG, "lambda and inv_count must be finite, inv_count >= 0");
+  NEED_PTR(loss);
+  if (d->B == 0 || d->T == 0) return MAGLEV_OK;
+  NEED_PTR(out);
+  NEED_PTR(m_target);
+  NEED_PTR(dout);
+  NEED_PTR(bwd_workspace);
+  NEED_PTR(loss_workspace);
+  const int64_t rows = (int64_t)d->B * d->T;
+  const int D = d->H * d->hd;
+  const double ic = inv_count == 0.0f ? 1.0 / (double)rows : (double)inv_count;
+  const double sl = (double)lambda * ic / std::sqrt((double)D);
+  const BwdLayout Wk = bwd_layout(d);
+  float* delta = at<float>(bwd_workspace, Wk.delta);
+  float* dq_acc = d->dtype == MAGLEV_BF16 ? at<float>(bwd_workspace, Wk.dq_acc) : nullptr;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MAGLEV_LAUNCH(2, s, launch_consistency_loss_prep(out, m_target, rows, d->H, d->hd, d->T, d->dtype, (float)sl,
+                                                   (float)(2.0 * sl), loss, dout, delta, dq_acc,
+                                                   static_cast<float*>(loss_workspace), s),
+                "consistency_loss_prep");
   return MAGLEV_OK;
 }
 

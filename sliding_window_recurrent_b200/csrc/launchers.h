@@ -74,6 +74,11 @@ cudaError_t launch_memstate_bwd(const void* o, const float* rstd, const void* dm
 cudaError_t launch_consistency_loss(const void* m, const void* mt, int64_t rows, int d, int dtype,
                                     float scale_loss, float scale_grad, float* loss, void* dm,
                                     void* dmt, int accumulate, float* partials, cudaStream_t st);
+// launch_consistency_loss of a layer's output (accumulating into dout) that also
+// writes the attention backward's Delta [B,H,T] and zeroes dq_acc (nullable).
+cudaError_t launch_consistency_loss_prep(const void* out, const void* mt, int64_t rows, int H, int hd, int seq,
+                                         int dtype, float scale_loss, float scale_grad, float* loss, void* dout,
+                                         float* delta, float* dq_acc, float* partials, cudaStream_t st);
 
 struct DecShape {
   int B, H, hd, W, inject, dtype;

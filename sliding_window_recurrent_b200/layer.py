@@ -7,8 +7,8 @@ from __future__ import annotations
 
 import torch
 
-from . import (DecodeDesc, MAGLEV_BF16, MAGLEV_DR_WRITE, MAGLEV_F32, SwaDesc, maglev_consistency_loss,
-               maglev_consistency_workspace_bytes, maglev_decode_mem_project, maglev_decode_step,
+from . import (DecodeDesc, MAGLEV_BF16, MAGLEV_BWD_PREPARED, MAGLEV_DR_WRITE, MAGLEV_F32, SwaDesc,
+               maglev_consistency_loss, maglev_consistency_loss_prepare_bwd, maglev_consistency_workspace_bytes, maglev_decode_mem_project, maglev_decode_step,
                maglev_decode_workspace_bytes,
                maglev_inject_swa_bwd, maglev_inject_swa_fwd, maglev_swa_bwd_workspace_bytes,
                maglev_swa_saved_bytes)
@@ -63,13 +63,22 @@ class InjectedSWALayer:
                                 self.loss, dm, None, accumulate_dm, self.loss_ws, stream)
         return self.loss
 
+    def consistency_prepare_bwd(self, target, lam, dout, inv_count=0.0, stream=None):
+        """The consistency loss of this layer's own output against target,
+        added into dout, together with the backward's first pass (the next
+        backward call is given prepared=True)."""
+        maglev_consistency_loss_prepare_bwd(self.desc, self.out, target, lam, inv_count, self.loss, dout,
+                                            self.workspace, self.loss_ws, stream)
+        return self.loss
+
     def backward(self, k, v, dout, gates=None, m_shift=None, w_mk=None, w_mv=None,
-                 dR_mode=MAGLEV_DR_WRITE, dR_acc=(None, None), stream=None):
+                 dR_mode=MAGLEV_DR_WRITE, dR_acc=(None, None), stream=None, prepared=False):
         """dR_mode / dR_acc: how dL/dR is stored (maglev_dr_mode) and the fp32
-        running sums it reads or writes when several layers share W^rec."""
+        running sums it reads or writes when several layers share W^rec;
+        prepared: consistency_prepare_bwd ran on this out and dout."""
         maglev_inject_swa_bwd(self.desc, k, v, self.R_k, self.R_v, gates, self.out, self.lse,
                               self.saved, dout, self.dq, self.dk, self.dv, self.dR_k, self.dR_v,
-                              dR_acc[0], dR_acc[1], dR_mode, self.dgate,
+                              dR_acc[0], dR_acc[1], dR_mode | (MAGLEV_BWD_PREPARED if prepared else 0), self.dgate,
                               m_shift if self.inject else None, w_mk, w_mv,
                               self.dm_shift, self.dw_mk, self.dw_mv, self.workspace, stream)
 

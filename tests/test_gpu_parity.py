@@ -36,7 +36,7 @@ def wl_of(name, **over):
     return wl
 
 
-def run_gpu(wl, x, inject=True, lam=None, bwd=True, pos0=0):
+def run_gpu(wl, x, inject=True, lam=None, bwd=True, pos0=0, fused=False):
     B, T, H, hd, d, W = wl["B"], wl["T"], wl["H"], wl["hd"], wl["d"], wl["W"]
     D = H * hd
     L = InjectedSWALayer(B, T, H, hd, d, W, dtype=wl["dtype"], inject=inject, pos0=pos0,
@@ -52,11 +52,16 @@ def run_gpu(wl, x, inject=True, lam=None, bwd=True, pos0=0):
         res["R_k"], res["R_v"] = host(L.R_k), host(L.R_v)
     if bwd:
         dout = dev(x["dout"]).clone()
-        if lam is not None:
+        if lam is not None and fused:  # the loss together with the backward's first pass
+            L.consistency_prepare_bwd(dev(x["target"]), lam, dout)
+            res["loss"] = float(L.loss.item())
+        elif lam is not None:
             L.consistency(L.out.view(B * T, D), dev(x["target"]).view(B * T, D), lam,
                           dm=dout.view(B * T, D), accumulate_dm=True)
             res["loss"] = float(L.loss.item())
-        L.backward(k, v, dout, gates, m, wk, wv)
+        L.backward(k, v, dout, gates, m, wk, wv, prepared=fused and lam is not None)
+        res["dout_total"] = host(dout)
+        res["loss_bits"] = L.loss.clone()
         for n in ("dq", "dk", "dv"):
             res[n] = host(getattr(L, n))
         if inject:
@@ -158,6 +163,29 @@ def test_layer_bf16_full_size():
     errs = compare(g, r, "bf16", FWD + BWD, report_elementwise=True)
     print("full-size layer errors:", {k: f"{v:.2e}" for k, v in errs.items()})
     assert abs(g["loss"] - r["loss"]) <= 2e-2 * abs(r["loss"])
+
+
+@pytest.mark.parametrize("name,over", [("tiny_f32", {}), ("layer_bf16", dict(B=2, T=300, H=3, hd=128, d=160, W=100)),
+                                       ("layer_bf16", dict(B=2, T=333, H=3, hd=64, d=160, W=47)), ("layer_bf16", {})])
+def test_loss_prepare_bwd_fused(name, over):
+    """maglev_consistency_loss_prepare_bwd, then the backward told it ran:
+    every output within tolerance of the oracle, and against the separate loss
+    and backward calls the same loss bit for bit and the same updated dO."""
+    wl = wl_of(name, **over)
+    if name == "layer_bf16" and over:
+        wl["target"] = "independent"
+    x = synth.layer_inputs(wl, 4321)
+    lam = 0.1 if wl["dtype"] == "bf16" else 1.0
+    g = run_gpu(wl, x, lam=lam, fused=True)
+    r = run_oracle(wl, x, lam=lam)
+    compare(g, r, wl["dtype"], FWD + BWD)
+    tol = 2e-2 if wl["dtype"] == "bf16" else 1e-4
+    assert abs(g["loss"] - r["loss"]) <= tol * abs(r["loss"])
+    p = run_gpu(wl, x, lam=lam)
+    assert torch.equal(g["loss_bits"], p["loss_bits"])
+    assert np.array_equal(g["dout_total"], p["dout_total"])
+    for n in BWD:  # only the order of Delta's fp32 sums differs between the two paths
+        assert normwise(g[n], p[n]) <= tol, n
 
 
 # --------------------------------------------------------------------------- bit-exact probes
