@@ -87,6 +87,32 @@ def test_empty_problems_enqueue_nothing():
                                FAKE, stream=0)
 
 
+def test_loss_prepare_bwd_validation():
+    """The fused loss / backward-preparation call checks its descriptor and
+    pointers before any launch; an empty problem enqueues nothing; the flag it
+    pairs with is accepted by the backward's dR_mode check (mode 7 | flag is not)."""
+    mg.maglev_consistency_loss_prepare_bwd(desc(B=0), FAKE, FAKE, 0.1, 0.0, FAKE, FAKE, FAKE, FAKE, stream=0)
+    with pytest.raises(mg.MaglevError) as e:
+        mg.maglev_consistency_loss_prepare_bwd(desc(), FAKE, FAKE, 0.1, 0.0, None, FAKE, FAKE, FAKE, stream=0)
+    assert e.value.status == mg.MAGLEV_ERR_INVALID_ARG and "loss" in str(e.value)
+    with pytest.raises(mg.MaglevError) as e:
+        mg.maglev_consistency_loss_prepare_bwd(desc(), FAKE, FAKE, 0.1, 0.0, FAKE, FAKE, None, FAKE, stream=0)
+    assert e.value.status == mg.MAGLEV_ERR_INVALID_ARG and "bwd_workspace" in str(e.value)
+    with pytest.raises(mg.MaglevError) as e:
+        mg.maglev_consistency_loss_prepare_bwd(desc(), FAKE, FAKE, float("inf"), 0.0, FAKE, FAKE, FAKE, FAKE,
+                                               stream=0)
+    assert e.value.status == mg.MAGLEV_ERR_INVALID_ARG
+    with pytest.raises(mg.MaglevError) as e:
+        mg.maglev_consistency_loss_prepare_bwd(desc(hd=96), FAKE, FAKE, 0.1, 0.0, FAKE, FAKE, FAKE, FAKE,
+                                               stream=0)
+    assert e.value.status == mg.MAGLEV_ERR_UNSUPPORTED
+    with pytest.raises(mg.MaglevError) as e:
+        mg.maglev_inject_swa_bwd(desc(), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                 FAKE, FAKE, FAKE, None, None, FAKE, FAKE, 7 | mg.MAGLEV_BWD_PREPARED, FAKE,
+                                 None, FAKE, FAKE, None, None, None, FAKE, stream=0)
+    assert e.value.status == mg.MAGLEV_ERR_INVALID_ARG and "dR_mode 7" in str(e.value)
+
+
 def test_bwd_and_loss_and_decode_validation():
     with pytest.raises(mg.MaglevError):  # dR_k is needed in mode WRITE
         mg.maglev_inject_swa_bwd(desc(), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
