@@ -751,8 +751,12 @@ maglev_status maglev_lm_head_ce(int64_t N, int d, int V, int dtype, float softca
   MAGLEV_LAUNCH(dz ? 3 : 2, s, launch_lm_ce_finish(N, V, lm_ce_tiles(V), ic, softcap, part, tgt, targets, c, lse,
                                                     ce, loss, dz, s),
                 "lm_ce_finish");
-  if (dm) MAGLEV_LAUNCH(1, s, launch_lm_dm_tc(N, d, V, dz, U, dm, lim, err, s), "lm_dm_tc");
-  if (dU) MAGLEV_LAUNCH(1, s, launch_lm_dU_tc(N, d, V, dz, m, dU, lim, err, s), "lm_dU_tc");
+  if (dm && dU && lm_bwd_grouped_available(N, d, V)) {  // both in one launch on SM pairs
+    MAGLEV_LAUNCH(1, s, launch_lm_bwd_grouped_pair(N, d, V, dz, U, m, dm, dU, lim, err, s), "lm_bwd_tc");
+  } else {
+    if (dm) MAGLEV_LAUNCH(1, s, launch_lm_dm_tc(N, d, V, dz, U, dm, lim, err, s), "lm_dm_tc");
+    if (dU) MAGLEV_LAUNCH(1, s, launch_lm_dU_tc(N, d, V, dz, m, dU, lim, err, s), "lm_dU_tc");
+  }
   return MAGLEV_OK;
 }
 

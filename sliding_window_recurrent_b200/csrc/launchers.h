@@ -116,6 +116,11 @@ cudaError_t launch_proj_bwd_dw_tc(int64_t M, int D, int d, const void* dRk, cons
 // dW and dm of the shared projection in one launch on SM pairs (tc_gemm_pair.cu),
 // when proj_bwd_grouped_available says it can run.
 bool proj_bwd_grouped_available(int64_t M, int D, int d);
+// The LM head's dm and dU in one launch on SM pairs (tc_gemm_pair.cu), when
+// lm_bwd_grouped_available says it can run.
+bool lm_bwd_grouped_available(int64_t N, int d, int V);
+cudaError_t launch_lm_bwd_grouped_pair(int64_t N, int d, int V, const void* dz, const void* U, const void* m,
+                                       void* dm, void* dU, int64_t spin_limit, int* err, cudaStream_t s);
 cudaError_t launch_proj_bwd_grouped_pair(int64_t M, int D, int d, const void* dRk, const void* dRv, const void* w_mk,
                                          const void* w_mv, const void* m_shift, void* dm, void* dwk, void* dwv,
                                          int64_t spin_limit, int* err, cudaStream_t s);

@@ -23,7 +23,8 @@
 // of 20 K blocks, 2.16 waves; dW 50 tiles of 64 K blocks). The host then
 // deals the tiles of both longest first, each to the pair with the least work
 // so far, and passes every pair its list: 100 K-block times for the two
-// instead of 60 + 64 back to back.
+// instead of 60 + 64 back to back. The LM head's backward GEMMs go the same
+// way: dm (160 tiles of 512 K blocks) with dU (1280 tiles of 64).
 //
 // Roles per CTA (6 warps): warp 0 TMA producer, warp 1 MMA issuer (leader
 // only), warps 2-5 epilogue (TMEM -> bf16 -> 128-byte row pieces). Loads in
@@ -57,7 +58,7 @@ constexpr int PM = 256;       // rows of a pair tile (128 per CTA)
 constexpr int PN = 256;       // columns of a pair tile (B: 128 per CTA)
 constexpr int PAIR_THREADS = 192;
 constexpr int PAIR_MAX_PAIRS = 80;   // schedule table (a B200 holds 74 pairs)
-constexpr int PAIR_MAX_ITEMS = 512;  // tiles of a scheduled launch
+constexpr int PAIR_MAX_ITEMS = 2048;  // tiles of a scheduled launch (the table is a kernel parameter)
 
 // One GEMM of a launch: out [M, N] bf16 = A [M, K] x B [K, N], fp32 in TMEM.
 // A is K-major (rows of K contiguous) or MN-major (a_mn: columns of M
@@ -616,6 +617,40 @@ cudaError_t launch_proj_bwd_dw_pair(int64_t M, int D, int d, const void* dRk, co
   if ((e = dw_problem(M, D, d, dRk, dRv, m_shift, dwk, dwv, mp, q)) != cudaSuccess) return e;
   PairParams p = pair_params(q, spin_limit, err);
   return run_pair<128>(mp, mp, p, false, s);
+}
+
+// dm [N, d] = dz [N, V] U [V, d] (K = V) and dU [V, d] = dz^T [V, N] m [N, d]
+// (K = N) in one launch, their tiles dealt longest first over the SM pairs.
+// cudaErrorNotSupported when clusters cannot be launched or the two have more
+// tiles than the schedule table holds; the caller then launches them one by one.
+bool lm_bwd_grouped_available(int64_t N, int d, int V) {
+  if (d % 8 != 0 || V % 8 != 0 || max_pairs<128>() < 1) return false;
+  const int64_t tiles = ((N + PM - 1) / PM + ((int64_t)V + PM - 1) / PM) * (((int64_t)d + PN - 1) / PN);
+  return tiles <= PAIR_MAX_ITEMS;
+}
+
+cudaError_t launch_lm_bwd_grouped_pair(int64_t N, int d, int V, const void* dz, const void* U, const void* m,
+                                       void* dm, void* dU, int64_t spin_limit, int* err, cudaStream_t s) {
+  PairMaps mm, mu;
+  cudaError_t e;
+  if ((e = make_tmap_bf16_2d(&mm.a0, dz, V, N, (uint64_t)V * 2, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&mm.b0, U, d, V, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
+  mm.a1 = mm.a0;
+  mm.b1 = mm.b0;
+  mu.a0 = mm.a0;  // dz read MN-major: the same {64 V, 128 N} boxes
+  if ((e = make_tmap_bf16_2d(&mu.b0, m, d, N, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
+  mu.a1 = mu.a0;
+  mu.b1 = mu.b0;
+  PairProblem qm = pair_problem((int)N, d, V, false, true, d);
+  qm.out0 = dm;
+  qm.out1 = dm;
+  PairProblem qu = pair_problem(V, d, (int)N, true, true, d);
+  qu.out0 = dU;
+  qu.out1 = dU;
+  PairParams p = pair_params(qm, spin_limit, err);
+  p.pr[1] = qu;
+  p.n_items = p.tiles0 + qu.tiles_m * qu.tiles_n;
+  return run_pair<128>(mm, mu, p, true, s);
 }
 
 // Whether launch_proj_bwd_grouped_pair can run dW and dm of these sizes.
