@@ -119,6 +119,11 @@ bool proj_bwd_grouped_available(int64_t M, int D, int d);
 // The LM head's dm and dU in one launch on SM pairs (tc_gemm_pair.cu), when
 // lm_bwd_grouped_available says it can run.
 bool lm_bwd_grouped_available(int64_t N, int d, int V);
+// The LM head's logits GEMM with its softcapped CE epilogue on SM pairs;
+// cudaErrorNotSupported when clusters cannot be launched (or V % 4 != 0).
+cudaError_t launch_lm_logits_ce_pair(int64_t N, int d, int V, float softcap, const void* m, const void* U,
+                                     const int64_t* targets, float* c, float2* part, float* tgt,
+                                     int64_t spin_limit, int* err, cudaStream_t s);
 cudaError_t launch_lm_bwd_grouped_pair(int64_t N, int d, int V, const void* dz, const void* U, const void* m,
                                        void* dm, void* dU, int64_t spin_limit, int* err, cudaStream_t s);
 cudaError_t launch_proj_bwd_grouped_pair(int64_t M, int D, int d, const void* dRk, const void* dRv, const void* w_mk,

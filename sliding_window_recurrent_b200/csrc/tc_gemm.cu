@@ -39,9 +39,9 @@ struct TcGemmParams {
   int out_switch_m, out_switch_n;
   int k_layers;  // > 0: A is [k_layers][M][a_switch_k], B [k_layers][a_switch_k][N] (3-D maps), K = 2 L a_switch_k
   // softcapped cross-entropy epilogue (EPI_CE): out0 receives the capped
-  // logits c = softcap * tanh(z / softcap) in fp32; per row and N tile the
-  // (max, sum of exp(c - max)) pair goes to ce_part[row * tiles_n + tile], and
-  // the capped logit of the row's target to ce_tgt[row]
+  // logits c = softcap * tanh(z / softcap) in fp32; per row and 128 columns the
+  // (max, sum of exp(c - max)) pair goes to ce_part[row * ceil(N / 128) + i],
+  // and the capped logit of the row's target to ce_tgt[row]
   const int64_t* targets;
   float softcap;
   float2* ce_part;
@@ -72,9 +72,11 @@ constexpr int EPI_BF16 = 0, EPI_CE = 1;
 
 // softcap * tanh(z / softcap), with tanh(x) = 1 - 2 / (1 + e^{2x}) (exact at
 // +-inf: e^{2x} = inf gives 1, 0 gives -1; absolute error ~1e-7 near 0).
+// cap * tanh(z / cap) = cap * (1 - 2 / (1 + e^(2z/cap))), with the hardware 2^x
+// and the fast division intrinsic (both ends exact: 2 / inf = 0, 2 / 1 = 2)
 __device__ __forceinline__ float softcap_of(float z, float cap, float two_log2e_over_cap) {
   const float e = ex2_fast(z * two_log2e_over_cap);
-  return cap * (1.0f - 2.0f * __frcp_rn(1.0f + e));
+  return cap * (1.0f - __fdividef(2.0f, 1.0f + e));
 }
 
 template <int BN, bool A_MN, bool B_MN, int EPI = EPI_BF16>
@@ -273,9 +275,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const int gm = m0 + row;
       const int64_t y = gm < p.M ? p.targets[gm] : -1;
+      const int ce_tiles = (p.N + 127) / 128;  // partials per row
       float mx = -INFINITY, sm = 0.f;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int c0 = 0; c0 < BN && n0 + c0 < p.N; c0 += 32) {
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::ACC_STRIDE + c0), r);
         tmem_wait_ld();
@@ -289,12 +292,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           cmx = fmaxf(cmx, cv);
           r[e] = __float_as_uint(cv);
         }
-        const float nmx = fmaxf(mx, cmx);  // finite: column n0 < N is in the first chunk
+        const float nmx = fmaxf(mx, cmx);  // finite: this chunk starts inside the row
         float se = 0.f;
 #pragma unroll
         for (int e = 0; e < 32; ++e) se += ex2_fast((__uint_as_float(r[e]) - nmx) * LOG2E_F);
         sm = sm * ex2_fast((mx - nmx) * LOG2E_F) + se;
         mx = nmx;
+        if (((c0 + 32) & 127) == 0 || n0 + c0 + 32 >= p.N) {  // the end of 128 columns (or of the row)
+          if (gm < p.M) p.ce_part[(int64_t)gm * ce_tiles + (n0 + c0) / 128] = make_float2(mx, sm);
+          mx = -INFINITY;
+          sm = 0.f;
+        }
 #pragma unroll
         for (int j = 0; j < 8; ++j)
           *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
@@ -313,7 +321,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
-      if (gm < p.M) p.ce_part[(int64_t)gm * p.tiles_n + tn] = make_float2(mx, sm);
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
@@ -677,6 +684,10 @@ cudaError_t launch_proj_bwd_dw_tc(int64_t M, int D, int d, const void* dRk, cons
 cudaError_t launch_lm_logits_ce_tc(int64_t N, int d, int V, float softcap, const void* m, const void* U,
                                    const int64_t* targets, float* c, float2* part, float* tgt,
                                    int64_t spin_limit, int* err, cudaStream_t s) {
+  {  // SM pairs first (tc_gemm_pair.cu); one SM per tile where clusters cannot run
+    const cudaError_t pe = launch_lm_logits_ce_pair(N, d, V, softcap, m, U, targets, c, part, tgt, spin_limit, err, s);
+    if (pe != cudaErrorNotSupported) return pe;
+  }
   constexpr int BN = 256;
   CUtensorMap a, b;
   cudaError_t e;
@@ -700,7 +711,7 @@ cudaError_t launch_lm_logits_ce_tc(int64_t N, int d, int V, float softcap, const
   return run_gemm<BN, false, false, EPI_CE>(a, a, b, b, p, s);
 }
 
-int lm_ce_tiles(int V) { return (V + 255) / 256; }
+int lm_ce_tiles(int V) { return (V + 127) / 128; }  // (max, sum) partials per row: one per 128 columns
 
 // dm [N, d] = dz [N, V] U [V, d] (K = V).
 cudaError_t launch_lm_dm_tc(int64_t N, int d, int V, const void* dz, const void* U, void* dm, int64_t spin_limit,

@@ -56,7 +56,15 @@ using namespace tc;
 
 constexpr int PM = 256;       // rows of a pair tile (128 per CTA)
 constexpr int PN = 256;       // columns of a pair tile (B: 128 per CTA)
-constexpr int PAIR_THREADS = 192;
+constexpr int EPI_BF16 = 0, EPI_CE = 1;
+// Epilogue warps: 4 (one per TMEM lane quarter) for the bf16 store; 8 for the
+// cross-entropy epilogue (two per lane quarter, each with 128 of the tile's 256
+// columns: its per-element softcap and exponentials would otherwise pace the
+// launch).
+template <int EPI>
+constexpr int pair_epi_warps() { return EPI == EPI_CE ? 8 : 4; }
+template <int EPI>
+constexpr int pair_threads() { return 64 + 32 * pair_epi_warps<EPI>(); }
 constexpr int PAIR_MAX_PAIRS = 80;   // schedule table (a B200 holds 74 pairs)
 constexpr int PAIR_MAX_ITEMS = 2048;  // tiles of a scheduled launch (the table is a kernel parameter)
 
@@ -90,11 +98,19 @@ struct PairParams {
   int sched;    // 1: pair i runs order[first[i] .. first[i + 1]); 0: items i, i + pairs, ...
   int64_t spin_limit;
   int* err;
+  // softcapped cross-entropy epilogue (one problem): out0 receives the capped
+  // logits c = softcap * tanh(z / softcap) in fp32; per row and 128 columns the
+  // (max, sum of exp(c - max)) pair goes to ce_part[row * ceil(N / 128) + i],
+  // and the capped logit of the row's target to ce_tgt[row]
+  const int64_t* ce_targets;
+  float softcap;
+  float2* ce_part;
+  float* ce_tgt;
   uint16_t first[PAIR_MAX_PAIRS + 1];
   uint16_t order[PAIR_MAX_ITEMS];
 };
 
-template <int PK>
+template <int PK, int EPI = EPI_BF16>
 struct PairCfg {
   // K block: 64 when both operands are K-major (one {64 K, 128 rows} box each,
   // six 32 KiB stages); 128 when one is MN-major, whose 16 KiB box is
@@ -110,8 +126,8 @@ struct PairCfg {
   static constexpr int TMEM_COLS = 512;                 // two 128 x 256 fp32 accumulators
   static constexpr int ACC_STRIDE = 256;
   static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
-  static constexpr int OFF_EPI = OFF_BAR + 256;         // 4 warps x [32 rows x 128 B] output staging
-  static constexpr size_t SMEM = 1024 + (size_t)OFF_EPI + 4 * 4096;
+  static constexpr int OFF_EPI = OFF_BAR + 256;         // per epilogue warp [32 rows x 128 B] output staging
+  static constexpr size_t SMEM = 1024 + (size_t)OFF_EPI + pair_epi_warps<EPI>() * 4096;
 };
 
 // The i-th item (tile) of this pair, or -1 past its last.
@@ -138,12 +154,20 @@ __device__ __forceinline__ PairTile pair_tile(const PairParams& p, int item) {
   return t;
 }
 
-template <int PK>
-__global__ void __launch_bounds__(PAIR_THREADS, 1)
+// cap * tanh(z / cap) = cap * (1 - 2 / (1 + e^(2z/cap))), with the hardware 2^x
+// and the fast division intrinsic (both ends exact: 2 / inf = 0, 2 / 1 = 2)
+__device__ __forceinline__ float pair_softcap(float z, float cap, float two_log2e_over_cap) {
+  const float e = ex2_fast(z * two_log2e_over_cap);
+  return cap * (1.0f - __fdividef(2.0f, 1.0f + e));
+}
+
+template <int PK, int EPI>
+__global__ void __launch_bounds__(pair_threads<EPI>(), 1)
     tc_gemm_pair_kernel(const __grid_constant__ PairMaps mp0, const __grid_constant__ PairMaps mp1,
                         const __grid_constant__ PairParams p) {
-  using C = PairCfg<PK>;
+  using C = PairCfg<PK, EPI>;
   constexpr int STAGES = C::STAGES;
+  constexpr int EPI_WARPS = pair_epi_warps<EPI>();
   extern __shared__ uint8_t smem_raw[];
   // the same offset in both CTAs: the pair MMA reads both CTAs' operands at one address
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -169,7 +193,7 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 8);  // one arrival per epilogue warp of both CTAs
+      mbar_init(&tempty[a], 2 * EPI_WARPS);  // one arrival per epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -333,6 +357,81 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
       }
       __syncwarp();
     }
+  } else if constexpr (EPI == EPI_CE) {
+    // -------------------------------------------------------------- CE epilogue (both CTAs)
+    // Thread = one of this CTA's 128 rows of the tile; warp w owns columns
+    // [128 h, 128 h + 128), h = (w - 2) / 4. 32 columns at a time: TMEM ->
+    // capped logits (running max / sum of exponentials of the row over the
+    // warp's 128 columns, target logit) -> the warp's 4 KiB of fp32 staging ->
+    // 128-byte row pieces; one (max, sum) partial per row and 128 columns.
+    constexpr float LOG2E_F = 1.4426950408889634f;
+    const float k2 = 2.0f * LOG2E_F / p.softcap;
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;
+    const int row = q * 32 + lane;
+    uint8_t* stg = smem + C::OFF_EPI + (warp - 2) * 4096;
+    const PairProblem& pr = p.pr[0];
+    const int ce_tiles = (pr.N + 127) / 128;  // partials per row
+    float* outc = static_cast<float*>(pr.out0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int i = 0;; ++i) {
+      const int item = pair_item(p, pair, npairs, i);
+      if (item < 0) break;
+      const PairTile tl = pair_tile(p, item);
+      const int m0 = tl.tm * PM + 128 * (int)rank, n0 = tl.tn * PN + 128 * half;
+      if (!warp_wait(&tfull[acc], acc_phase, ab)) break;
+      tc_fence_after();
+      const int gm = m0 + row;
+      const int64_t y = gm < pr.M ? p.ce_targets[gm] : -1;
+      float mx = -INFINITY, sm = 0.f;
+      const bool any = n0 < pr.N;  // the warp's columns start inside the row
+#pragma unroll 1
+      for (int c0 = 0; c0 < (any ? 128 : 0); c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::ACC_STRIDE + 128 * half + c0), r);
+        tmem_wait_ld();
+        float cmx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int col = n0 + c0 + e;
+          const float c = pair_softcap(__uint_as_float(r[e]), p.softcap, k2);
+          if (col == y) p.ce_tgt[gm] = c;
+          const float cv = col < pr.N ? c : -INFINITY;
+          cmx = fmaxf(cmx, cv);
+          r[e] = __float_as_uint(cv);
+        }
+        const float nmx = fmaxf(mx, cmx);  // finite: column n0 < N is in the first chunk
+        float se = 0.f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) se += ex2_fast((__uint_as_float(r[e]) - nmx) * LOG2E_F);
+        sm = sm * ex2_fast((mx - nmx) * LOG2E_F) + se;
+        mx = nmx;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+              make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int rr = 4 * k + (lane >> 3), j = lane & 7;  // row of the warp's 32, 16-byte chunk
+          const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 128 + ((j ^ (rr & 7)) << 4));
+          const int col = n0 + c0 + 4 * j;
+          const int grow = m0 + q * 32 + rr;
+          if (grow < pr.M && col + 4 <= pr.N && MAGLEV_CHECK(p.err, grow >= 0 && col >= 0 && col + 4 <= pr.ldo))
+            *reinterpret_cast<uint4*>(outc + (int64_t)grow * pr.ldo + col) = v;
+        }
+        __syncwarp();
+      }
+      if (gm < pr.M && any) p.ce_part[(int64_t)gm * ce_tiles + 2 * tl.tn + half] = make_float2(mx, sm);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_cluster(smem_u32(&tempty[acc]), 0));  // the leader may reuse it
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
   } else {
     // -------------------------------------------------------------- epilogue (both CTAs)
     // This CTA's 128 rows of the tile, 64 columns at a time: TMEM -> bf16 ->
@@ -417,17 +516,17 @@ namespace {
 
 // Largest number of two-CTA clusters of this kernel that can be resident at
 // once (0 when clusters cannot be launched), cached per instantiation.
-template <int PK>
+template <int PK, int EPI = EPI_BF16>
 int max_pairs() {
   static int cached = -1;
   if (cached >= 0) return cached;
-  using C = PairCfg<PK>;
-  auto kern = tc_gemm_pair_kernel<PK>;
+  using C = PairCfg<PK, EPI>;
+  auto kern = tc_gemm_pair_kernel<PK, EPI>;
   int n = 0;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM) == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * 74, 1, 1);
-    cfg.blockDim = dim3(PAIR_THREADS, 1, 1);
+    cfg.blockDim = dim3(pair_threads<EPI>(), 1, 1);
     cfg.dynamicSmemBytes = C::SMEM;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -470,10 +569,10 @@ void lpt_schedule(PairParams& p, int pairs) {
   p.sched = 1;
 }
 
-template <int PK>
+template <int PK, int EPI = EPI_BF16>
 cudaError_t run_pair(const PairMaps& m0, const PairMaps& m1, PairParams& p, bool schedule, cudaStream_t s) {
-  using C = PairCfg<PK>;
-  const int cap = max_pairs<PK>();
+  using C = PairCfg<PK, EPI>;
+  const int cap = max_pairs<PK, EPI>();
   if (cap < 1) return cudaErrorNotSupported;
   const int pairs = p.n_items < cap ? p.n_items : cap;
   if (schedule) {
@@ -482,7 +581,7 @@ cudaError_t run_pair(const PairMaps& m0, const PairMaps& m1, PairParams& p, bool
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(PAIR_THREADS, 1, 1);
+  cfg.blockDim = dim3(pair_threads<EPI>(), 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -492,7 +591,7 @@ cudaError_t run_pair(const PairMaps& m0, const PairMaps& m1, PairParams& p, bool
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<PK>, m0, m1, p);
+  return cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<PK, EPI>, m0, m1, p);
 }
 
 PairProblem pair_problem(int M, int N, int K, bool a_mn, bool b_mn, int64_t ldo) {
@@ -651,6 +750,30 @@ cudaError_t launch_lm_bwd_grouped_pair(int64_t N, int d, int V, const void* dz, 
   p.pr[1] = qu;
   p.n_items = p.tiles0 + qu.tiles_m * qu.tiles_n;
   return run_pair<128>(mm, mu, p, true, s);
+}
+
+// The LM head's logits z = m [N, d] U^T (U [V, d]) with the softcapped
+// cross-entropy epilogue (see PairParams): capped logits c [N, V] fp32,
+// part [N, ceil(V / 128)] and tgt [N].
+cudaError_t launch_lm_logits_ce_pair(int64_t N, int d, int V, float softcap, const void* m, const void* U,
+                                     const int64_t* targets, float* c, float2* part, float* tgt,
+                                     int64_t spin_limit, int* err, cudaStream_t s) {
+  if (V % 4 != 0) return cudaErrorNotSupported;
+  PairMaps mp;
+  cudaError_t e;
+  if ((e = make_tmap_bf16_2d(&mp.a0, m, d, N, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2d(&mp.b0, U, d, V, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
+  mp.a1 = mp.a0;
+  mp.b1 = mp.b0;
+  PairProblem q = pair_problem((int)N, V, d, false, false, V);
+  q.out0 = c;
+  q.out1 = c;
+  PairParams p = pair_params(q, spin_limit, err);
+  p.ce_targets = targets;
+  p.softcap = softcap;
+  p.ce_part = part;
+  p.ce_tgt = tgt;
+  return run_pair<64, EPI_CE>(mp, mp, p, false, s);
 }
 
 // Whether launch_proj_bwd_grouped_pair can run dW and dm of these sizes.
