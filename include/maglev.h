@@ -194,11 +194,7 @@ typedef enum {
  *   dgate_logits [4,H] fp32 ([2,H] with shared_kv_gates; out, overwritten);
  *     NULL when inject == 0.
  *   m_shift, w_mk, w_mv, dm_shift, dw_mk, dw_mv: if m_shift != NULL the call
- *     finishes with maglev_mem_project_bwd on dR_k, dR_v (modes WRITE and LAST),
- *     and the gate sums run beside that GEMM on a second stream the library
- *     owns (one per device, made by the first such call outside a stream
- *     capture); it is forked from and joined back to `stream` with events
- *     inside this call, so `stream` still orders everything the call writes.
+ *     finishes with maglev_mem_project_bwd on dR_k, dR_v (modes WRITE and LAST).
  *   workspace: maglev_swa_bwd_workspace_bytes(desc) bytes of scratch.
  * Errors: INVALID_ARG for a bad dR_mode, for m_shift != NULL in modes FIRST or
  * ADD, and for a NULL pointer the mode needs. */

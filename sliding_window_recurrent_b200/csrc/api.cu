@@ -175,44 +175,6 @@ maglev_status status_word(int** out, cudaStream_t s);
 
 int64_t spin_limit_of(int64_t v) { return v > 0 ? v : DEFAULT_SPIN_LIMIT; }
 
-// A second stream per device for a kernel that may run beside the caller's
-// stream inside one call: forked and joined with events, which CUDA graph
-// capture records as graph edges. Created by the first call that is not being
-// captured; a captured call before that runs everything on the caller's stream.
-struct SideStream {
-  cudaStream_t s = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
-};
-SideStream g_side[128];
-std::mutex g_side_mu;
-
-SideStream* side_stream(cudaStream_t caller) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) {
-    (void)cudaGetLastError();
-    return nullptr;
-  }
-  SideStream& ss = g_side[dev];
-  if (ss.s) return &ss;
-  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-  if (cudaStreamIsCapturing(caller, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) {
-    (void)cudaGetLastError();
-    return nullptr;
-  }
-  cudaStream_t st = nullptr;
-  cudaEvent_t f = nullptr, j = nullptr;
-  if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess ||
-      cudaEventCreateWithFlags(&f, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&j, cudaEventDisableTiming) != cudaSuccess) {
-    (void)cudaGetLastError();
-    return nullptr;
-  }
-  ss.fork = f;
-  ss.join = j;
-  ss.s = st;
-  return &ss;
-}
-
 maglev_status run_mem_project(const maglev_swa_desc* d, const void* m, const void* wk,
                               const void* wv, void* Rk, void* Rv, cudaStream_t st) {
   const int64_t M = (int64_t)d->B * d->T, D = (int64_t)d->H * d->hd, K = d->d_mem;
@@ -572,39 +534,13 @@ maglev_status maglev_inject_swa_bwd(const maglev_swa_desc* d, const void* k, con
                                    dR_acc_k, dR_acc_v, dR_mode, gpart, dq_acc, dq, s),
                 "unmix");
   if (d->inject) {
-    // The gate sums and the projection backward both read only what unmix wrote:
-    // with the projection's GEMM to follow, the sums run beside it on the side
-    // stream (40 small blocks next to the GEMM's one CTA per SM).
-    std::unique_lock<std::mutex> side_lock(g_side_mu);
-    SideStream* ss = m_shift ? side_stream(s) : nullptr;
-    if (!ss) side_lock.unlock();
-    cudaStream_t gs = s;
-    bool forked = false;
-    if (ss) {
-      if (cudaEventRecord(ss->fork, s) == cudaSuccess && cudaStreamWaitEvent(ss->s, ss->fork, 0) == cudaSuccess) {
-        forked = true;
-        gs = ss->s;
-      } else {
-        (void)cudaGetLastError();  // the sums then run on the caller's stream
-      }
-    }
-    cudaError_t ge;
-    {
-      ProfScope ps_("gate_reduce", 1, gs);
-      ge = launch_gate_reduce((int64_t)d->B * d->T, d->H, d->shared_kv_gates ? 1 : 0, gpart, gate_logits,
-                              dgate_logits, gs);
-    }
-    st = MAGLEV_OK;
-    if (ge == cudaSuccess && m_shift)
+    MAGLEV_LAUNCH(1, s, launch_gate_reduce((int64_t)d->B * d->T, d->H, d->shared_kv_gates ? 1 : 0, gpart,
+                                           gate_logits, dgate_logits, s),
+                  "gate_reduce");
+    if (m_shift) {
       st = run_mem_project_bwd(d, m_shift, w_mk, w_mv, dR_k, dR_v, dm_shift, dw_mk, dw_mv, s);
-    if (forked) {
-      // Joined on every path, so a captured graph never ends with the side branch open.
-      cudaError_t je = cudaEventRecord(ss->join, ss->s);
-      if (je == cudaSuccess) je = cudaStreamWaitEvent(s, ss->join, 0);
-      if (je != cudaSuccess && ge == cudaSuccess && st == MAGLEV_OK) return cuda_fail(je, "side stream join");
+      if (st != MAGLEV_OK) return st;
     }
-    if (ge != cudaSuccess) return cuda_fail(ge, "gate_reduce");
-    if (st != MAGLEV_OK) return st;
   }
   return MAGLEV_OK;
 }

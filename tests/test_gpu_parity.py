@@ -299,6 +299,58 @@ def test_mem_project_bwd_outputs(which):
     assert mg.maglev_device_status() == 0
 
 
+# --------------------------------------------------------------------------- projection in the call
+LAYER_OUTPUTS = ("out", "lse", "R_k", "R_v", "dq", "dk", "dv", "dR_k", "dR_v", "dgate", "dm_shift", "dw_mk",
+                 "dw_mv")
+
+
+def test_projection_in_call_matches_separate_calls_bitwise():
+    """The shared projection run inside the forward and backward calls (m_shift
+    given) against maglev_mem_project / maglev_mem_project_bwd called on their
+    own around calls without it: every output agrees bit for bit, eagerly on a
+    non-default caller stream and replayed from a CUDA graph captured from the
+    same calls. dq is reproducible here because W < 128: each query row takes
+    the contributions of at most two 128-key tiles, and two fp32 adds into the
+    zeroed accumulator give the same sum in either order."""
+    wl = wl_of("layer_bf16", B=2, T=300, H=3, hd=128, d=160, W=100, target="independent")
+    x = synth.layer_inputs(wl, 99)
+    B, T, H, hd, d, W = (wl[n] for n in ("B", "T", "H", "hd", "d", "W"))
+    q, k, v, gates = dev(x["q"]), dev(x["k"]), dev(x["v"]), dev(x["gates"])
+    m, wk, wv, dout = dev(x["m_shift"]), dev(x["w_mk"]), dev(x["w_mv"]), dev(x["dout"])
+
+    def layer():
+        return InjectedSWALayer(B, T, H, hd, d, W, dtype="bf16", rope_base=wl["rope_base"], eps=wl["eps"])
+
+    sep = layer()
+    mg.maglev_mem_project(sep.desc, m, wk, wv, sep.R_k, sep.R_v)
+    sep.forward(q, k, v, gates)
+    sep.backward(k, v, dout, gates)
+    mg.maglev_mem_project_bwd(sep.desc, m, wk, wv, sep.dR_k, sep.dR_v, sep.dm_shift, sep.dw_mk, sep.dw_mv)
+    torch.cuda.synchronize()
+
+    eager = layer()
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(st):
+        eager.forward(q, k, v, gates, m, wk, wv, stream=st)
+        eager.backward(k, v, dout, gates, m, wk, wv, stream=st)
+    st.synchronize()
+    for n in LAYER_OUTPUTS:
+        assert torch.equal(getattr(eager, n), getattr(sep, n)), n
+
+    graphed = layer()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        graphed.forward(q, k, v, gates, m, wk, wv)
+        graphed.backward(k, v, dout, gates, m, wk, wv)
+    g.replay()
+    torch.cuda.synchronize()
+    for n in LAYER_OUTPUTS:
+        assert torch.equal(getattr(graphed, n), getattr(sep, n)), n
+    del g
+    assert mg.maglev_device_status() == 0
+
+
 # --------------------------------------------------------------------------- consistency loss
 @pytest.mark.parametrize("dtype,rows,d", [("f32", 256, 128), ("bf16", 8192, 1280), ("bf16", 3, 17)])
 def test_consistency_loss(dtype, rows, d):
